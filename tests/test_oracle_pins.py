@@ -1,0 +1,296 @@
+"""Pins of the fp64 oracle to facts fixed outside the oracle itself.
+
+Each check compares the oracle with something it does not compute: hand-derived
+values (tests/golden/hand_cases.txt), a library FFT (numpy.fft.rfft / irfft), closed
+forms (orthonormality, Parseval, exact reconstruction at k = M, lossless integer
+frequencies) and brute force on tiny inputs. The mutation tests at the end plant
+plausible mistakes in copies of the oracle's basis and check that a pin catches each.
+"""
+import itertools
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import fourier_oracle as fo
+
+TOL = 1e-12
+
+
+# ----------------------------------------------------------------------------- checks
+# Written as functions of a basis generator so the mutation tests can reuse them.
+
+def check_orthonormal(basis_fn, M, k):
+    phi = basis_fn(M, k)
+    return np.abs(phi.T @ phi - np.eye(k)).max()
+
+
+def check_rfft_bins(basis_fn, M, k, rng):
+    """C = Phi^T x against numpy's rfft R: C0 = R0/sqrt(M), C_{2f-1} = sqrt(2/M) Re R_f,
+    C_{2f} = -sqrt(2/M) Im R_f (Nyquist: C = R_{M/2}/sqrt(M))."""
+    x = rng.standard_normal(M)
+    C = basis_fn(M, k).T @ x
+    R = np.fft.rfft(x)
+    ref = np.empty(k)
+    for j in range(k):
+        f = (j + 1) // 2
+        if j == 0:
+            ref[j] = R[0].real / np.sqrt(M)
+        elif 2 * f == M:
+            ref[j] = R[f].real / np.sqrt(M)
+        elif j % 2 == 1:
+            ref[j] = np.sqrt(2.0 / M) * R[f].real
+        else:
+            ref[j] = -np.sqrt(2.0 / M) * R[f].imag
+    return np.abs(C - ref).max() / max(1.0, np.abs(ref).max())
+
+
+def check_truncated_irfft(basis_fn, M, kb, rng):
+    """Skill page Step 4: keep the first kb rfft bins, zero the rest, irfft(n=M).
+    Must equal Phi Phi^T x with k = 2 kb - 1 real functions (kb < M/2)."""
+    x = rng.standard_normal(M)
+    R = np.fft.rfft(x)
+    R[kb:] = 0
+    ref = np.fft.irfft(R, n=M)
+    phi = basis_fn(M, 2 * kb - 1)
+    return np.abs(phi @ (phi.T @ x) - ref).max()
+
+
+# ----------------------------------------------------------------------------- partition
+
+def test_partition_brute_force():
+    for L, S, R in itertools.product(range(0, 12), range(0, 6), range(0, 6)):
+        s, r, m = fo.partition(L, S, R)
+        assert s + m + r == L and min(s, r, m) >= 0
+        # brute force: label every token, each exactly once
+        labels = ["sink" if t < s else ("recent" if t >= L - r else "mid") for t in range(L)]
+        if L > S + R:  # the skill page compresses only when the sequence is longer than S+R
+            assert (s, r, m) == (S, R, L - S - R)
+            assert labels.count("mid") == L - S - R
+        else:
+            assert m == 0 and s == min(S, L)
+
+
+def test_split_dims_brute_force():
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        mask = (rng.random(128) < rng.random()).astype(np.uint8)
+        cd, ed = fo.split_dims(mask)
+        assert list(cd) == [d for d in range(128) if mask[d]]
+        assert list(ed) == [d for d in range(128) if not mask[d]]
+
+
+# ----------------------------------------------------------------------------- basis
+
+def test_basis_hand_values(hand_cases):
+    for M in (4, 3):
+        phi = fo.basis(M, M)
+        for j in range(M):
+            ref = np.array(hand_cases[f"basis_M{M}_j{j}"])
+            assert np.abs(phi[:, j] - ref).max() < 1e-15
+
+
+@pytest.mark.parametrize("M,k", [(1, 1), (2, 2), (3, 3), (4, 4), (7, 5), (8, 8), (8, 7),
+                                 (64, 63), (127, 127), (128, 128), (1952, 63), (4099, 1023),
+                                 (32672, 255)])
+def test_basis_orthonormal(M, k):
+    assert check_orthonormal(fo.basis, M, k) < TOL
+
+
+def test_basis_orthonormal_large_M_compensated():
+    """M = 128992 (the 128K-context middle span): Gram entries by exact fsum."""
+    import math
+    M, k = 128992, 1023
+    rows = fo.basis(M, 8, 0, M)        # first 8 functions, all tokens
+    last = fo.basis(M, k, 0, M)[:, -4:]  # and the last 4 (highest frequency)
+    cols = np.concatenate([rows, last], axis=1)
+    for a in range(cols.shape[1]):
+        for b in range(a, cols.shape[1]):
+            g = math.fsum(cols[:, a] * cols[:, b])
+            assert abs(g - (1.0 if a == b else 0.0)) < TOL
+
+
+def test_basis_chunk_rows_match():
+    M, k = 1000, 31
+    full = fo.basis(M, k)
+    part = fo.basis(M, k, 300, 700)
+    assert np.array_equal(full[300:700], part)
+
+
+def test_basis_rejects_bad_k():
+    with pytest.raises(ValueError):
+        fo.basis(4, 5)
+    with pytest.raises(ValueError):
+        fo.basis(4, 0)
+
+
+@pytest.mark.parametrize("M,k", [(16, 16), (17, 17), (16, 9), (1952, 63), (2047, 255),
+                                 (4096, 4096)])
+def test_rfft_bins(M, k):
+    assert check_rfft_bins(fo.basis, M, k, np.random.default_rng(M + k)) < TOL
+
+
+@pytest.mark.parametrize("M,kb", [(16, 3), (17, 8), (1952, 32), (2048, 128)])
+def test_truncated_irfft_equals_projection(M, kb):
+    assert check_truncated_irfft(fo.basis, M, kb, np.random.default_rng(M)) < TOL
+
+
+# ----------------------------------------------------------------------------- compress
+
+def test_compress_hand_example(hand_cases):
+    x = np.array(hand_cases["compress_x"])[:, None]
+    mask = np.ones(1)
+    h4 = fo.compress(x, mask, 0, 0, 4)
+    assert np.abs(h4.C[:, 0] - hand_cases["compress_C_k4"]).max() < 1e-15
+    assert np.abs(fo.reconstruct(h4)[:, 0] - hand_cases["recon_k4"]).max() < 1e-14
+    h3 = fo.compress(x, mask, 0, 0, 3)
+    assert np.abs(fo.reconstruct(h3)[:, 0] - hand_cases["recon_k3"]).max() < 1e-14
+
+
+@pytest.mark.parametrize("M", [1, 2, 5, 64, 127, 128, 255])
+def test_k_equals_M_reconstructs_exactly(M):
+    rng = np.random.default_rng(M)
+    S, R, D = 3, 2, 128
+    X = rng.standard_normal((S + M + R, D))
+    mask = (rng.random(D) < 0.75).astype(np.uint8)
+    h = fo.compress(X, mask, S, R, M)
+    assert np.abs(fo.reconstruct(h) - X).max() < TOL * max(1.0, np.abs(X).max()) * 10
+
+
+@pytest.mark.parametrize("M,k", [(500, 63), (1952, 63), (1000, 1000), (999, 2)])
+def test_parseval(M, k):
+    rng = np.random.default_rng(k)
+    X = rng.standard_normal((M, 128))
+    h = fo.compress(X, np.ones(128), 0, 0, k)
+    resid = X - fo.reconstruct(h)
+    lhs = (X ** 2).sum(0)
+    rhs = (h.C ** 2).sum(0) + (resid ** 2).sum(0)
+    assert np.abs(lhs - rhs).max() / lhs.max() < TOL
+
+
+def test_lossless_integer_frequencies():
+    """A sum of cosines with integer frequency f <= floor(k/2) lies in the span."""
+    M, k = 1952, 63
+    rng = np.random.default_rng(1)
+    t = np.arange(M)
+    X = np.zeros((M, 4))
+    for col in range(4):
+        for f in rng.integers(0, k // 2 + 1, size=3):
+            X[:, col] += rng.standard_normal() * np.cos(2 * np.pi * f * t / M + rng.uniform(0, 2 * np.pi))
+    h = fo.compress(X, np.ones(4), 0, 0, k)
+    assert np.abs(fo.reconstruct(h) - X).max() < 1e-11
+
+
+def test_sink_recent_retained_are_exact_copies():
+    rng = np.random.default_rng(2)
+    L, S, R, D = 300, 32, 64, 128
+    X = rng.standard_normal((L, D))
+    mask = (rng.random(D) < 0.75).astype(np.uint8)
+    h = fo.compress(X, mask, S, R, 31)
+    Xt = fo.reconstruct(h)
+    cd, ed = fo.split_dims(mask)
+    assert np.array_equal(Xt[:S], X[:S]) and np.array_equal(Xt[L - R:], X[L - R:])
+    assert np.array_equal(Xt[S:L - R][:, ed], X[S:L - R][:, ed])
+    assert np.array_equal(h.E, X[S:L - R][:, ed])
+    # compressed dims changed (k < M), so the projection really ran on them
+    assert np.abs(Xt[S:L - R][:, cd] - X[S:L - R][:, cd]).max() > 1e-3
+
+
+# ----------------------------------------------------------------------------- attention
+
+def test_attention_hand_case(hand_cases):
+    q = np.array([hand_cases["attn_q"]])
+    K = np.array([hand_cases["attn_K0"], hand_cases["attn_K1"]])
+    V = np.array([hand_cases["attn_V0"], hand_cases["attn_V1"]])
+    out = fo.attention(q, K, V, 1.0)
+    assert np.abs(out[0] - hand_cases["attn_out"]).max() < 1e-14
+
+
+def test_attention_matches_torch_softmax():
+    rng = np.random.default_rng(3)
+    q, K, V = rng.standard_normal((4, 128)), rng.standard_normal((200, 128)), rng.standard_normal((200, 128))
+    sc = 1 / np.sqrt(128)
+    p = torch.softmax(torch.from_numpy(q) @ torch.from_numpy(K).T * sc, dim=-1)
+    ref = (p @ torch.from_numpy(V)).numpy()
+    assert np.abs(fo.attention(q, K, V, sc) - ref).max() < 1e-13
+
+
+@pytest.mark.parametrize("case", ["no_dims", "no_middle"])
+def test_nothing_compressed_is_plain_attention(case):
+    rng = np.random.default_rng(4)
+    L, D = 400, 128
+    K, V, q = rng.standard_normal((L, D)), rng.standard_normal((L, D)), rng.standard_normal((4, D))
+    if case == "no_dims":
+        mask, S, R = np.zeros(D), 32, 64
+    else:
+        mask, S, R = np.ones(D), 300, 200
+    hk, hv = fo.compress(K, mask, S, R, 15), fo.compress(V, mask, S, R, 15)
+    ref = fo.attention(q, K, V, 1 / np.sqrt(D))
+    assert np.abs(fo.decode(q, hk, hv) - ref).max() < 1e-13
+
+
+def test_coefficient_domain_identity():
+    """Scores and values in the coefficient domain equal those on the reconstruction:
+    q . X^_t = q_e . E_t + (Phi (C_K q_c))_t and p^T X^ = (Phi^T p)^T C_V."""
+    rng = np.random.default_rng(6)
+    L, S, R, D, k = 700, 32, 64, 128, 63
+    mask = (rng.random(D) < 0.75).astype(np.uint8)
+    K, V, q = rng.standard_normal((L, D)), rng.standard_normal((L, D)), rng.standard_normal(D)
+    hk, hv = fo.compress(K, mask, S, R, k), fo.compress(V, mask, S, R, k)
+    Kt, Vt = fo.reconstruct(hk), fo.reconstruct(hv)
+    phi = fo.basis(hk.M, k)
+    cd, ed = hk.cd, hk.ed
+    s_ref = Kt[S:L - R] @ q
+    s_coef = hk.E @ q[ed] + phi @ (hk.C @ q[cd])
+    assert np.abs(s_ref - s_coef).max() < 1e-11
+    p = rng.random(hk.M)
+    v_ref = p @ Vt[S:L - R]
+    assert np.abs(v_ref[cd] - (phi.T @ p) @ hv.C).max() < 1e-11
+    assert np.abs(v_ref[ed] - p @ hv.E).max() < 1e-11
+
+
+def test_gqa_head_grouping_matches_per_head_loop():
+    rng = np.random.default_rng(7)
+    L, D, G = 300, 128, 4
+    K, V = rng.standard_normal((L, D)), rng.standard_normal((L, D))
+    q = rng.standard_normal((G, D))
+    mask = (rng.random(D) < 0.5).astype(np.uint8)
+    hk, hv = fo.compress(K, mask, 8, 16, 41), fo.compress(V, mask, 8, 16, 41)
+    joint = fo.decode(q, hk, hv)
+    for h in range(G):
+        assert np.abs(joint[h] - fo.decode(q[h:h + 1], hk, hv)[0]).max() < 1e-14
+
+
+# ----------------------------------------------------------------------------- mutations
+# Each mutant is a plausible slip in writing the basis; some pin above must reject it.
+
+def _mutant(kind):
+    def fn(M, k, t0=0, t1=None):
+        phi = fo.basis(M, k, t0, t1).copy()
+        t = np.arange(t0, M if t1 is None else t1)
+        if kind == "sin_sign" and k > 2:
+            phi[:, 2] *= -1
+        elif kind == "swap_cos_sin" and k > 2:
+            phi[:, [1, 2]] = phi[:, [2, 1]]
+        elif kind == "norm_dc_like" and k > 1:
+            phi[:, 1] *= np.sqrt(0.5)
+        elif kind == "freq_off_by_one" and k > 1:
+            phi[:, 1] = np.sqrt(2.0 / M) * np.cos(2 * np.pi * 2 * t / M)
+        elif kind == "angle_no_reduce":      # phase computed in fp32 without reduction
+            f = (np.arange(k) + 1) // 2
+            ang = (np.float32(2 * np.pi / M) * (f[None, :] * t[:, None]).astype(np.float32)).astype(np.float64)
+            base = np.where((np.arange(k) % 2 == 0) & (np.arange(k) > 0), np.sin(ang), np.cos(ang))
+            phi = base * np.where((f == 0) | (2 * f == M), 1 / np.sqrt(M), np.sqrt(2.0 / M))
+        return phi
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["sin_sign", "swap_cos_sin", "norm_dc_like", "freq_off_by_one",
+                                  "angle_no_reduce"])
+def test_pins_reject_planted_mistakes(kind):
+    fn = _mutant(kind)
+    rng = np.random.default_rng(0)
+    caught = (check_orthonormal(fn, 4099, 255) > TOL
+              or check_rfft_bins(fn, 4099, 255, rng) > TOL
+              or check_truncated_irfft(fn, 4099, 100, rng) > TOL)
+    assert caught, kind
