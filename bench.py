@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the Fourier-approximated KV cache hot path on B200.
+
+One step = one pass of the whole path over one batch of the workload: build the basis
+table, fa_compress (sink/recent copy, retained-dim packing and the tcgen05 projection of
+K and V) and one fa_decode step (prologue, split-L main kernel, combine). Default
+workload: LLaMA-2-7B attention shape, batch 8, 32 MHA heads, L = 32768, S = 32, R = 64,
+k = 255, 96 of 128 dims compressed per head (seeded random masks), synthetic caches.
+
+Prints ONE JSON line (rank 0). ``value`` is microseconds per step (lower is better),
+timed with CUDA events on the launching stream over exactly --steps steps after
+--warmup steps, max over ranks. With --gpus N each rank runs its own batch (weak
+scaling, no collective in the data path).
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded sample of the
+same workload (whole (batch, KV head) pairs, scaled to the full step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fa_decode μs/step & HBM GB/s; fa_compress TFLOP/s; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama2_7b_mha_b8_L32768_k255")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    return ap.parse_args()
+
+
+def workload_by_name(name):
+    import workloads as wl
+    for w in wl.CONFIGS:
+        if w.name == name:
+            return w
+    raise SystemExit(f"unknown workload {name}; known: {[w.name for w in wl.CONFIGS]}")
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+
+def work_model(w, plan):
+    """Algorithmic bytes / flops per step, from the plan's per-head dim split."""
+    B, Hkv, G, D = w.B, w.Hkv, w.G, 128
+    S, R, M, k = plan.S, plan.R, plan.M, w.k
+    dcs = [plan.dc[g] for g in range(Hkv)]
+    des = [plan.de[g] for g in range(Hkv)]
+    # compress: read the middle rows once, write C and E, copy the sink/recent rows (K and V)
+    c_bytes = 2 * 2 * B * sum(M * D + k * dc + M * de + 2 * (S + R) * D for dc, de in zip(dcs, des))
+    c_flops = 2 * 2 * B * sum(k * M * dc for dc in dcs)
+    # decode: read F, E and C of K and V, the queries, write the outputs
+    d_bytes = 2 * 2 * B * sum((S + R) * D + M * de + k * dc for dc, de in zip(dcs, des)) \
+        + 2 * 2 * B * w.Hq * D
+    d_flops = B * G * sum(4 * D * (S + R) + 4 * de * M + 4 * k * dc + 4 * M * k
+                          for dc, de in zip(dcs, des))
+    return dict(compress_bytes=c_bytes, compress_flops=c_flops, decode_bytes=d_bytes,
+                decode_flops=d_flops)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            pk = json.load(fh)
+        return pk, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def compress_traffic():
+    """Measured DRAM traffic of the compress kernel (profiles/), if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    src = os.path.join(ROOT, "fourier_basis_attention_b200", "csrc", rec.get("source", ""))
+    if not os.path.exists(src):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return rec if digest == rec.get("source_sha256_16") else None
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.out = open("/tmp/fa_clocks_%d.csv" % os.getpid(), "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_index, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.out.name) as fh:
+            for line in fh:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), sm_max=float(parts[2]),
+                                     power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                     hw=parts[5], hw_thermal=parts[6], sw_thermal=parts[7],
+                                     sw_power=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.out.name)
+        return rows
+
+
+def summarize_clocks(rows):
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    loaded = [r for r in rows if r["power"] > 200.0] or rows
+    reasons = set()
+    for r in loaded:
+        for key, name in (("hw", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                          ("sw_thermal", "sw_thermal_slowdown"), ("sw_power", "sw_power_cap")):
+            if r[key].lower().startswith("active"):
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(r["sm"] for r in loaded),
+            "sm_max_mhz": max(r["sm_max"] for r in rows), "reasons": sorted(reasons),
+            "samples": len(loaded)}
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, K_pairs, V_pairs, q_pairs, masks):
+    """Time the fp64 oracle on whole (batch, KV head) pairs; returns seconds per pair."""
+    from oracle import fourier_oracle as fo
+    t0 = time.perf_counter()
+    for (Kh, Vh, qh, m) in zip(K_pairs, V_pairs, q_pairs, masks):
+        hk = fo.compress(Kh, m, w.S, w.R, w.k)
+        hv = fo.compress(Vh, m, w.S, w.R, w.k)
+        fo.decode(qh, hk, hv)
+    return (time.perf_counter() - t0) / len(K_pairs)
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info), default=1)
+        return int(n)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def host_pairs(w, n_pairs, seed_shift=0):
+    """A few (batch, KV head) pairs of the workload drawn on the host (fp64 arrays)."""
+    import workloads as wl
+    ws = wl.shrink(w, B=1, seed=w.seed + seed_shift)
+    K = wl.kv_cache(ws, "K")[0]
+    V = wl.kv_cache(ws, "V")[0]
+    q = wl.queries(ws)[0]
+    mask = wl.dim_mask(w)
+    out = []
+    for g in range(min(n_pairs, w.Hkv)):
+        out.append((K[g].double().numpy(), V[g].double().numpy(),
+                    q[g * w.G:(g + 1) * w.G].double().numpy(), mask[g]))
+    return out
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workload_by_name(args.workload)
+    pairs = host_pairs(w, 1)
+    n_units = w.B * w.Hkv
+    for _ in range(args.warmup):
+        oracle_sample(w, *zip(*pairs))
+    times = [oracle_sample(w, *zip(*pairs)) for _ in range(args.steps)]
+    us = statistics.mean(times) * n_units * 1e6
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": us, "unit": "us/step",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.L, "k": w.k,
+                   "S": w.S, "R": w.R, "parallelism": "host"},
+        "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
+                         "sample": f"1 of {n_units} (batch, KV head) pairs per step, fp64 "
+                                   f"compress K+V + decode, scaled x{n_units}"},
+        "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_ours(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    base = workload_by_name(args.workload)
+    w = wl.shrink(base, seed=base.seed + 1000 * rank) if rank else base
+    mask = wl.dim_mask(base)
+    dev = torch.device("cuda", local)
+    K = wl.kv_cache(w, "K", device=dev)
+    V = wl.kv_cache(w, "V", device=dev)
+    q = wl.queries(w, device=dev)
+    plan = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    cache = fa.Cache(plan, device=dev)
+    phiT = torch.empty(w.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_size(plan), dtype=torch.uint8, device=dev)
+    out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+        fa.fa_compress(plan, K, V, phiT, cache, stream)
+        fa.fa_decode(plan, q, cache, out, ws, 0, stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    fa.fa_device_status(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local if world > 1 else 0]
+    sampler = ClockSampler(gpu_index)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        e = ev[i]
+        e[0].record(stream)
+        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+        e[1].record(stream)
+        fa.fa_compress(plan, K, V, phiT, cache, stream)
+        e[2].record(stream)
+        fa.fa_decode(plan, q, cache, out, ws, 0, stream)
+        e[3].record(stream)
+    t_end.record(stream)
+    barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    rows = sampler.stop()
+    clock_note = "sampled during the timed region"
+    if len([r for r in rows if r["power"] > 200.0]) < 3:
+        # timed region too short for the 100 ms sampler: sample the same step for ~1 s more
+        sampler2 = ClockSampler(gpu_index)
+        sampler2.start()
+        time.sleep(0.3)
+        t_end_probe = time.time() + 1.2
+        while time.time() < t_end_probe:
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize(dev)
+        rows = rows + sampler2.stop()
+        clock_note = "timed region plus ~1.2 s more of the same step (region shorter than the sampler period)"
+    fa.fa_device_status(stream)
+    t_basis = [e[0].elapsed_time(e[1]) for e in ev]
+    t_comp = [e[1].elapsed_time(e[2]) for e in ev]
+    t_dec = [e[2].elapsed_time(e[3]) for e in ev]
+    ms_step = total_ms / args.steps
+    comp_ms = statistics.mean(t_comp)
+    dec_ms = statistics.mean(t_dec)
+    basis_ms = statistics.mean(t_basis)
+    if world > 1:
+        t = torch.tensor([ms_step, comp_ms, dec_ms, basis_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, comp_ms, dec_ms, basis_ms = t.tolist()
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    e2e_us = None
+    h2d = d2h = 0
+    if args.e2e_steps > 0:
+        Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+        Vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+        qh = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+        oh = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        Kh.copy_(K)
+        Vh.copy_(V)
+        qh.copy_(q)
+        Kd, Vd, qd = torch.empty_like(K), torch.empty_like(V), torch.empty_like(q)
+        del K, V
+        torch.cuda.synchronize(dev)
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            Kd.copy_(Kh, non_blocking=True)
+            Vd.copy_(Vh, non_blocking=True)
+            qd.copy_(qh, non_blocking=True)
+            fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+            fa.fa_compress(plan, Kd, Vd, phiT, cache, stream)
+            fa.fa_decode(plan, qd, cache, out, ws, 0, stream)
+            oh.copy_(out, non_blocking=True)
+        b.record(stream)
+        barrier()
+        e2e_ms = a.elapsed_time(b) / args.e2e_steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = t.item()
+        e2e_us = e2e_ms * 1e3
+        h2d = Kh.numel() * 2 + Vh.numel() * 2 + qh.numel() * 2
+        d2h = oh.numel() * 2
+
+    # ---------------------------------------------------------------- roofline
+    wm = work_model(w, plan)
+    peaks, peak_src = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    ridge = tc * 1e12 / (hbm * 1e9)
+    c_ai = wm["compress_flops"] / wm["compress_bytes"]
+    c_gbs = wm["compress_bytes"] / (comp_ms * 1e-3) / 1e9
+    c_tflops = wm["compress_flops"] / (comp_ms * 1e-3) / 1e12
+    d_gbs = wm["decode_bytes"] / (dec_ms * 1e-3) / 1e9
+    d_tflops = wm["decode_flops"] / (dec_ms * 1e-3) / 1e12
+    traffic = compress_traffic()
+    if c_ai < ridge:
+        roof = {"bound": "hbm", "achieved": c_gbs, "peak": hbm, "unit": "GB/s", "frac": c_gbs / hbm}
+    else:
+        roof = {"bound": "tensor", "achieved": c_tflops, "peak": tc, "unit": "TFLOP/s",
+                "frac": c_tflops / tc}
+    roof.update({"kernel": "fa_compress (compress_kernel + copy_sink_recent_kernel)",
+                 "traffic": (traffic["bytes_per_launch_scaled"] if traffic else None),
+                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)"
+                 if peak_src == "measured" else "fallback"})
+
+    line = {
+        "metric": METRIC, "value": ms_step * 1e3, "unit": "us/step", "n_gpus": world,
+        "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L,
+                   "Hq": w.Hq, "Hkv": w.Hkv, "k": w.k, "S": w.S, "R": w.R,
+                   "dims_compressed_per_head": int(plan.dc[0]), "parallelism": f"replica x{world}",
+                   "l2": "inputs larger than L2 (K+V %.2f GB, E %.2f GB per step)" % (
+                       2 * K_bytes(w) / 1e9, 2 * plan.e_elems * 2 / 1e9)},
+        "components": {
+            "fa_build_basis": {"us": basis_ms * 1e3},
+            "fa_compress": {"us": comp_ms * 1e3, "tflops": c_tflops, "hbm_gbs": c_gbs,
+                            "arith_intensity": c_ai, "algorithmic_bytes": wm["compress_bytes"],
+                            "algorithmic_flops": wm["compress_flops"],
+                            "frac_hbm": c_gbs / hbm, "frac_tensor": c_tflops / tc},
+            "fa_decode": {"us": dec_ms * 1e3, "hbm_gbs": d_gbs, "frac_hbm": d_gbs / hbm,
+                          "tflops_fp32": d_tflops, "algorithmic_bytes": wm["decode_bytes"],
+                          "algorithmic_flops": wm["decode_flops"]},
+        },
+        "roofline": roof,
+        "clocks": {**summarize_clocks(rows), "note": clock_note},
+        "gpu_launches": 6 * args.steps,
+        "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        pairs = host_pairs(base, 2)
+        n_units = base.B * base.Hkv
+        per_pair = oracle_sample(base, *zip(*pairs))
+        line["cpu_baseline"] = {
+            "value": per_pair * n_units * 1e6, "unit": "us/step", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"2 of {n_units} (batch, KV head) pairs (fp64 compress K+V + decode), "
+                      f"scaled x{n_units / 2:g}"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+
+
+def K_bytes(w):
+    return w.B * w.Hkv * w.L * 128 * 2
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,215 @@
+// fa_abi.cu -- the extern "C" entry points: argument validation, plan derivation,
+// launches, error reporting. See include/fourier_attention.h for the contract.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "fa_host.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(FA_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int round8(int x) { return (x + 7) & ~7; }
+
+int check_ptr(const void* p, const char* name, bool required) {
+  if (!p) return required ? fail(FA_ERR_INVALID, "%s is NULL", name) : FA_OK;
+  if (!aligned16(p)) return fail(FA_ERR_INVALID, "%s is not 16-byte aligned", name);
+  return FA_OK;
+}
+
+// Re-checks the fields kernels rely on, so a plan edited by hand cannot drive a launch
+// out of bounds.
+int check_plan(const fa_plan* plan) {
+  if (!plan) return fail(FA_ERR_INVALID, "plan is NULL");
+  const fa_shape& s = plan->shape;
+  if (s.D != FA_HEAD_DIM) return fail(FA_ERR_UNSUPPORTED, "head dim %d != 128", s.D);
+  if (s.Hkv < 1 || s.Hkv > FA_MAX_KV_HEADS || s.Hq < 1 || s.Hq % s.Hkv != 0 || s.B < 1 ||
+      s.L < 1)
+    return fail(FA_ERR_INVALID, "plan shape is inconsistent");
+  if (plan->S < 0 || plan->R < 0 || plan->M < 0 || plan->S + plan->M + plan->R != s.L)
+    return fail(FA_ERR_INVALID, "plan token partition is inconsistent");
+  if (plan->G != s.Hq / s.Hkv) return fail(FA_ERR_INVALID, "plan G is inconsistent");
+  long long ce = 0, ee = 0;
+  for (int g = 0; g < s.Hkv; ++g) {
+    if (plan->dc[g] < 0 || plan->dc[g] > FA_HEAD_DIM || plan->de[g] != FA_HEAD_DIM - plan->dc[g] ||
+        plan->dc_ld[g] != round8(plan->dc[g]) || plan->de_ld[g] != round8(plan->de[g]) ||
+        plan->c_off[g] != ce || plan->e_off[g] != ee)
+      return fail(FA_ERR_INVALID, "plan dims of KV head %d are inconsistent", g);
+    bool seen[FA_HEAD_DIM] = {false};
+    for (int i = 0; i < FA_HEAD_DIM; ++i) {
+      const int d = plan->perm[g][i];
+      if (d >= FA_HEAD_DIM || seen[d])
+        return fail(FA_ERR_INVALID, "plan perm of KV head %d is not a permutation", g);
+      seen[d] = true;
+    }
+    ce += (long long)plan->kk * plan->dc_ld[g];
+    ee += (long long)plan->M * plan->de_ld[g];
+  }
+  if (plan->c_batch != ce || plan->e_batch != ee)
+    return fail(FA_ERR_INVALID, "plan batch strides are inconsistent");
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) {
+  if (!shape || !dim_mask || !plan) return fail(FA_ERR_INVALID, "NULL argument");
+  const fa_shape s = *shape;
+  if (s.D != FA_HEAD_DIM) return fail(FA_ERR_UNSUPPORTED, "head dim %d != 128", s.D);
+  if (s.B < 1 || s.Hq < 1 || s.Hkv < 1 || s.L < 1 || s.S < 0 || s.R < 0 || s.k < 1)
+    return fail(FA_ERR_INVALID, "shape fields out of range (B=%d Hq=%d Hkv=%d L=%d S=%d R=%d k=%d)",
+                s.B, s.Hq, s.Hkv, s.L, s.S, s.R, s.k);
+  if (s.Hkv > FA_MAX_KV_HEADS)
+    return fail(FA_ERR_UNSUPPORTED, "Hkv=%d exceeds %d", s.Hkv, FA_MAX_KV_HEADS);
+  if (s.Hq % s.Hkv != 0) return fail(FA_ERR_INVALID, "Hq=%d is not a multiple of Hkv=%d", s.Hq, s.Hkv);
+  memset(plan, 0, sizeof(*plan));
+  plan->shape = s;
+  plan->S = s.S < s.L ? s.S : s.L;
+  plan->R = s.R < s.L - plan->S ? s.R : s.L - plan->S;
+  plan->M = s.L - plan->S - plan->R;
+  plan->kk = plan->M > 0 ? s.k : 0;
+  plan->G = s.Hq / s.Hkv;
+  plan->phi_ld = round8(plan->M > 8 ? plan->M : 8);
+  bool any_dc = false;
+  long long ce = 0, ee = 0;
+  for (int g = 0; g < s.Hkv; ++g) {
+    int n = 0;
+    for (int d = 0; d < FA_HEAD_DIM; ++d)
+      if (dim_mask[g * FA_HEAD_DIM + d]) plan->perm[g][n++] = (uint8_t)d;
+    plan->dc[g] = n;
+    for (int d = 0; d < FA_HEAD_DIM; ++d)
+      if (!dim_mask[g * FA_HEAD_DIM + d]) plan->perm[g][n++] = (uint8_t)d;
+    plan->de[g] = FA_HEAD_DIM - plan->dc[g];
+    plan->dc_ld[g] = round8(plan->dc[g]);
+    plan->de_ld[g] = round8(plan->de[g]);
+    plan->c_off[g] = ce;
+    plan->e_off[g] = ee;
+    ce += (long long)plan->kk * plan->dc_ld[g];
+    ee += (long long)plan->M * plan->de_ld[g];
+    any_dc = any_dc || plan->dc[g] > 0;
+  }
+  if (plan->M > 0 && any_dc && s.k > plan->M)
+    return fail(FA_ERR_UNSUPPORTED, "k=%d exceeds the middle span M=%d", s.k, plan->M);
+  plan->c_batch = ce;
+  plan->e_batch = ee;
+  plan->f_elems = (long long)s.B * s.Hkv * (plan->S + plan->R) * FA_HEAD_DIM;
+  plan->e_elems = (long long)s.B * ee;
+  plan->c_elems = (long long)s.B * ce;
+  return FA_OK;
+}
+
+int fa_build_basis(int32_t M, int32_t k, int32_t dtype, void* phiT, int64_t ld, void* stream) {
+  if (M < 1 || k < 1 || k > M) return fail(FA_ERR_INVALID, "need 1 <= k <= M (k=%d, M=%d)", k, M);
+  if (dtype != FA_BF16 && dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
+  if (ld < M || ld % 8 != 0) return fail(FA_ERR_INVALID, "ld=%lld must be >= M and a multiple of 8", (long long)ld);
+  if (int r = check_ptr(phiT, "phiT", true)) return r;
+  int dev = 0, sms = 148;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_build_basis: device query");
+  e = fa::launch_build_basis(M, k, ld, dtype, phiT, static_cast<cudaStream_t>(stream), sms);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_build_basis: launch");
+  return FA_OK;
+}
+
+int fa_compress(const fa_plan* plan, const void* K, const void* V, const void* phiT,
+                const fa_cache* cache, void* stream) {
+  if (int r = check_plan(plan)) return r;
+  if (!cache) return fail(FA_ERR_INVALID, "cache is NULL");
+  if (int r = check_ptr(K, "K", true)) return r;
+  if (int r = check_ptr(V, "V", true)) return r;
+  const bool mid = plan->M > 0;
+  if (int r = check_ptr(phiT, "phiT", mid)) return r;
+  if (int r = check_ptr(cache->F_K, "cache->F_K", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->F_V, "cache->F_V", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_K, "cache->E_K", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_V, "cache->E_V", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_K, "cache->C_K", plan->c_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_V, "cache->C_V", plan->c_elems > 0)) return r;
+  const char* why = nullptr;
+  cudaError_t e = fa::launch_compress(plan, K, V, phiT, cache, static_cast<cudaStream_t>(stream), &why);
+  if (e != cudaSuccess) {
+    if (why) return fail(FA_ERR_CUDA, "fa_compress: %s", why);
+    return cuda_fail(e, "fa_compress: launch");
+  }
+  return FA_OK;
+}
+
+static int decode_checks(const fa_plan* plan) {
+  if (int r = check_plan(plan)) return r;
+  const int G = plan->G;
+  if (G != 1 && G != 2 && G != 4 && G != 8)
+    return fail(FA_ERR_UNSUPPORTED, "fa_decode supports Hq/Hkv in {1, 2, 4, 8}, got %d", G);
+  if (plan->M > 0 && plan->shape.k > FA_MAX_K_DECODE)
+    return fail(FA_ERR_UNSUPPORTED, "fa_decode supports k <= %d, got %d", FA_MAX_K_DECODE, plan->shape.k);
+  if (plan->M >= (1 << 21)) return fail(FA_ERR_UNSUPPORTED, "fa_decode supports M < 2^21");
+  return FA_OK;
+}
+
+size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits) {
+  if (decode_checks(plan) != FA_OK) return 0;
+  fa::DecodeConfig c;
+  if (fa::decode_configure(plan, num_splits, &c) != cudaSuccess) return 0;
+  return c.qw_bytes + c.rec_bytes;
+}
+
+int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
+              void* workspace, size_t workspace_bytes, int32_t num_splits, void* stream) {
+  if (int r = decode_checks(plan)) return r;
+  if (!cache) return fail(FA_ERR_INVALID, "cache is NULL");
+  if (int r = check_ptr(q, "q", true)) return r;
+  if (int r = check_ptr(out, "out", true)) return r;
+  if (int r = check_ptr(cache->F_K, "cache->F_K", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->F_V, "cache->F_V", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_K, "cache->E_K", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_V, "cache->E_V", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_K, "cache->C_K", plan->c_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_V, "cache->C_V", plan->c_elems > 0)) return r;
+  if (int r = check_ptr(workspace, "workspace", true)) return r;
+  fa::DecodeConfig c;
+  cudaError_t e = fa::decode_configure(plan, num_splits, &c);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_decode: configure");
+  if (workspace_bytes < c.qw_bytes + c.rec_bytes)
+    return fail(FA_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                workspace_bytes, c.qw_bytes + c.rec_bytes);
+  e = fa::launch_decode(plan, c, q, cache, out, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_decode: launch");
+  return FA_OK;
+}
+
+int fa_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: stream");
+  unsigned int w = 0;
+  e = fa::read_and_clear_watchdog(&w);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: watchdog");
+  if (w != 0)
+    return fail(FA_ERR_DEVICE, "kernel %u hit the wait limit at site %u", w >> 8, w & 0xFFu);
+  return FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,77 @@
+// fa_basis.cu -- the orthonormal real Fourier basis over the middle span, as a table.
+//
+// Basis ([abstract] "orthogonal Fourier bases"; [skill] Step 2, leading real-FFT terms):
+//   phi_0(t) = 1/sqrt(M);  phi_{2f-1}(t) = s_f cos(2 pi f t / M);  phi_{2f}(t) = s_f sin(2 pi f t / M)
+// with s_f = sqrt(2/M), except s_f = 1/sqrt(M) for the Nyquist cosine f = M/2 (M even).
+// The table is stored transposed, phiT[j][t], so that it is the K-major A operand of the
+// tensor-core projection in fa_compress.
+#include "fa_host.h"
+#include "fa_internal.cuh"
+
+namespace fa {
+
+// One thread writes 8 consecutive columns t0..t0+7 of row j (a 16-byte store for bf16).
+// The phase r = (f * t) mod M advances by f per column, in exact integer arithmetic, and
+// is mapped to x = 2r/M in (-1, 1] before sincospif, so the angle carries no
+// large-argument rounding.
+template <typename T>
+__global__ void __launch_bounds__(256) build_basis_kernel(int M, int k, long long ld,
+                                                          float norm_single, float norm_pair,
+                                                          T* __restrict__ out) {
+  const long long nchunk = ld / 8;
+  const long long total = (long long)k * nchunk;
+  for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
+       id += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(id / nchunk);
+    const long long t0 = (id - (long long)j * nchunk) * 8;
+    const int f = (j + 1) >> 1;
+    const bool is_sin = (j > 0) && ((j & 1) == 0);
+    const float nrm = (f == 0 || 2 * f == M) ? norm_single : norm_pair;
+    long long r = ((long long)f * t0) % M;
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const long long t = t0 + e;
+      if (t < M) {
+        const long long rr = (2 * r > M) ? r - M : r;  // phase in (-M/2, M/2]
+        float s, c;
+        sincospif((float)(2 * rr) / (float)M, &s, &c);
+        v[e] = nrm * (is_sin ? s : c);
+        r += f;
+        if (r >= M) r -= M;
+      } else {
+        v[e] = 0.0f;
+      }
+    }
+    T* dst = out + (long long)j * ld + t0;
+    if constexpr (sizeof(T) == 2) {
+      __nv_bfloat162 p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) p[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+      *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<uint4*>(p);
+    } else {
+      reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
+      reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+  }
+}
+
+cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, void* out,
+                               cudaStream_t stream, int num_sms) {
+  const float norm_single = (float)(1.0 / sqrt((double)M));
+  const float norm_pair = (float)sqrt(2.0 / (double)M);
+  const long long total = (long long)k * (ld / 8);
+  long long blocks = (total + 255) / 256;
+  const long long cap = (long long)num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  if (dtype == FA_BF16)
+    build_basis_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, stream>>>(
+        M, k, ld, norm_single, norm_pair, static_cast<__nv_bfloat16*>(out));
+  else
+    build_basis_kernel<float><<<(unsigned)blocks, 256, 0, stream>>>(
+        M, k, ld, norm_single, norm_pair, static_cast<float*>(out));
+  return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,401 @@
+// fa_compress.cu -- prefill compression of one layer on the tcgen05 tensor cores.
+//
+// [skill] Step 3 splits each KV head's tokens into sink / middle / recent; Step 2 projects
+// the middle span onto the leading Fourier functions; [abstract] restricts the
+// projection to the long-context-insensitive (masked) head dims. Per (batch b, KV head g,
+// X in {K, V}):
+//     C_X = Phi^T . X[S : S+M, compressed dims]          (k x dc, fp32 accumulate -> bf16)
+//     E_X = X[S : S+M, retained dims]                     (bit-exact copy)
+//     F_X = X[sink and recent tokens, all dims]           (bit-exact copy)
+//
+// GEMM mapping (one CTA per 128-coefficient tile x head x {K, V}):
+//   D[128 coefs x 128 dims] += A[128 coefs x 64 tokens] . B[64 tokens x 128 dims]
+//   A = Phi^T tile, K-major (tokens contiguous), loaded by TMA with 128-byte swizzle.
+//   B = cache rows, MN-major (dims contiguous, the cache's own layout), two 64-dim TMA
+//       boxes per stage. The full 128 dims are multiplied; the epilogue keeps the masked
+//       ones (a column gather on the B side is not expressible as a TMA box).
+//   D lives in tensor memory (128 lanes x 128 fp32 columns).
+// Warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread), warps 2-5 pack
+// the retained dims of every stage (coefficient tile 0 only) and run the epilogue.
+// Tokens past the middle span read a zero A (TMA out-of-bounds fill), so the ragged last
+// stage needs no masking.
+#include <cuda.h>
+
+#include "fa_host.h"
+#include "fa_internal.cuh"
+
+namespace fa {
+
+constexpr int CK_BM = 128;
+constexpr int CK_BN = 128;
+constexpr int CK_BK = 64;
+constexpr int CK_STAGES = 4;
+constexpr int CK_A_BYTES = CK_BM * CK_BK * 2;
+constexpr int CK_B_BYTES = CK_BN * CK_BK * 2;
+constexpr int CK_STAGE_BYTES = CK_A_BYTES + CK_B_BYTES;
+constexpr int CK_THREADS = 192;
+constexpr int CK_STAGE_LD = CK_BN + 4;  // fp32 staging row stride (bank-conflict free)
+constexpr int CK_SMEM = CK_STAGES * CK_STAGE_BYTES + 1024 /*align*/ + 1024 /*misc*/;
+static_assert(CK_BM * CK_STAGE_LD * 4 <= CK_STAGES * CK_STAGE_BYTES, "staging fits");
+
+struct CompressParams {
+  int M, k, S, Hkv, n_ktiles;
+  long long c_batch, e_batch;
+  long long c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
+  int dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
+  int de_ld[FA_MAX_KV_HEADS];
+  unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
+  __nv_bfloat16* C[2];
+  __nv_bfloat16* E[2];
+};
+
+// Bounded wait used on abort paths only (no abort-flag check): lets in-flight async
+// copies land before the CTA's shared memory is released.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > 200000000ull) break;
+  }
+}
+
+__global__ void __launch_bounds__(CK_THREADS, 1)
+    compress_kernel(const __grid_constant__ CUtensorMap tm_phi,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CompressParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = smem;
+  uint8_t* misc = smem + CK_STAGES * CK_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* empty = full + CK_STAGES;
+  uint64_t* accum = empty + CK_STAGES;
+  uint64_t* drain = accum + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  unsigned char* perm_s = reinterpret_cast<unsigned char*>(misc + 256);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int ktile = blockIdx.x % p.n_ktiles;
+  const int rest = blockIdx.x / p.n_ktiles;
+  const int which = rest & 1;  // 0 = K, 1 = V
+  const int head = rest >> 1;  // flattened b * Hkv + g
+  const int b = head / p.Hkv;
+  const int g = head - b * p.Hkv;
+  const int dc = p.dc[g];
+  const bool do_pack = (ktile == 0);
+  const int nk = (p.M + CK_BK - 1) / CK_BK;
+  // A head with no compressed dims needs only the packing pass of tile 0.
+  if (dc == 0 && ktile != 0) return;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < CK_STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + (do_pack ? 4 : 0));
+    }
+    mbar_init(accum, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_phi);
+    prefetch_tmap(which ? &tm_v : &tm_k);
+  }
+  if (threadIdx.x < FA_HEAD_DIM) perm_s[threadIdx.x] = p.perm[g][threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, CK_BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_d = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const CUtensorMap* tm_x = which ? &tm_v : &tm_k;
+      int issued = 0;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % CK_STAGES;
+        const uint32_t use = (uint32_t)(it / CK_STAGES);
+        if (it >= CK_STAGES &&
+            !mbar_wait(&empty[s], (use & 1u) ^ 1u, abort_flag, WD_COMPRESS | 1u))
+          break;
+        uint8_t* a_s = stages + s * CK_STAGE_BYTES;
+        uint8_t* b_s = a_s + CK_A_BYTES;
+        mbar_arrive_expect_tx(&full[s], CK_STAGE_BYTES);
+        tma_load_2d(a_s, &tm_phi, &full[s], it * CK_BK, ktile * CK_BM);
+        tma_load_3d(b_s, tm_x, &full[s], 0, p.S + it * CK_BK, head);
+        tma_load_3d(b_s + CK_B_BYTES / 2, tm_x, &full[s], 64, p.S + it * CK_BK, head);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let the copies already issued land before shared memory goes away
+        for (int it = (issued > CK_STAGES ? issued - CK_STAGES : 0); it < issued; ++it)
+          drain_wait(&full[it % CK_STAGES], (uint32_t)(it / CK_STAGES) & 1u);
+      } else {
+        // tail: every stage's last release (MMA commit + pack arrivals) has landed
+        for (int it = (nk > CK_STAGES ? nk - CK_STAGES : 0); it < nk; ++it)
+          mbar_wait(&empty[it % CK_STAGES], (uint32_t)(it / CK_STAGES) & 1u, abort_flag,
+                    WD_COMPRESS | 5u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(CK_BM, CK_BN, /*b_mn_major=*/true);
+      bool ok = true;
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % CK_STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(it / CK_STAGES) & 1u, abort_flag, WD_COMPRESS | 2u)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(stages + s * CK_STAGE_BYTES);
+        const uint32_t b_addr = a_addr + CK_A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < CK_BK / 16; ++kk) {
+          // A: 16 tokens = 32 bytes further along the swizzled 128-byte row.
+          const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+          // B: 16 tokens = two 8-row groups of 128-byte rows; the 64-dim halves are
+          // CK_B_BYTES/2 apart (leading byte offset).
+          const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, CK_B_BYTES / 2, 1024);
+          mma_bf16(tmem_d, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&empty[s]);
+      }
+      if (ok) {
+        mma_commit(accum);
+        // tensor memory is released only after every MMA of this CTA has completed
+        mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 6u);
+      } else {
+        mma_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- pack + epilogue
+    const int et = threadIdx.x - 64;  // 0..127
+    if (do_pack) {
+      const int de = FA_HEAD_DIM - dc;
+      const int de_ld = p.de_ld[g];
+      const int nchunk = de_ld >> 3;
+      __nv_bfloat16* E = p.E[which] + (long long)b * p.e_batch + p.e_off[g];
+      for (int it = 0; it < nk; ++it) {
+        const int s = it % CK_STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(it / CK_STAGES) & 1u, abort_flag, WD_COMPRESS | 3u))
+          break;
+        const uint8_t* b_s = stages + s * CK_STAGE_BYTES + CK_A_BYTES;
+        const int ntok = min(CK_BK, p.M - it * CK_BK);
+        for (int c = et; c < ntok * nchunk; c += 128) {
+          const int tau = c / nchunk;
+          const int q = c - tau * nchunk;
+          uint32_t w[4];
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            uint32_t lohi[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int i = q * 8 + e2 * 2 + h;
+              uint32_t bits = 0;
+              if (i < de) {
+                const int d = perm_s[dc + i];
+                const int half = d >> 6;
+                const int col = d & 63;
+                // 128-byte swizzle: 16-byte chunk index XOR (row mod 8)
+                const int off = half * (CK_B_BYTES / 2) + tau * 128 +
+                                ((((col >> 3) ^ (tau & 7)) << 4) | ((col & 7) << 1));
+                bits = *reinterpret_cast<const unsigned short*>(b_s + off);
+              }
+              lohi[h] = bits;
+            }
+            w[e2] = lohi[0] | (lohi[1] << 16);
+          }
+          *reinterpret_cast<uint4*>(E + (long long)(it * CK_BK + tau) * de_ld + q * 8) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    if (!*abort_flag && dc > 0 && mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u)) {
+      tc_fence_after();
+      float* stage_f = reinterpret_cast<float*>(stages);
+      const int rb = warp & 3;  // TMEM lanes this warp may access: 32*rb .. 32*rb+31
+      const int row = rb * 32 + lane;
+#pragma unroll
+      for (int cb = 0; cb < CK_BN / 32; ++cb) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(rb * 32) << 16) + cb * 32, r);
+        tmem_ld_wait();
+        float4* dst = reinterpret_cast<float4*>(stage_f + row * CK_STAGE_LD + cb * 32);
+#pragma unroll
+        for (int v = 0; v < 8; ++v)
+          dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const int dc_ld = p.dc_ld[g];
+      const int nchunk = dc_ld >> 3;
+      __nv_bfloat16* C = p.C[which] + (long long)b * p.c_batch + p.c_off[g];
+      const int rows = min(CK_BM, p.k - ktile * CK_BM);
+      for (int c = et; c < rows * nchunk; c += 128) {
+        const int r = c / nchunk;
+        const int q = c - r * nchunk;
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int i = q * 8 + e;
+          v[e] = (i < dc) ? stage_f[r * CK_STAGE_LD + perm_s[i]] : 0.0f;
+        }
+        __nv_bfloat162 o[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+        *reinterpret_cast<uint4*>(C + (long long)(ktile * CK_BM + r) * dc_ld + q * 8) =
+            *reinterpret_cast<uint4*>(o);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_d, CK_BN);
+  }
+}
+
+// Sink and recent rows, all dims: F[head][i] = X[head][i < S ? i : L - R + (i - S)].
+__global__ void __launch_bounds__(256) copy_sink_recent_kernel(
+    const uint4* __restrict__ K, const uint4* __restrict__ V, uint4* __restrict__ FK,
+    uint4* __restrict__ FV, int L, int S, int R, long long n_heads) {
+  const int nrow = S + R;
+  const long long total = n_heads * nrow * 16;  // 16 x 16 bytes per 128-dim row
+  for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
+       id += (long long)gridDim.x * blockDim.x) {
+    const long long row = id >> 4;
+    const int c = (int)(id & 15);
+    const long long head = row / nrow;
+    const int i = (int)(row - head * nrow);
+    const long long t = (i < S) ? i : (long long)(L - R) + (i - S);
+    const long long src = ((head * L + t) << 4) + c;
+    FK[id] = K[src];
+    FV[id] = V[src];
+  }
+}
+
+// ------------------------------------------------------------------------- host side
+cudaError_t read_and_clear_watchdog(unsigned int* word) {
+  cudaError_t e = cudaMemcpyFromSymbol(word, g_watchdog, sizeof(unsigned int));
+  if (e != cudaSuccess) return e;
+  const unsigned int zero = 0;
+  return cudaMemcpyToSymbol(g_watchdog, &zero, sizeof(unsigned int));
+}
+
+typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                    const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                    CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled get_encode_fn() {
+  static PFN_encodeTiled fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_encodeTiled>(ptr);
+  }
+  return fn;
+}
+
+// Returns a CUDA error, or cudaErrorInvalidValue with *why set for a host-side reason.
+cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
+                            const void* phiT, const fa_cache* cache, cudaStream_t stream,
+                            const char** why) {
+  const fa_shape& sh = plan->shape;
+  const long long n_heads = (long long)sh.B * sh.Hkv;
+  const int nrow = plan->S + plan->R;
+  if (nrow > 0) {
+    const long long total = n_heads * nrow * 16;
+    long long blocks = (total + 255) / 256;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    copy_sink_recent_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const uint4*>(K), static_cast<const uint4*>(V),
+        static_cast<uint4*>(cache->F_K), static_cast<uint4*>(cache->F_V), sh.L, plan->S,
+        plan->R, n_heads);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  if (plan->M == 0) return cudaSuccess;
+
+  PFN_encodeTiled encode = get_encode_fn();
+  if (!encode) {
+    *why = "cuTensorMapEncodeTiled is unavailable from the driver";
+    return cudaErrorInvalidValue;
+  }
+  CUtensorMap tm_phi, tm_k, tm_v;
+  {
+    cuuint64_t dims[2] = {(cuuint64_t)plan->M, (cuuint64_t)sh.k};
+    cuuint64_t strides[1] = {(cuuint64_t)plan->phi_ld * 2};
+    cuuint32_t box[2] = {CK_BK, CK_BM};
+    cuuint32_t estr[2] = {1, 1};
+    if (encode(&tm_phi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(phiT), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled rejected the basis table";
+      return cudaErrorInvalidValue;
+    }
+  }
+  for (int w = 0; w < 2; ++w) {
+    cuuint64_t dims[3] = {FA_HEAD_DIM, (cuuint64_t)sh.L, (cuuint64_t)n_heads};
+    cuuint64_t strides[2] = {FA_HEAD_DIM * 2, (cuuint64_t)sh.L * FA_HEAD_DIM * 2};
+    cuuint32_t box[3] = {64, CK_BK, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    if (encode(w ? &tm_v : &tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+               const_cast<void*>(w ? V : K), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled rejected the K/V cache";
+      return cudaErrorInvalidValue;
+    }
+  }
+
+  CompressParams cp;
+  memset(&cp, 0, sizeof(cp));
+  cp.M = plan->M;
+  cp.k = sh.k;
+  cp.S = plan->S;
+  cp.Hkv = sh.Hkv;
+  cp.n_ktiles = (sh.k + CK_BM - 1) / CK_BM;
+  cp.c_batch = plan->c_batch;
+  cp.e_batch = plan->e_batch;
+  for (int g = 0; g < sh.Hkv; ++g) {
+    cp.c_off[g] = plan->c_off[g];
+    cp.e_off[g] = plan->e_off[g];
+    cp.dc[g] = plan->dc[g];
+    cp.dc_ld[g] = plan->dc_ld[g];
+    cp.de_ld[g] = plan->de_ld[g];
+    memcpy(cp.perm[g], plan->perm[g], FA_HEAD_DIM);
+  }
+  cp.C[0] = static_cast<__nv_bfloat16*>(cache->C_K);
+  cp.C[1] = static_cast<__nv_bfloat16*>(cache->C_V);
+  cp.E[0] = static_cast<__nv_bfloat16*>(cache->E_K);
+  cp.E[1] = static_cast<__nv_bfloat16*>(cache->E_V);
+
+  cudaError_t e = cudaFuncSetAttribute(compress_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, CK_SMEM);
+  if (e != cudaSuccess) return e;
+  const long long grid = (long long)cp.n_ktiles * 2 * n_heads;
+  compress_kernel<<<(unsigned)grid, CK_THREADS, CK_SMEM, stream>>>(tm_phi, tm_k, tm_v, cp);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

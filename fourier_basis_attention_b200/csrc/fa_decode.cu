@@ -1,0 +1,850 @@
+// fa_decode.cu -- one decode step over the hybrid cache, in the coefficient domain.
+//
+// [skill] Step 4 restores the compressed dims during decoding; here the restoration is
+// folded into the attention algebra instead of materialised. For query head h of batch
+// row b (KV head g = h / G) and middle token t (basis row phi(t)):
+//     score_t  = sigma * ( q_e . E_K[t]  +  phi(t) . w ),     w = C_K^T q_c   (k values)
+//     out_c    = (Phi^T p) C_V  = u C_V,                      u = sum_t p_t phi(t)
+//     out_e    = sum_t p_t E_V[t]
+// and sink / recent tokens use all 128 dims exactly. By associativity this equals softmax
+// attention over the reconstruction Phi C ([skill] Step 4), which the oracle computes.
+//
+// Three launches on the caller's stream:
+//   prologue  per KV head: q_c / q_e gathered by the dim mask, w = C_K^T q_c, with the
+//             softmax scale, log2(e) and the basis normalisation folded in.
+//   main      split-L: CTA (head set, split) streams its token range of E_K / E_V in
+//             tiles of 64 tokens for 8 query heads at once, regenerating cos/sin of the
+//             basis by a rotation recurrence (re-seeded from sincospif of the exactly
+//             reduced phase), with an fp32 online softmax. Extra CTAs do the sink /
+//             recent rows of each KV head. Every CTA writes a partial record
+//             (running max, running sum, value accumulator, u).
+//   combine   per KV head: merges the records, out_c = u C_V, scatters the dims back,
+//             normalises and stores bf16.
+#include "fa_host.h"
+#include "fa_internal.cuh"
+
+namespace fa {
+
+constexpr int DT = 64;    // tokens per tile
+constexpr int DNT = 256;  // threads per CTA
+constexpr int HL = 8;     // query heads per CTA (zero-padded)
+constexpr int FT = 256;   // sink/recent rows per CTA
+
+struct DecodeParams {
+  int B, Hq, Hkv, G, M, k, F, F_pad, nF;
+  int n_splits, split_len, n_fsplits, NKV, n_mid, n_rec;
+  int rec_stride, qw_stride;
+  int NTU, TG, DEC, TGE;
+  float qscale, norm_single, norm_pair, two_over_M;
+  long long e_batch, c_batch;
+  long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
+  int de[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS], dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
+  unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
+  const __nv_bfloat16 *q, *FK, *FV, *EK, *EV, *CK, *CV;
+  __nv_bfloat16* out;
+  float* qw;
+  float* rec;
+};
+
+// cos / sin of 2 pi r / M for an exactly reduced integer phase 0 <= r < M.
+__device__ __forceinline__ void phase_sincos(long long r, int M, float two_over_M, float* s,
+                                             float* c) {
+  const long long rr = (2 * r > M) ? r - M : r;  // (-M/2, M/2]
+  sincospif((float)rr * two_over_M, s, c);
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&x)[8]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// ------------------------------------------------------------------------- prologue
+__global__ void __launch_bounds__(DNT) decode_prologue_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ float qc_s[];  // [G][128]
+  const int kvh = blockIdx.x;
+  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
+  const int dc = p.dc[g], de = p.de[g], dc_ld = p.dc_ld[g];
+  const int tid = threadIdx.x;
+  for (int h = 0; h < p.G; ++h) {
+    const long long gh = (long long)b * p.Hq + (long long)g * p.G + h;
+    float* rec = p.qw + gh * p.qw_stride;
+    if (tid < FA_HEAD_DIM) {
+      const int d = p.perm[g][tid];
+      const float v = __bfloat162float(p.q[gh * FA_HEAD_DIM + d]) * p.qscale;
+      if (tid < dc) {
+        qc_s[h * FA_HEAD_DIM + tid] = v;
+        rec[de + tid] = 0.0f;  // q_e padding [de, 128)
+      } else {
+        qc_s[h * FA_HEAD_DIM + tid] = 0.0f;
+        rec[tid - dc] = v;
+      }
+    }
+    for (int i = tid; i < 2 * p.F_pad; i += DNT) rec[FA_HEAD_DIM + i] = 0.0f;
+  }
+  __syncthreads();
+  const __nv_bfloat16* CK = p.CK + (long long)b * p.c_batch + p.c_off[g];
+  for (int j = tid; j < p.k; j += DNT) {
+    float acc[HL];
+#pragma unroll
+    for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
+    const __nv_bfloat16* row = CK + (long long)j * dc_ld;
+    for (int c = 0; c < dc_ld; c += 8) {
+      float x[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c), x);
+#pragma unroll
+      for (int h = 0; h < HL; ++h) {
+        if (h < p.G) {
+          const float4 q0 = *reinterpret_cast<const float4*>(qc_s + h * FA_HEAD_DIM + c);
+          const float4 q1 = *reinterpret_cast<const float4*>(qc_s + h * FA_HEAD_DIM + c + 4);
+          acc[h] += q0.x * x[0] + q0.y * x[1] + q0.z * x[2] + q0.w * x[3] + q1.x * x[4] +
+                    q1.y * x[5] + q1.z * x[6] + q1.w * x[7];
+        }
+      }
+    }
+    const int f = (j + 1) >> 1;
+    const int comp = (j > 0 && (j & 1) == 0) ? 1 : 0;
+    const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+#pragma unroll
+    for (int h = 0; h < HL; ++h) {
+      if (h < p.G) {
+        const long long gh = (long long)b * p.Hq + (long long)g * p.G + h;
+        p.qw[gh * p.qw_stride + FA_HEAD_DIM + 2 * f + comp] = acc[h] * nrm;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- main: middle
+template <int SPT>
+__device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, int cta) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int hs = cta / p.n_splits, sp = cta - (cta / p.n_splits) * p.n_splits;
+  const int lo = sp * p.split_len;
+  const int hi = min(p.M, lo + p.split_len);
+  const int M = p.M;
+
+  float* Ws = sm;                           // [F_pad][HL][2]
+  float* qes = Ws + p.F_pad * HL * 2;       // [HL][128]
+  float* ps = qes + HL * FA_HEAD_DIM;       // [DT][HL]
+  float* red = ps + DT * HL;                // [4][DT][HL]
+  float* mx = red + 4 * DT * HL;            // [8][HL]
+  float* alpha_s = mx + 8 * HL;             // [HL]
+  float* mrun_s = alpha_s + HL;             // [HL]
+  float* ured = mrun_s + HL;                // [DNT][16]
+  long long* ebase_s = reinterpret_cast<long long*>(ured + DNT * 16);  // [HL]
+  int* deld_s = reinterpret_cast<int*>(ebase_s + HL);                  // [HL]
+  int* gh_s = deld_s + HL;                                             // [HL]
+
+  if (tid < HL) {
+    const int n = tid / p.G;
+    const int kv = hs * p.NKV + n;
+    const bool valid = (n < p.NKV) && (kv < p.B * p.Hkv);
+    if (valid) {
+      const int b = kv / p.Hkv, g = kv - (kv / p.Hkv) * p.Hkv;
+      gh_s[tid] = b * p.Hq + g * p.G + (tid - n * p.G);
+      ebase_s[tid] = (long long)b * p.e_batch + p.e_off[g];
+      deld_s[tid] = p.de_ld[g];
+    } else {
+      gh_s[tid] = -1;
+      ebase_s[tid] = 0;
+      deld_s[tid] = 0;
+    }
+    mrun_s[tid] = -INFINITY;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < p.F_pad * HL * 2; idx += DNT) {
+    const int f = idx >> 4, i = (idx >> 1) & 7, c = idx & 1;
+    const int gh = gh_s[i];
+    Ws[idx] = (gh >= 0 && f < p.F) ? p.qw[(long long)gh * p.qw_stride + FA_HEAD_DIM + 2 * f + c]
+                                   : 0.0f;
+  }
+  for (int idx = tid; idx < HL * FA_HEAD_DIM; idx += DNT) {
+    const int i = idx >> 7, d = idx & 127;
+    const int gh = gh_s[i];
+    qes[idx] = gh >= 0 ? p.qw[(long long)gh * p.qw_stride + d] : 0.0f;
+  }
+  __syncthreads();
+
+  // scores role: token tau, quarter qf of the frequency slots
+  const int tau = ((warp & 1) << 5) | lane;
+  const int qf = warp >> 1;
+  const int FQ = (p.F + 3) >> 2;
+  const int fb = qf * FQ, fe = min(p.F, fb + FQ);
+  const int i0 = 2 * qf, i1 = 2 * qf + 1;
+  const bool v0 = gh_s[i0] >= 0, v1 = gh_s[i1] >= 0;
+  const long long eb0 = ebase_s[i0], eb1 = ebase_s[i1];
+  const int dl0 = deld_s[i0], dl1 = deld_s[i1];
+  // softmax role: token tau2, heads 2hp, 2hp+1
+  const int tau2 = tid >> 2, hp = tid & 3;
+  float l0 = 0.0f, l1 = 0.0f;
+  // u role: slots ui + j * NTU, token group uq
+  const int ui = tid % p.NTU, uq = tid / p.NTU;
+  const int UT = DT / p.TG;
+  float uacc[SPT][HL][2];
+  float cb[SPT], sb[SPT];
+#pragma unroll
+  for (int j = 0; j < SPT; ++j) {
+    phase_sincos((long long)(ui + j * p.NTU) % M, M, p.two_over_M, &sb[j], &cb[j]);
+#pragma unroll
+    for (int h = 0; h < HL; ++h) uacc[j][h][0] = uacc[j][h][1] = 0.0f;
+  }
+  // exact-dim value role: head ie, 8-dim chunk ce, token group qg
+  const int ei = tid % (HL * p.DEC), qg = tid / (HL * p.DEC);
+  const int ie = ei / p.DEC, ce = ei - (ei / p.DEC) * p.DEC;
+  const bool e_on = gh_s[ie] >= 0 && ce * 8 < deld_s[ie];
+  const long long ebe = ebase_s[ie];
+  const int dle = deld_s[ie];
+  const int ET = DT / p.TGE;
+  float acce[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acce[e] = 0.0f;
+
+  for (int t0 = lo; t0 < hi; t0 += DT) {
+    const int nt = min(DT, hi - t0);
+    // prefetch the next tile's rows into L2
+    if (tid < 2 * HL) {
+      const int i = (tid & 7);
+      const int tn = t0 + DT;
+      if (gh_s[i] >= 0 && (i % p.G) == 0 && tn < hi) {
+        const int nb = min(DT, hi - tn);
+        const __nv_bfloat16* base = (tid < HL ? p.EK : p.EV) + ebase_s[i] + (long long)tn * deld_s[i];
+        prefetch_l2_bulk(base, (uint32_t)(nb * deld_s[i] * 2));
+      }
+    }
+    // ---------------------------------------------------------------- scores
+    float part[HL];
+#pragma unroll
+    for (int h = 0; h < HL; ++h) part[h] = 0.0f;
+    const int tm = t0 + tau;
+    if (tau < nt) {
+      if (fb < fe) {
+        float sa, ca;
+        phase_sincos(tm, M, p.two_over_M, &sa, &ca);
+        for (int f0 = fb; f0 < fe; f0 += 32) {
+          float s, c;
+          phase_sincos(((long long)f0 * tm) % M, M, p.two_over_M, &s, &c);
+          const int f1 = min(fe, f0 + 32);
+          for (int f = f0; f < f1; ++f) {
+            const float4* w4 = reinterpret_cast<const float4*>(Ws + f * (HL * 2));
+            const float4 a = w4[0], bq = w4[1], cq = w4[2], dq = w4[3];
+            part[0] += c * a.x + s * a.y;
+            part[1] += c * a.z + s * a.w;
+            part[2] += c * bq.x + s * bq.y;
+            part[3] += c * bq.z + s * bq.w;
+            part[4] += c * cq.x + s * cq.y;
+            part[5] += c * cq.z + s * cq.w;
+            part[6] += c * dq.x + s * dq.y;
+            part[7] += c * dq.z + s * dq.w;
+            const float cn = c * ca - s * sa;
+            s = s * ca + c * sa;
+            c = cn;
+          }
+        }
+      }
+      // exact dims of the middle tokens for heads i0, i1
+      float e0 = 0.0f, e1 = 0.0f;
+      if (v0) {
+        const __nv_bfloat16* row = p.EK + eb0 + (long long)tm * dl0;
+        for (int c8 = 0; c8 < dl0; c8 += 8) {
+          float x[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c8), x);
+          const float4 qa = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8);
+          const float4 qb = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8 + 4);
+          e0 += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
+                qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
+        }
+      }
+      if (v1) {
+        const __nv_bfloat16* row = p.EK + eb1 + (long long)tm * dl1;
+        for (int c8 = 0; c8 < dl1; c8 += 8) {
+          float x[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c8), x);
+          const float4 qa = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8);
+          const float4 qb = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8 + 4);
+          e1 += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
+                qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < HL; ++h) {
+        if (h == i0) part[h] += e0;
+        if (h == i1) part[h] += e1;
+      }
+    }
+    {
+      float4* dst = reinterpret_cast<float4*>(red + (qf * DT + tau) * HL);
+      dst[0] = make_float4(part[0], part[1], part[2], part[3]);
+      dst[1] = make_float4(part[4], part[5], part[6], part[7]);
+    }
+    __syncthreads();
+    // ---------------------------------------------------------------- online softmax
+    float s0, s1;
+    {
+      const int h0 = 2 * hp;
+      s0 = red[(0 * DT + tau2) * HL + h0] + red[(1 * DT + tau2) * HL + h0] +
+           red[(2 * DT + tau2) * HL + h0] + red[(3 * DT + tau2) * HL + h0];
+      s1 = red[(0 * DT + tau2) * HL + h0 + 1] + red[(1 * DT + tau2) * HL + h0 + 1] +
+           red[(2 * DT + tau2) * HL + h0 + 1] + red[(3 * DT + tau2) * HL + h0 + 1];
+      if (tau2 >= nt) s0 = s1 = -INFINITY;
+      float m0 = s0, m1 = s1;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, o));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      }
+      if (lane < 4) {
+        mx[warp * HL + 2 * lane] = m0;
+        mx[warp * HL + 2 * lane + 1] = m1;
+      }
+    }
+    __syncthreads();
+    if (tid < HL) {
+      float tmx = mx[tid];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) tmx = fmaxf(tmx, mx[w * HL + tid]);
+      const float mold = mrun_s[tid];
+      const float mnew = fmaxf(mold, tmx);
+      alpha_s[tid] = (mold == -INFINITY) ? 0.0f : exp2f(mold - mnew);
+      mrun_s[tid] = mnew;
+    }
+    __syncthreads();
+    {
+      const int h0 = 2 * hp;
+      const float pv0 = exp2f(s0 - mrun_s[h0]);
+      const float pv1 = exp2f(s1 - mrun_s[h0 + 1]);
+      *reinterpret_cast<float2*>(ps + tau2 * HL + h0) = make_float2(pv0, pv1);
+      l0 = l0 * alpha_s[h0] + pv0;
+      l1 = l1 * alpha_s[h0 + 1] + pv1;
+    }
+    __syncthreads();
+    // ---------------------------------------------------------------- u += p phi
+    {
+      float al[HL];
+#pragma unroll
+      for (int h = 0; h < HL; ++h) al[h] = alpha_s[h];
+#pragma unroll
+      for (int j = 0; j < SPT; ++j)
+#pragma unroll
+        for (int h = 0; h < HL; ++h) {
+          uacc[j][h][0] *= al[h];
+          uacc[j][h][1] *= al[h];
+        }
+      const int tb = uq * UT, te = min(nt, tb + UT);
+      if (tb < te) {
+        float c[SPT], s[SPT];
+#pragma unroll
+        for (int j = 0; j < SPT; ++j)
+          phase_sincos(((long long)(ui + j * p.NTU) * (t0 + tb)) % M, M, p.two_over_M, &s[j],
+                       &c[j]);
+        for (int t = tb; t < te; ++t) {
+          const float4 pa = *reinterpret_cast<const float4*>(ps + t * HL);
+          const float4 pb = *reinterpret_cast<const float4*>(ps + t * HL + 4);
+          const float pr[HL] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+#pragma unroll
+          for (int j = 0; j < SPT; ++j) {
+#pragma unroll
+            for (int h = 0; h < HL; ++h) {
+              uacc[j][h][0] += pr[h] * c[j];
+              uacc[j][h][1] += pr[h] * s[j];
+            }
+            const float cn = c[j] * cb[j] - s[j] * sb[j];
+            s[j] = s[j] * cb[j] + c[j] * sb[j];
+            c[j] = cn;
+          }
+        }
+      }
+    }
+    // ---------------------------------------------------------------- exact-dim values
+    {
+      const float ae = alpha_s[ie];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acce[e] *= ae;
+      if (e_on) {
+        const int tb = qg * ET, te = min(nt, tb + ET);
+        for (int t = tb; t < te; ++t) {
+          const float pv = ps[t * HL + ie];
+          float x[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(p.EV + ebe + (long long)(t0 + t) * dle +
+                                                        ce * 8),
+                        x);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acce[e] += pv * x[e];
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ------------------------------------------------------------------ partial record
+  const long long bhq = (long long)p.B * p.Hq;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  if (lane < 4) {
+    mx[warp * HL + 2 * lane] = l0;
+    mx[warp * HL + 2 * lane + 1] = l1;
+  }
+  // exact-dim accumulators: reduce over token groups
+  {
+    float4* dst = reinterpret_cast<float4*>(red + (qg * (HL * p.DEC) + ei) * 8);
+    dst[0] = make_float4(acce[0], acce[1], acce[2], acce[3]);
+    dst[1] = make_float4(acce[4], acce[5], acce[6], acce[7]);
+  }
+  if (p.TG > 1) {
+    // SPT == 1 whenever TG > 1
+    float4* dst = reinterpret_cast<float4*>(ured + tid * 16);
+#pragma unroll
+    for (int h = 0; h < HL; h += 2)
+      dst[h / 2] = make_float4(uacc[0][h][0], uacc[0][h][1], uacc[0][h + 1][0], uacc[0][h + 1][1]);
+  }
+  __syncthreads();
+  if (tid < HL && gh_s[tid] >= 0) {
+    float l = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) l += mx[w * HL + tid];
+    float* rec = p.rec + ((long long)sp * bhq + gh_s[tid]) * p.rec_stride;
+    rec[0] = mrun_s[tid];
+    rec[1] = l;
+  }
+  if (qg == 0 && e_on) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+    for (int q2 = 0; q2 < p.TGE; ++q2) {
+      const float* src = red + (q2 * (HL * p.DEC) + ei) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] += src[e];
+    }
+    float* rec = p.rec + ((long long)sp * bhq + gh_s[ie]) * p.rec_stride + 4 + ce * 8;
+    reinterpret_cast<float4*>(rec)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(rec)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+  if (p.TG > 1) {
+    if (uq == 0 && ui < p.F) {
+      float v[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = 0.0f;
+      for (int q2 = 0; q2 < p.TG; ++q2) {
+        const float* src = ured + (q2 * p.NTU + ui) * 16;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[e] += src[e];
+      }
+#pragma unroll
+      for (int h = 0; h < HL; ++h) {
+        if (gh_s[h] >= 0) {
+          float* rec = p.rec + ((long long)sp * bhq + gh_s[h]) * p.rec_stride + 4 + FA_HEAD_DIM;
+          *reinterpret_cast<float2*>(rec + 2 * ui) = make_float2(v[2 * h], v[2 * h + 1]);
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < SPT; ++j) {
+      const int f = ui + j * p.NTU;
+      if (f < p.F) {
+#pragma unroll
+        for (int h = 0; h < HL; ++h) {
+          if (gh_s[h] >= 0) {
+            float* rec = p.rec + ((long long)sp * bhq + gh_s[h]) * p.rec_stride + 4 + FA_HEAD_DIM;
+            *reinterpret_cast<float2*>(rec + 2 * f) = make_float2(uacc[j][h][0], uacc[j][h][1]);
+          }
+        }
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------------- main: sink/recent
+__device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float* sm, int fid) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int kvh = fid / p.n_fsplits, fs = fid - (fid / p.n_fsplits) * p.n_fsplits;
+  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
+  const int r0 = fs * FT, nr = min(FT, p.nF - r0);
+  const int G = p.G;
+  float* qs = sm;                       // [HL][128]
+  float* sc = qs + HL * FA_HEAD_DIM;    // [FT][HL]
+  float* mxs = sc + FT * HL;            // [8][HL]
+  float* mh = mxs + 8 * HL;             // [HL]
+  float* red = mh + HL;                 // [DNT][8]
+
+  for (int idx = tid; idx < HL * FA_HEAD_DIM; idx += DNT) {
+    const int h = idx >> 7, d = idx & 127;
+    qs[idx] = (h < G) ? __bfloat162float(p.q[((long long)b * p.Hq + g * G + h) * FA_HEAD_DIM + d]) *
+                            p.qscale
+                      : 0.0f;
+  }
+  __syncthreads();
+  const __nv_bfloat16* FKh = p.FK + (long long)kvh * p.nF * FA_HEAD_DIM;
+  const __nv_bfloat16* FVh = p.FV + (long long)kvh * p.nF * FA_HEAD_DIM;
+  float s[HL];
+#pragma unroll
+  for (int h = 0; h < HL; ++h) s[h] = 0.0f;
+  if (tid < nr) {
+    const __nv_bfloat16* row = FKh + (long long)(r0 + tid) * FA_HEAD_DIM;
+    for (int c = 0; c < FA_HEAD_DIM; c += 8) {
+      float x[8];
+      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c), x);
+#pragma unroll
+      for (int h = 0; h < HL; ++h) {
+        if (h < G) {
+          const float4 qa = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c);
+          const float4 qb = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c + 4);
+          s[h] += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
+                  qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < HL; ++h)
+    if (tid >= nr || h >= G) s[h] = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < HL; ++h) {
+    float m = s[h];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) mxs[warp * HL + h] = m;
+  }
+  __syncthreads();
+  if (tid < HL) {
+    float m = mxs[tid];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) m = fmaxf(m, mxs[w * HL + tid]);
+    mh[tid] = m;
+  }
+  __syncthreads();
+  float l[HL];
+#pragma unroll
+  for (int h = 0; h < HL; ++h) {
+    const float pv = (h < G && tid < nr) ? exp2f(s[h] - mh[h]) : 0.0f;
+    sc[tid * HL + h] = pv;
+    l[h] = pv;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < HL; ++h) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
+    if (lane == 0) mxs[warp * HL + h] = l[h];
+  }
+  // values: item (head h, 8-dim chunk c), token group grp
+  const int items = G * 16;
+  const int it = tid % items, grp = tid / items, ngrp = DNT / items;
+  const int h = it >> 4, c = it & 15;
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+  for (int rr = grp; rr < nr; rr += ngrp) {
+    const float pv = sc[rr * HL + h];
+    float x[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += pv * x[e];
+  }
+  {
+    float4* dst = reinterpret_cast<float4*>(red + tid * 8);
+    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+  }
+  __syncthreads();
+  const long long bhq = (long long)p.B * p.Hq;
+  const int rix = p.n_splits + fs;
+  if (tid < G) {
+    float ls = 0.0f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) ls += mxs[w * HL + tid];
+    float* rec = p.rec + ((long long)rix * bhq + (long long)b * p.Hq + g * G + tid) * p.rec_stride;
+    rec[0] = mh[tid];
+    rec[1] = ls;
+  }
+  if (grp == 0) {
+    float v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+    for (int q2 = 0; q2 < ngrp; ++q2) {
+      const float* src = red + (q2 * items + it) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] += src[e];
+    }
+    float* rec = p.rec + ((long long)rix * bhq + (long long)b * p.Hq + g * G + h) * p.rec_stride +
+                 4 + c * 8;
+    reinterpret_cast<float4*>(rec)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(rec)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+}
+
+template <int SPT>
+__global__ void __launch_bounds__(DNT, 1) decode_main_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(16) float sm[];
+  const int cta = blockIdx.x;
+  if (cta < p.n_mid)
+    decode_middle<SPT>(p, sm, cta);
+  else
+    decode_sink_recent(p, sm, cta - p.n_mid);
+}
+
+// ------------------------------------------------------------------------- combine
+__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(16) float cs[];
+  const int kvh = blockIdx.x, tid = threadIdx.x;
+  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
+  const int G = p.G, dc = p.dc[g], dc_ld = p.dc_ld[g], nrec = p.n_rec;
+  const int k_pad = (p.k + 3) & ~3;
+  float* wts = cs;                        // [G][nrec]
+  float* u = wts + G * nrec;              // [G][k_pad]
+  float* oacc = u + G * k_pad;            // [G][128]
+  float* lsum = oacc + G * FA_HEAD_DIM;   // [G] (padded to 8)
+  int* inv = reinterpret_cast<int*>(lsum + 8);  // [128]
+  const long long bhq = (long long)p.B * p.Hq;
+
+  inv[p.perm[g][tid]] = tid;
+  for (int h = 0; h < G; ++h) {
+    const long long gh = (long long)b * p.Hq + g * G + h;
+    float mstar = -INFINITY;
+    for (int r = 0; r < nrec; ++r) mstar = fmaxf(mstar, p.rec[((long long)r * bhq + gh) * p.rec_stride]);
+    for (int r = tid; r < nrec; r += 128)
+      wts[h * nrec + r] = exp2f(p.rec[((long long)r * bhq + gh) * p.rec_stride] - mstar);
+  }
+  __syncthreads();
+  for (int h = 0; h < G; ++h) {
+    const long long gh = (long long)b * p.Hq + g * G + h;
+    if (tid == 0) {
+      float l = 0.0f;
+      for (int r = 0; r < nrec; ++r) l += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 1];
+      lsum[h] = l;
+    }
+    const int d = tid;
+    const int i = inv[d];
+    float v = 0.0f;
+    if (i >= dc)
+      for (int r = 0; r < p.n_splits; ++r)
+        v += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + (i - dc)];
+    for (int r = p.n_splits; r < nrec; ++r)
+      v += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + d];
+    oacc[h * FA_HEAD_DIM + d] = v;
+    for (int j = tid; j < p.k; j += 128) {
+      const int f = (j + 1) >> 1;
+      const int comp = (j > 0 && (j & 1) == 0) ? 1 : 0;
+      const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+      float acc = 0.0f;
+      for (int r = 0; r < p.n_splits; ++r)
+        acc += wts[h * nrec + r] *
+               p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + FA_HEAD_DIM + 2 * f + comp];
+      u[h * k_pad + j] = acc * nrm;
+    }
+  }
+  __syncthreads();
+  if (tid < dc && p.n_splits > 0) {
+    const __nv_bfloat16* CV = p.CV + (long long)b * p.c_batch + p.c_off[g] + tid;
+    float acc[HL];
+#pragma unroll
+    for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
+    for (int j = 0; j < p.k; ++j) {
+      const float cv = __bfloat162float(CV[(long long)j * dc_ld]);
+#pragma unroll
+      for (int h = 0; h < HL; ++h)
+        if (h < G) acc[h] += u[h * k_pad + j] * cv;
+    }
+    const int d = p.perm[g][tid];
+#pragma unroll
+    for (int h = 0; h < HL; ++h)
+      if (h < G) oacc[h * FA_HEAD_DIM + d] += acc[h];
+  }
+  __syncthreads();
+  for (int h = 0; h < G; ++h) {
+    const long long gh = (long long)b * p.Hq + g * G + h;
+    p.out[gh * FA_HEAD_DIM + tid] = __float2bfloat16_rn(oacc[h * FA_HEAD_DIM + tid] / lsum[h]);
+  }
+}
+
+// ------------------------------------------------------------------------- host side
+static int next_pow2(int x) {
+  int v = 1;
+  while (v < x) v <<= 1;
+  return v;
+}
+
+static size_t main_smem_bytes(int F_pad) {
+  const size_t mid = (size_t)(F_pad * HL * 2 + HL * FA_HEAD_DIM + DT * HL + 4 * DT * HL + 8 * HL +
+                              2 * HL + DNT * 16) * 4 +
+                     HL * 8 + 2 * HL * 4;
+  const size_t fpart = (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + DNT * 8) * 4;
+  return mid > fpart ? mid : fpart;
+}
+
+template <int SPT>
+static cudaError_t occupancy(int* blocks, size_t smem) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(decode_main_kernel<SPT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_main_kernel<SPT>, DNT, smem);
+}
+
+// Derive the launch configuration. `requested` <= 0 selects the split count from a
+// wave-quantisation cost model for the current device.
+cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c) {
+  const fa_shape& sh = plan->shape;
+  const int M = plan->M;
+  c->F = sh.k / 2 + 1;
+  c->F_pad = (c->F + 3) & ~3;
+  c->SPT = c->F <= 256 ? 1 : (c->F <= 512 ? 2 : 4);
+  int ntu = next_pow2((c->F + c->SPT - 1) / c->SPT);
+  if (ntu < 4) ntu = 4;
+  if (ntu > DNT) ntu = DNT;
+  c->NTU = ntu;
+  c->TG = DNT / ntu;
+  int de_ld_max = 8;
+  for (int g = 0; g < sh.Hkv; ++g) de_ld_max = plan->de_ld[g] > de_ld_max ? plan->de_ld[g] : de_ld_max;
+  c->DEC = next_pow2(de_ld_max / 8);
+  c->TGE = DNT / (HL * c->DEC);
+  c->NKV = HL / plan->G;
+  const int n_heads = sh.B * sh.Hkv;
+  const int n_headsets = (n_heads + c->NKV - 1) / c->NKV;
+  c->smem_main = main_smem_bytes(c->F_pad);
+  const int ntiles = (M + DT - 1) / DT;
+  if (M == 0) {
+    c->n_splits = 0;
+    c->split_len = 0;
+  } else {
+    int ns;
+    if (requested > 0) {
+      ns = requested < ntiles ? requested : ntiles;
+    } else {
+      int dev = 0, sms = 148, occ = 1;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return e;
+      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return e;
+      e = c->SPT == 1 ? occupancy<1>(&occ, c->smem_main)
+                      : (c->SPT == 2 ? occupancy<2>(&occ, c->smem_main) : occupancy<4>(&occ, c->smem_main));
+      if (e != cudaSuccess) return e;
+      if (occ < 1) occ = 1;
+      const long long slots = (long long)sms * occ;
+      // cost = waves x tiles per CTA, plus a small per-split charge for the record
+      // traffic and the combine work
+      double best = 1e300;
+      ns = 1;
+      for (int cand = 1; cand <= ntiles && cand <= 4096; ++cand) {
+        const int per = (ntiles + cand - 1) / cand;
+        const int eff = (ntiles + per - 1) / per;
+        if (eff != cand) continue;
+        const long long ctas = (long long)n_headsets * cand;
+        const long long waves = (ctas + slots - 1) / slots;
+        const double cost = (double)waves * (per + 1.0) + 0.02 * cand;
+        if (cost < best) {
+          best = cost;
+          ns = cand;
+        }
+      }
+    }
+    const int per = (ntiles + ns - 1) / ns;
+    c->n_splits = (ntiles + per - 1) / per;
+    c->split_len = per * DT;
+  }
+  const int nF = plan->S + plan->R;
+  c->n_fsplits = (nF + FT - 1) / FT;
+  c->n_rec = c->n_splits + c->n_fsplits;
+  c->rec_stride = 4 + FA_HEAD_DIM + 2 * c->F_pad;
+  c->qw_stride = FA_HEAD_DIM + 2 * c->F_pad;
+  const long long bhq = (long long)sh.B * sh.Hq;
+  c->qw_bytes = (size_t)(bhq * c->qw_stride * 4);
+  c->rec_bytes = (size_t)((long long)c->n_rec * bhq * c->rec_stride * 4);
+  const int k_pad = (sh.k + 3) & ~3;
+  c->smem_combine = (size_t)(plan->G * c->n_rec + plan->G * k_pad + plan->G * FA_HEAD_DIM + 8) * 4 +
+                    FA_HEAD_DIM * 4;
+  return cudaSuccess;
+}
+
+cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
+                          const fa_cache* cache, void* out, void* workspace, cudaStream_t stream) {
+  const fa_shape& sh = plan->shape;
+  DecodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.B = sh.B;
+  p.Hq = sh.Hq;
+  p.Hkv = sh.Hkv;
+  p.G = plan->G;
+  p.M = plan->M;
+  p.k = plan->M > 0 ? sh.k : 0;
+  p.F = c.F;
+  p.F_pad = c.F_pad;
+  p.nF = plan->S + plan->R;
+  p.n_splits = c.n_splits;
+  p.split_len = c.split_len;
+  p.n_fsplits = c.n_fsplits;
+  p.NKV = c.NKV;
+  const int n_heads = sh.B * sh.Hkv;
+  const int n_headsets = (n_heads + c.NKV - 1) / c.NKV;
+  p.n_mid = n_headsets * c.n_splits;
+  p.n_rec = c.n_rec;
+  p.rec_stride = c.rec_stride;
+  p.qw_stride = c.qw_stride;
+  p.NTU = c.NTU;
+  p.TG = c.TG;
+  p.DEC = c.DEC;
+  p.TGE = c.TGE;
+  p.qscale = (float)(1.4426950408889634 / sqrt((double)FA_HEAD_DIM));
+  const int Mq = plan->M > 0 ? plan->M : 1;
+  p.norm_single = (float)(1.0 / sqrt((double)Mq));
+  p.norm_pair = (float)sqrt(2.0 / (double)Mq);
+  p.two_over_M = (float)(2.0 / (double)Mq);
+  p.e_batch = plan->e_batch;
+  p.c_batch = plan->c_batch;
+  for (int g = 0; g < sh.Hkv; ++g) {
+    p.e_off[g] = plan->e_off[g];
+    p.c_off[g] = plan->c_off[g];
+    p.de[g] = plan->de[g];
+    p.de_ld[g] = plan->de_ld[g];
+    p.dc[g] = plan->dc[g];
+    p.dc_ld[g] = plan->dc_ld[g];
+    memcpy(p.perm[g], plan->perm[g], FA_HEAD_DIM);
+  }
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.FK = static_cast<const __nv_bfloat16*>(cache->F_K);
+  p.FV = static_cast<const __nv_bfloat16*>(cache->F_V);
+  p.EK = static_cast<const __nv_bfloat16*>(cache->E_K);
+  p.EV = static_cast<const __nv_bfloat16*>(cache->E_V);
+  p.CK = static_cast<const __nv_bfloat16*>(cache->C_K);
+  p.CV = static_cast<const __nv_bfloat16*>(cache->C_V);
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.qw = static_cast<float*>(workspace);
+  p.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) + c.qw_bytes);
+
+  cudaError_t e;
+  if (p.M > 0) {
+    decode_prologue_kernel<<<n_heads, DNT, plan->G * FA_HEAD_DIM * 4, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const int grid = p.n_mid + n_heads * c.n_fsplits;
+  if (grid > 0) {
+    int occ = 0;
+    if (c.SPT == 1) {
+      if ((e = occupancy<1>(&occ, c.smem_main)) != cudaSuccess) return e;
+      decode_main_kernel<1><<<grid, DNT, c.smem_main, stream>>>(p);
+    } else if (c.SPT == 2) {
+      if ((e = occupancy<2>(&occ, c.smem_main)) != cudaSuccess) return e;
+      decode_main_kernel<2><<<grid, DNT, c.smem_main, stream>>>(p);
+    } else {
+      if ((e = occupancy<4>(&occ, c.smem_main)) != cudaSuccess) return e;
+      decode_main_kernel<4><<<grid, DNT, c.smem_main, stream>>>(p);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (c.smem_combine > 48 * 1024) {
+    e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)c.smem_combine);
+    if (e != cudaSuccess) return e;
+  }
+  decode_combine_kernel<<<n_heads, 128, c.smem_combine, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

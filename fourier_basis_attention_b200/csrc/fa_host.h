@@ -1,0 +1,29 @@
+// fa_host.h -- host-side interfaces between the C ABI (fa_abi.cu) and the kernel units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "../../include/fourier_attention.h"
+
+namespace fa {
+
+// Launch configuration of one fa_decode call (derived by decode_configure).
+struct DecodeConfig {
+  int n_splits, split_len, n_fsplits, n_rec, F, F_pad, SPT, NTU, TG, DEC, TGE, NKV;
+  size_t qw_bytes, rec_bytes, smem_main, smem_combine;
+  int rec_stride, qw_stride;
+};
+
+cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, void* out,
+                               cudaStream_t stream, int num_sms);
+cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
+                            const void* phiT, const fa_cache* cache, cudaStream_t stream,
+                            const char** why);
+cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c);
+cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
+                          const fa_cache* cache, void* out, void* workspace,
+                          cudaStream_t stream);
+cudaError_t read_and_clear_watchdog(unsigned int* word);
+
+}  // namespace fa

@@ -1,0 +1,192 @@
+/*
+ * fourier_attention.h -- C ABI of the B200 (sm_100a) Fourier-approximated KV cache.
+ *
+ * The method (FourierAttention, arXiv 2506.11886): the head dimensions of a KV cache
+ * that are insensitive to long context are projected, over the middle span of the
+ * sequence, onto the first k functions of an orthonormal real Fourier basis; the first
+ * S ("sink") tokens, the last R ("recent") tokens and the remaining head dimensions stay
+ * exact. Decoding attends over this hybrid cache directly in the coefficient domain.
+ *
+ * Sources, cited by page title and section:
+ *   [abstract] shd-paper.top summary of arXiv 2506.11886, "Beyond Homogeneous Attention:
+ *              Memory-Efficient LLMs via Fourier-Approximated KV Cache", abstract and
+ *              "method details".
+ *   [skill]    agent-skills.jp "fourier-approximated-kv-cache" skill page: "Architecture
+ *              overview", Step 2 (fourier_compress_kv_cache), Step 3
+ *              (selective_preserve_tokens), Step 4 (reconstruct_from_fourier), "Practical
+ *              guidance" (custom kernels for the memory-bound prefill/decode work).
+ *
+ * Conventions shared by every entry point
+ *   - Head dimension D is fixed at 128. Query head h of batch row b reads KV head
+ *     g = h / (Hq / Hkv) (grouped-query attention).
+ *   - Every device pointer is caller-owned device memory (for example from PyTorch) and
+ *     must be 16-byte aligned. The library never allocates device memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *     All work is enqueued asynchronously on it; host arguments are consumed before the
+ *     call returns.
+ *   - Return value: FA_OK, or an error code with a message in fa_last_error(). Argument
+ *     errors are detected on the host before anything is launched. Nothing aborts the
+ *     process.
+ *   - bf16 = IEEE bfloat16 (round-to-nearest-even on every store); fp32 accumulation.
+ */
+#ifndef FOURIER_ATTENTION_H
+#define FOURIER_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FA_HEAD_DIM 128
+#define FA_MAX_KV_HEADS 64   /* KV heads per layer */
+#define FA_MAX_K_DECODE 2047 /* largest k fa_decode supports */
+
+enum fa_status {
+  FA_OK = 0,
+  FA_ERR_INVALID = 1,     /* bad argument: null/misaligned pointer, inconsistent shape */
+  FA_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels implement (D != 128, ...) */
+  FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  FA_ERR_DEVICE = 4       /* a kernel's bounded wait expired (see fa_device_status) */
+};
+
+enum fa_dtype { FA_BF16 = 0, FA_F32 = 1 };
+
+/* Shape of one layer's cache. B batch rows, Hq query heads, Hkv KV heads (Hq % Hkv == 0),
+ * D = 128, L cached tokens, S sink and R recent tokens kept exact, k basis functions. */
+typedef struct fa_shape {
+  int32_t B, Hq, Hkv, D, L, S, R, k;
+} fa_shape;
+
+/*
+ * fa_plan: everything derived on the host from (shape, dim mask); plain data, no pointers.
+ *
+ * Token partition ([skill] Step 3): sink [0, S), middle [S, S + M), recent [L - R, L),
+ * each token in exactly one part. If L <= S + R the middle is empty (M = 0) and the
+ * sink/recent windows shrink so that they cover the L tokens once: S = min(S, L),
+ * R = min(R, L - S).
+ *
+ * Dim split ([abstract]: only the long-context-insensitive dims are projected): for KV
+ * head g, perm[g][0 .. dc[g]) lists the compressed dims in ascending order and
+ * perm[g][dc[g] .. 128) the retained dims in ascending order.
+ *
+ * Hybrid cache layout (element offsets, bf16):
+ *   F (sink + recent rows, all dims): [B][Hkv][S + R][128]; row i < S is token i, row
+ *     S + i is token L - R + i.
+ *   E (middle rows, retained dims): block of KV head (b, g) starts at
+ *     b * e_batch + e_off[g] and is [M][de_ld[g]] row-major; columns [de[g], de_ld[g])
+ *     are zero.
+ *   C (Fourier coefficients of the middle rows, compressed dims): block of (b, g) starts
+ *     at b * c_batch + c_off[g] and is [kk][dc_ld[g]] row-major, kk = (M > 0 ? k : 0);
+ *     columns [dc[g], dc_ld[g]) are zero. Row j is basis function j.
+ * de_ld / dc_ld are de / dc rounded up to a multiple of 8 (16-byte rows).
+ *
+ * Basis table (fa_build_basis) row stride: phi_ld = M rounded up to a multiple of 8.
+ */
+typedef struct fa_plan {
+  fa_shape shape;
+  int32_t S, R, M, kk, G;
+  int32_t phi_ld;
+  int32_t dc[FA_MAX_KV_HEADS], de[FA_MAX_KV_HEADS];
+  int32_t dc_ld[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS];
+  int64_t c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
+  int64_t c_batch, e_batch;
+  int64_t f_elems, e_elems, c_elems; /* elements of each of F_K/F_V, E_K/E_V, C_K/C_V */
+  uint8_t perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
+} fa_plan;
+
+/* The hybrid cache of one layer: six caller-allocated bf16 device buffers sized by the
+ * plan (f_elems, e_elems, c_elems). This is the dict {initial, recent,
+ * middle_compressed} of [skill] Step 3, with the retained dims of the middle (E) kept
+ * beside the coefficients (C). */
+typedef struct fa_cache {
+  void* F_K;
+  void* F_V;
+  void* E_K;
+  void* E_V;
+  void* C_K;
+  void* C_V;
+} fa_cache;
+
+/*
+ * fa_plan_init -- derive the plan of one layer.
+ *   shape     host pointer; D must be 128, 1 <= Hkv <= FA_MAX_KV_HEADS, Hq % Hkv == 0,
+ *             B >= 1, L >= 1, S >= 0, R >= 0, k >= 1. If the middle is non-empty and
+ *             some dim is compressed, k <= M is required.
+ *   dim_mask  host uint8 [Hkv][128]; nonzero = that dim of that KV head is compressed.
+ *   plan      host output, fully written on success.
+ * Returns FA_ERR_INVALID / FA_ERR_UNSUPPORTED for shapes the rules above reject.
+ * Pure host function; touches no device.
+ */
+int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan);
+
+/*
+ * fa_build_basis -- the orthonormal real Fourier basis over a span of M tokens, transposed.
+ * ([abstract] "orthogonal Fourier bases"; [skill] Step 2 keeps the leading spectral
+ * terms of a real FFT along the sequence.)
+ *   phiT[j * ld + t] = phi_j(t) for j < k, t < M; columns [M, ld) are written as 0.
+ *   phi_0(t) = 1/sqrt(M); for j >= 1, f = (j + 1) / 2 and phi_j is sqrt(2/M) cos(2 pi f t / M)
+ *   (j odd) or sqrt(2/M) sin(2 pi f t / M) (j even); the cosine at f = M/2 (M even) uses
+ *   1/sqrt(M). The phase f*t is reduced modulo M exactly in integers first.
+ *   dtype FA_BF16 (table for fa_compress) or FA_F32. Requires 1 <= k <= M,
+ *   ld >= M, ld * sizeof(dtype) a multiple of 16. phiT: device, k * ld elements.
+ */
+int fa_build_basis(int32_t M, int32_t k, int32_t dtype, void* phiT, int64_t ld, void* stream);
+
+/*
+ * fa_compress -- prefill compression of one layer ([skill] Steps 2-3; [abstract]).
+ *   K, V   device bf16 [B][Hkv][L][128], the full-precision cache (read only).
+ *   phiT   device bf16 [k][plan->phi_ld] from fa_build_basis(M, k, FA_BF16, ...); may be
+ *          NULL only when M == 0.
+ *   cache  host struct of device output buffers (see fa_plan for layouts); written:
+ *          F = sink/recent rows, E = retained dims of the middle (bit-exact copies),
+ *          C = Phi^T X[S:S+M, compressed dims] with fp32 accumulation, rounded to bf16.
+ * The projection runs on the tcgen05 tensor cores (TMA-fed, accumulator in TMEM).
+ * Requires bf16 values to be finite (a non-finite recent-token value meets a zero basis
+ * entry in the ragged last K tile).
+ */
+int fa_compress(const fa_plan* plan, const void* K, const void* V, const void* phiT,
+                const fa_cache* cache, void* stream);
+
+/*
+ * fa_decode_workspace_size -- bytes of scratch fa_decode needs for `num_splits` split-L
+ * partitions of the middle span (num_splits <= 0: the automatic choice fa_decode makes
+ * for the current device). Returns 0 if the plan is unusable for decode.
+ */
+size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits);
+
+/*
+ * fa_decode -- one decode step: every query attends to all L tokens of the hybrid cache.
+ * ([skill] Step 4, restore during decoding; [abstract].)
+ *   q     device bf16 [B][Hq][128], one query per sequence and head.
+ *   cache the hybrid cache written by fa_compress with the same plan.
+ *   out   device bf16 [B][Hq][128].
+ * Scores of the compressed dims are Phi (C_K q_c) and their values (Phi^T p) C_V, with the
+ * basis regenerated in-kernel (sincos recurrence), never read from memory; the exact dims,
+ * sink and recent tokens use plain dot products. Softmax scale 1/sqrt(128); fp32 online
+ * softmax across split-L partitions merged by a combine pass. The result equals softmax
+ * attention over the reconstructed cache (Phi C on the compressed dims of the middle).
+ *   workspace  device scratch of at least fa_decode_workspace_size(plan, num_splits) bytes.
+ * Requires k <= FA_MAX_K_DECODE and M < 2^21 tokens.
+ */
+int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
+              void* workspace, size_t workspace_bytes, int32_t num_splits, void* stream);
+
+/*
+ * fa_device_status -- synchronise `stream`, then read and clear the library's kernel
+ * watchdog word. Returns FA_OK if no kernel launched since the last call hit a wait
+ * limit, FA_ERR_DEVICE (message names the kernel and wait) if one did, FA_ERR_CUDA if
+ * the stream reported an error. Kernels that hit a limit stop their work, release their
+ * tensor memory and return instead of hanging.
+ */
+int fa_device_status(void* stream);
+
+/* Message of the last non-FA_OK return on the calling thread ("" if none). */
+const char* fa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FOURIER_ATTENTION_H */

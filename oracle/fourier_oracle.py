@@ -37,6 +37,7 @@ Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
 from __future__ import annotations
 
 from dataclasses import dataclass
+from functools import lru_cache
 
 import numpy as np
 
@@ -85,6 +86,15 @@ def _norm(f: np.ndarray, M: int) -> np.ndarray:
     """Orthonormal scale of frequency f: 1/sqrt(M) for DC and Nyquist, else sqrt(2/M)."""
     single = (f == 0) | (2 * f == M)
     return np.where(single, 1.0 / np.sqrt(M), np.sqrt(2.0 / M))
+
+
+@lru_cache(maxsize=2)
+def _basis_full(M: int, k: int) -> np.ndarray:
+    """The whole table, cached (read-only) so that one head's K, V and reconstruction
+    share it; the values are those of ``basis``."""
+    phi = basis(M, k, 0, M)
+    phi.setflags(write=False)
+    return phi
 
 
 def basis(M: int, k: int, t0: int = 0, t1: int | None = None) -> np.ndarray:
@@ -148,7 +158,7 @@ def compress(X, mask_row, S: int, R: int, k: int) -> Hybrid:
     cd, ed = split_dims(mask_row)
     mid = X[s_eff:L - r_eff]
     if M > 0 and cd.size > 0:
-        phi = basis(M, k)
+        phi = _basis_full(M, k)
         C = phi.T @ mid[:, cd]
     else:
         C = np.zeros((k if M > 0 else 0, cd.size))
@@ -171,7 +181,7 @@ def reconstruct(h: Hybrid) -> np.ndarray:
         mid = np.zeros((h.M, h.D))
         mid[:, h.ed] = h.E
         if h.cd.size > 0:
-            mid[:, h.cd] = basis(h.M, h.k) @ h.C
+            mid[:, h.cd] = _basis_full(h.M, h.k) @ h.C
         Xt[h.S:h.S + h.M] = mid
     return Xt
 

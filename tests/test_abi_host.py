@@ -1,0 +1,145 @@
+"""C-ABI checks that need no GPU: exports, host-side plan derivation, argument rejection.
+
+Only host code runs here (fa_plan_init is a pure host function; the other entry points
+are called with arguments the host-side validation rejects before any CUDA call).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import numpy as np
+import pytest
+
+import fourier_basis_attention_b200 as fa
+import workloads as wl
+from oracle import fourier_oracle as fo
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "fourier_attention.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_library_exports_every_declared_function():
+    names = declared_functions()
+    assert set(names) == set(fa.EXPORTED), names
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(fa.LIB, n)
+
+
+def test_plan_struct_matches_header_size():
+    # fa_plan is plain data; the ctypes mirror must have the C layout the header implies
+    assert ctypes.sizeof(fa.fa_shape) == 32
+    expected = 32 + 6 * 4 + 4 * 4 * 64 + 2 * 8 * 64 + 5 * 8 + 64 * 128
+    assert ctypes.sizeof(fa.fa_plan) == expected
+
+
+@pytest.mark.parametrize("w", wl.CONFIGS + [wl.llama3_8b_layer(64, 131072, 5)], ids=lambda w: w.name)
+def test_plan_partition_and_dims_bit_exact(w):
+    m = wl.dim_mask(w)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, m)
+    assert (p.S, p.R, p.M) == fo.partition(w.L, w.S, w.R)
+    for g in range(w.Hkv):
+        cd, ed = fa.perm_lists(p, g)
+        ocd, oed = fo.split_dims(m[g])
+        assert np.array_equal(cd, ocd) and np.array_equal(ed, oed)
+        assert p.dc[g] == len(ocd) and p.de[g] == len(oed)
+
+
+def test_plan_layout_offsets():
+    w = wl.LLAMA3_8B_GQA_32K
+    m = wl.dim_mask(w)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, m)
+    e, c = 0, 0
+    for g in range(w.Hkv):
+        assert p.e_off[g] == e and p.c_off[g] == c
+        assert p.de_ld[g] % 8 == 0 and p.dc_ld[g] % 8 == 0
+        e += p.M * p.de_ld[g]
+        c += w.k * p.dc_ld[g]
+    assert p.e_batch == e and p.c_batch == c
+    assert p.e_elems == w.B * e and p.c_elems == w.B * c
+    assert p.f_elems == w.B * w.Hkv * (w.S + w.R) * 128
+    assert p.phi_ld % 8 == 0 and p.phi_ld >= p.M
+
+
+@pytest.mark.parametrize("L,S,R", [(1, 32, 64), (50, 32, 64), (96, 32, 64), (97, 32, 64),
+                                   (10, 0, 0), (10, 20, 0), (10, 0, 20)])
+def test_plan_edge_partitions(L, S, R):
+    p = fa.fa_plan_init(1, 1, 1, L, S, R, 1, np.ones((1, 128)))
+    assert (p.S, p.R, p.M) == fo.partition(L, S, R)
+    assert p.kk == (1 if p.M > 0 else 0)
+
+
+def test_plan_rejections():
+    m = np.ones((2, 128))
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_plan_init(1, 4, 2, 100, 32, 64, 5, m)   # k=5 > M=4
+    assert e.value.code == fa.FA_ERR_UNSUPPORTED
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_plan_init(1, 3, 2, 1000, 32, 64, 5, m)  # Hq % Hkv != 0
+    assert e.value.code == fa.FA_ERR_INVALID
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_plan_init(1, 4, 2, 1000, 32, 64, 0, m)  # k = 0
+    assert e.value.code == fa.FA_ERR_INVALID
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_plan_init(1, 4, 2, 1000, 32, 64, 5, np.ones((2, 64)), D=64)
+    assert e.value.code == fa.FA_ERR_UNSUPPORTED
+    with pytest.raises(fa.FaError):
+        fa.fa_plan_init(1, 130, 65, 1000, 32, 64, 5, np.ones((65, 128)))
+    # k > M is fine when nothing is compressed
+    p = fa.fa_plan_init(1, 4, 2, 100, 32, 64, 5, np.zeros((2, 128)))
+    assert p.M == 4
+
+
+def test_null_and_misaligned_pointers_rejected_on_host():
+    p = fa.fa_plan_init(1, 4, 1, 300, 32, 64, 31, np.ones((1, 128)))
+    cache = fa.fa_cache(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000)
+    lib = fa.LIB
+    r = lib.fa_compress(ctypes.byref(p), None, 0x1000, 0x1000, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_INVALID and "K" in fa.fa_last_error()
+    r = lib.fa_compress(ctypes.byref(p), 0x1008, 0x1000, 0x1000, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_INVALID and "aligned" in fa.fa_last_error()
+    r = lib.fa_decode(ctypes.byref(p), 0x1000, ctypes.byref(cache), None, 0x1000, 1 << 20, 4, None)
+    assert r == fa.FA_ERR_INVALID and "out" in fa.fa_last_error()
+    r = lib.fa_build_basis(100, 101, fa.FA_BF16, 0x1000, 104, None)
+    assert r == fa.FA_ERR_INVALID
+    r = lib.fa_build_basis(100, 10, fa.FA_BF16, 0x1000, 100, None)  # ld not a multiple of 8
+    assert r == fa.FA_ERR_INVALID
+    # a corrupted plan is rejected before any launch
+    bad = fa.fa_plan_init(1, 4, 1, 300, 32, 64, 31, np.ones((1, 128)))
+    bad.perm[0][5] = bad.perm[0][6]
+    r = lib.fa_compress(ctypes.byref(bad), 0x1000, 0x1000, 0x1000, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_INVALID and "perm" in fa.fa_last_error()
+
+
+def test_decode_rejects_unsupported_group_and_k():
+    p = fa.fa_plan_init(1, 3, 1, 300, 32, 64, 31, np.ones((1, 128)))  # G = 3
+    assert fa.fa_decode_workspace_size(p, 4) == 0
+    p = fa.fa_plan_init(1, 4, 1, 5000, 32, 64, 2049, np.ones((1, 128)))
+    assert fa.fa_decode_workspace_size(p, 4) == 0
+    p = fa.fa_plan_init(1, 4, 1, 5000, 32, 64, 2047, np.ones((1, 128)))
+    assert fa.fa_decode_workspace_size(p, 4) > 0
+
+
+def test_workspace_size_formula():
+    w = wl.LLAMA2_7B_MHA_32K
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    F = w.k // 2 + 1
+    F_pad = (F + 3) // 4 * 4
+    ns = 37
+    ntiles = (p.M + 63) // 64
+    per = -(-ntiles // ns)
+    ns_eff = -(-ntiles // per)
+    n_rec = ns_eff + 1  # one sink/recent split (S + R = 96 rows)
+    bhq = w.B * w.Hq
+    expect = bhq * (128 + 2 * F_pad) * 4 + n_rec * bhq * (4 + 128 + 2 * F_pad) * 4
+    assert fa.fa_decode_workspace_size(p, ns) == expect

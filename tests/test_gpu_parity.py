@@ -1,0 +1,212 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle.
+
+Bars (from the method's tolerances):
+* token / dim partition, sink/recent rows (F) and retained dims (E): bit-exact;
+* floating point (basis table, coefficients C, decode output): max |err| <= 3e-3 * max |ref|
+  over the compared tensor, for bf16 I/O with fp32 accumulation.
+
+Three decode checks: "isolated" (oracle attention over the GPU-written hybrid cache),
+"end-to-end" (oracle compress + attention from the original cache vs GPU compress +
+decode), and the basis / coefficient checks of fa_compress itself. Oracle-sized cases
+compare every element; the full-size workloads compare sampled (batch, KV head) pairs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import fourier_basis_attention_b200 as fa
+import workloads as wl
+from oracle import fourier_oracle as fo
+
+pytestmark = pytest.mark.gpu
+TOL = 3e-3
+D = 128
+
+
+def close(gpu, ref, tol=TOL):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    if ref.size == 0:
+        return 0.0
+    err = np.abs(gpu - ref).max()
+    scale = np.abs(ref).max()
+    assert err <= tol * scale, f"max err {err:.3e} > {tol} * {scale:.3e}"
+    return err / scale
+
+
+def run_path(w, K, V, q, mask, num_splits=0):
+    """GPU compress + decode through the binding (inputs already on the device)."""
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    phiT = fa.basis_table(p)
+    cache = fa.Cache(p)
+    fa.fa_compress(p, K, V, phiT, cache)
+    fa.fa_device_status()
+    ws = torch.empty(max(fa.fa_decode_workspace_size(p, num_splits), 16), dtype=torch.uint8,
+                     device="cuda")
+    out = torch.empty(w.B, w.Hq, D, dtype=torch.bfloat16, device="cuda")
+    fa.fa_decode(p, q, cache, out, ws, num_splits)
+    fa.fa_device_status()
+    torch.cuda.synchronize()
+    return p, cache, out
+
+
+def gpu_hybrid(p, cache, which, b, g, L):
+    """The GPU-written hybrid cache of one head, as an oracle Hybrid (fp64)."""
+    cd, ed = fa.perm_lists(p, g)
+    F = cache.F(which)[b, g].float().cpu().numpy().astype(np.float64)
+    C = cache.C(which, b, g).float().cpu().numpy().astype(np.float64) if p.M > 0 else np.zeros((0, len(cd)))
+    E = cache.E(which, b, g).float().cpu().numpy().astype(np.float64) if p.M > 0 else np.zeros((0, len(ed)))
+    return fo.Hybrid(L=L, D=D, S=p.S, R=p.R, M=p.M, k=p.shape.k, cd=cd, ed=ed,
+                     sink=F[:p.S], recent=F[p.S:], E=E, C=C)
+
+
+def check_head(w, p, cache, out, Kh, Vh, qh, mask_row, b, g):
+    """All parity checks of one (b, g). Kh, Vh: bf16 [L, D] host tensors; qh: [G, D]."""
+    Kd, Vd = Kh.double().numpy(), Vh.double().numpy()
+    hk, hv = fo.compress(Kd, mask_row, w.S, w.R, w.k), fo.compress(Vd, mask_row, w.S, w.R, w.k)
+    # bit-exact parts: sink/recent rows and retained dims
+    for which, X in (("K", Kh), ("V", Vh)):
+        F = cache.F(which)[b, g].cpu()
+        assert torch.equal(F[:p.S], X[:p.S]) and torch.equal(F[p.S:], X[w.L - p.R:])
+        if p.M > 0:
+            ed = torch.from_numpy(fa.perm_lists(p, g)[1])
+            assert torch.equal(cache.E(which, b, g).cpu(), X[p.S:p.S + p.M][:, ed])
+            assert not cache.E_raw(which, b, g)[:, p.de[g]:].any().item()
+            assert not cache.C_raw(which, b, g)[:, p.dc[g]:].any().item()
+    # coefficients
+    if p.M > 0 and p.dc[g] > 0:
+        close(cache.C("K", b, g).float().cpu().numpy(), hk.C)
+        close(cache.C("V", b, g).float().cpu().numpy(), hv.C)
+    o = out[b, g * w.G:(g + 1) * w.G].float().cpu().numpy()
+    q64 = qh.double().numpy()
+    # isolated decode: oracle attention over the GPU-written hybrid cache
+    ref_iso = fo.decode(q64, gpu_hybrid(p, cache, "K", b, g, w.L), gpu_hybrid(p, cache, "V", b, g, w.L))
+    close(o, ref_iso)
+    # end to end: oracle compress + attention from the original cache
+    close(o, fo.decode(q64, hk, hv))
+
+
+def run_small(w, mask=None, num_splits=0, heads=None):
+    mask = wl.dim_mask(w) if mask is None else mask
+    K, V, q = wl.kv_cache(w, "K"), wl.kv_cache(w, "V"), wl.queries(w)
+    p, cache, out = run_path(w, K.cuda(), V.cuda(), q.cuda(), mask, num_splits)
+    pairs = heads or [(b, g) for b in range(w.B) for g in range(w.Hkv)]
+    for b, g in pairs:
+        check_head(w, p, cache, out, K[b, g], V[b, g], q[b, g * w.G:(g + 1) * w.G], mask[g], b, g)
+    return p
+
+
+# ----------------------------------------------------------------------------- basis table
+
+@pytest.mark.parametrize("M,k", [(1, 1), (2, 2), (4, 4), (7, 7), (64, 63), (1952, 63),
+                                 (4096, 4096), (32672, 255), (128992, 1023)])
+def test_basis_table(M, k):
+    ld = (M + 7) // 8 * 8
+    t32 = torch.full((k, ld), 7.0, dtype=torch.float32, device="cuda")
+    t16 = torch.full((k, ld), 7.0, dtype=torch.bfloat16, device="cuda")
+    fa.fa_build_basis(M, k, t32, ld)
+    fa.fa_build_basis(M, k, t16, ld)
+    torch.cuda.synchronize()
+    rows = np.unique(np.linspace(0, k - 1, min(k, 64)).astype(int))
+    cols = np.unique(np.concatenate([np.arange(min(M, 512)), np.linspace(0, M - 1, 2048).astype(int)]))
+    ref = fo.basis(M, k)[np.ix_(cols, rows)].T
+    g32 = t32[rows][:, cols].double().cpu().numpy()
+    g16 = t16[rows][:, cols].double().cpu().numpy()
+    scale = np.sqrt(2.0 / M)
+    assert np.abs(g32 - ref).max() <= 4e-6 * scale
+    assert np.all(np.abs(g16 - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-7 * scale)
+    assert not t32[:, M:].any().item() and not t16[:, M:].any().item()
+
+
+# ----------------------------------------------------------------------------- oracle-sized cases
+
+SMALL = [
+    wl.SINGLE_HEAD_2K,
+    wl.shrink(wl.LLAMA2_7B_MHA_32K, B=2, Hq=4, Hkv=4, L=1000),
+    wl.shrink(wl.LLAMA3_8B_GQA_32K, B=2, Hq=8, Hkv=2, L=1800),
+    wl.shrink(wl.LLAMA3_8B_GQA_128K, B=1, Hq=8, Hkv=2, L=4200),
+    wl.shrink(wl.llama3_8b_layer(1, 8192, 7), B=2, Hq=8, Hkv=2, L=3000),
+]
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: f"{w.name}_B{w.B}_L{w.L}")
+def test_small_workloads_all_heads(w):
+    run_small(w)
+
+
+@pytest.mark.parametrize("ns", [1, 3, 7, 1000])
+def test_forced_split_counts(ns):
+    run_small(wl.shrink(wl.LLAMA3_8B_GQA_32K, B=1, Hq=8, Hkv=2, L=1500), num_splits=ns)
+
+
+@pytest.mark.parametrize("name,kw,mask", [
+    ("no_middle", dict(L=90), "rand96"),                     # L <= S + R
+    ("middle_of_one", dict(L=97, k=1), "rand96"),
+    ("nothing_compressed", dict(L=700), "none"),
+    ("everything_compressed", dict(L=700), "all"),
+    ("k_equals_M", dict(L=96 + 127, k=127), "rand96"),
+    ("k_even", dict(L=700, k=64), "rand96"),
+    ("k_one_dc_only", dict(L=700, k=1), "rand96"),
+    ("k_two", dict(L=700, k=2), "rand96"),
+    ("single_ragged_tile", dict(L=96 + 40, k=17), "rand96"),
+    ("group_2", dict(L=900, Hq=4, Hkv=2, k=31), "rand64or96"),
+    ("group_8", dict(L=900, Hq=16, Hkv=2, k=31), "rand64or96"),
+    ("mha_partial_head_set", dict(L=900, Hq=3, Hkv=3, k=31), "rand96"),
+    ("no_sink", dict(L=800, S=0, k=63), "rand96"),
+    ("no_recent", dict(L=800, R=0, k=63), "rand96"),
+])
+def test_edge_cases(name, kw, mask):
+    base = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=1, Hq=2, Hkv=2, L=700, S=32, R=64, k=31)
+    w = wl.shrink(base, mask=mask, **kw)
+    run_small(w)
+
+
+def test_ragged_mask_padding():
+    """Popcounts that are not multiples of 8 exercise the padded C / E row strides."""
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=2, Hq=4, Hkv=4, L=600, k=47)
+    rng = np.random.default_rng(11)
+    mask = np.zeros((4, D), dtype=np.uint8)
+    for g, dc in enumerate([37, 1, 127, 90]):
+        mask[g, rng.permutation(D)[:dc]] = 1
+    run_small(w, mask=mask)
+
+
+def test_k_equals_M_matches_plain_attention():
+    """With k = M nothing is lost: decode is plain attention over the original cache."""
+    w = wl.shrink(wl.SINGLE_HEAD_2K, L=96 + 127, k=127)
+    K, V, q = wl.kv_cache(w, "K"), wl.kv_cache(w, "V"), wl.queries(w)
+    p, cache, out = run_path(w, K.cuda(), V.cuda(), q.cuda(), wl.dim_mask(w))
+    ref = fo.attention(q[0].double().numpy(), K[0, 0].double().numpy(), V[0, 0].double().numpy(),
+                       1 / np.sqrt(D))
+    close(out[0].float().cpu().numpy(), ref)
+
+
+def test_repeat_calls_are_deterministic():
+    w = wl.shrink(wl.LLAMA3_8B_GQA_32K, B=1, Hq=8, Hkv=2, L=1500)
+    K, V, q = (t.cuda() for t in (wl.kv_cache(w, "K"), wl.kv_cache(w, "V"), wl.queries(w)))
+    _, c1, o1 = run_path(w, K, V, q, wl.dim_mask(w))
+    _, c2, o2 = run_path(w, K, V, q, wl.dim_mask(w))
+    assert torch.equal(c1.C_K, c2.C_K) and torch.equal(o1, o2)
+
+
+# ----------------------------------------------------------------------------- full-size workloads
+
+FULL = [wl.LLAMA2_7B_MHA_32K, wl.LLAMA3_8B_GQA_32K, wl.LLAMA3_8B_GQA_128K,
+        wl.llama3_8b_layer(8, 32768, 3)]
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_full_size_sampled_heads(w):
+    mask = wl.dim_mask(w)
+    K = wl.kv_cache(w, "K", device="cuda")
+    V = wl.kv_cache(w, "V", device="cuda")
+    q = wl.queries(w, device="cuda")
+    p, cache, out = run_path(w, K, V, q, mask)
+    for b, g in [(0, 0), (w.B - 1, w.Hkv - 1)]:
+        check_head(w, p, cache, out, K[b, g].cpu(), V[b, g].cpu(),
+                   q[b, g * w.G:(g + 1) * w.G].cpu(), mask[g], b, g)
+    # every output is finite and every head's F rows are exact copies
+    assert torch.isfinite(out.float()).all().item()
+    idx = torch.cat([torch.arange(p.S), torch.arange(w.L - p.R, w.L)]).cuda()
+    assert torch.equal(cache.F("K"), K[:, :, idx]) and torch.equal(cache.F("V"), V[:, :, idx])
