@@ -61,11 +61,13 @@ def work_model(w, plan):
     S, R, M, k = plan.S, plan.R, plan.M, w.k
     dcs = [plan.dc[g] for g in range(Hkv)]
     des = [plan.de[g] for g in range(Hkv)]
-    # compress: read the middle rows once, write C and E, copy the sink/recent rows (K and V)
-    c_bytes = 2 * 2 * B * sum(M * D + k * dc + M * de + 2 * (S + R) * D for dc, de in zip(dcs, des))
+    # compress: read the middle rows once, write C (fp32) and E, copy the sink/recent rows
+    # (K and V)
+    c_bytes = 2 * B * sum(2 * M * D + 4 * k * dc + 2 * M * de + 2 * 2 * (S + R) * D
+                          for dc, de in zip(dcs, des))
     c_flops = 2 * 2 * B * sum(k * M * dc for dc in dcs)
-    # decode: read F, E and C of K and V, the queries, write the outputs
-    d_bytes = 2 * 2 * B * sum((S + R) * D + M * de + k * dc for dc, de in zip(dcs, des)) \
+    # decode: read F, E (bf16) and C (fp32) of K and V, the queries, write the outputs
+    d_bytes = 2 * B * sum(2 * (S + R) * D + 2 * M * de + 4 * k * dc for dc, de in zip(dcs, des)) \
         + 2 * 2 * B * w.Hq * D
     d_flops = B * G * sum(4 * D * (S + R) + 4 * de * M + 4 * k * dc + 4 * M * k
                           for dc, de in zip(dcs, des))
@@ -258,7 +260,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
         fa.fa_compress(plan, K, V, phiT, cache, stream)
         fa.fa_decode(plan, q, cache, out, ws, 0, stream)
 
@@ -283,7 +285,7 @@ def run_ours(args):
     for i in range(args.steps):
         e = ev[i]
         e[0].record(stream)
-        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
         e[1].record(stream)
         fa.fa_compress(plan, K, V, phiT, cache, stream)
         e[2].record(stream)
@@ -341,7 +343,7 @@ def run_ours(args):
             Kd.copy_(Kh, non_blocking=True)
             Vd.copy_(Vh, non_blocking=True)
             qd.copy_(qh, non_blocking=True)
-            fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, stream)
+            fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
             fa.fa_compress(plan, Kd, Vd, phiT, cache, stream)
             fa.fa_decode(plan, qd, cache, out, ws, 0, stream)
             oh.copy_(out, non_blocking=True)

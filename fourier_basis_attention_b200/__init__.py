@@ -69,11 +69,12 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.fa_plan_init.argtypes = [ctypes.POINTER(fa_shape), P, ctypes.POINTER(fa_plan)]
-    lib.fa_build_basis.argtypes = [I32, I32, I32, P, I64, P]
+    lib.fa_build_basis.argtypes = [I32, I32, I32, I32, P, I64, P]
     lib.fa_compress.argtypes = [ctypes.POINTER(fa_plan), P, P, P, ctypes.POINTER(fa_cache), P]
     lib.fa_decode_workspace_size.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_decode_workspace_size.restype = SZ
-    lib.fa_decode.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, P, SZ, I32, P]
+    lib.fa_decode.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32, P, SZ,
+                              I32, P]
     lib.fa_device_status.argtypes = [P]
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
@@ -121,13 +122,16 @@ def fa_plan_init(B, Hq, Hkv, L, S, R, k, mask, D=HEAD_DIM) -> fa_plan:
     return plan
 
 
-def fa_build_basis(M: int, k: int, phiT, ld: int | None = None, stream=None) -> None:
-    """Fill device tensor ``phiT`` ([k, ld], bf16 or fp32) with the transposed basis."""
+def fa_build_basis(M: int, k: int, phiT, ld: int | None = None, normalized: bool = False,
+                   stream=None) -> None:
+    """Fill device tensor ``phiT`` ([k, ld], bf16 or fp32) with the transposed basis
+    (``normalized=False``: the unit-amplitude table fa_compress reads)."""
     import torch
     dtype = FA_BF16 if phiT.dtype == torch.bfloat16 else FA_F32
     if ld is None:
         ld = phiT.shape[-1]
-    _check(LIB.fa_build_basis(M, k, dtype, _ptr(phiT), ld, _stream(stream)))
+    _check(LIB.fa_build_basis(M, k, dtype, int(bool(normalized)), _ptr(phiT), ld,
+                              _stream(stream)))
 
 
 def fa_compress(plan: fa_plan, K, V, phiT, cache: "Cache", stream=None) -> None:
@@ -141,9 +145,12 @@ def fa_decode_workspace_size(plan: fa_plan, num_splits: int = 0) -> int:
 
 def fa_decode(plan: fa_plan, q, cache: "Cache", out, workspace, num_splits: int = 0,
               stream=None) -> None:
+    """One decode step; ``out`` is a [B, Hq, 128] fp32 or bf16 device tensor."""
+    import torch
+    out_dtype = FA_F32 if out.dtype == torch.float32 else FA_BF16
     nbytes = workspace.numel() * workspace.element_size()
     _check(LIB.fa_decode(ctypes.byref(plan), _ptr(q), ctypes.byref(cache.c), _ptr(out),
-                         _ptr(workspace), nbytes, num_splits, _stream(stream)))
+                         out_dtype, _ptr(workspace), nbytes, num_splits, _stream(stream)))
 
 
 def fa_device_status(stream=None) -> None:
@@ -153,7 +160,8 @@ def fa_device_status(stream=None) -> None:
 # ----------------------------------------------------------------------------- marshalling helpers
 
 class Cache:
-    """Device buffers of one layer's hybrid cache (allocated by torch) + the C struct."""
+    """Device buffers of one layer's hybrid cache (allocated by torch) + the C struct.
+    F and E are bf16, C is fp32 (see fa_plan in the header)."""
 
     def __init__(self, plan: fa_plan, device="cuda"):
         import torch
@@ -163,7 +171,7 @@ class Cache:
         self.F_V = torch.empty_like(self.F_K)
         self.E_K = torch.empty(max(plan.e_elems, 8), dtype=bf, device=device)
         self.E_V = torch.empty_like(self.E_K)
-        self.C_K = torch.empty(max(plan.c_elems, 8), dtype=bf, device=device)
+        self.C_K = torch.empty(max(plan.c_elems, 8), dtype=torch.float32, device=device)
         self.C_V = torch.empty_like(self.C_K)
         self.c = fa_cache(*(t.data_ptr() for t in (self.F_K, self.F_V, self.E_K, self.E_V,
                                                   self.C_K, self.C_V)))
@@ -205,7 +213,7 @@ def basis_table(plan: fa_plan, device="cuda", stream=None):
     if plan.M == 0:
         return None
     phiT = torch.empty(plan.shape.k, plan.phi_ld, dtype=torch.bfloat16, device=device)
-    fa_build_basis(plan.M, plan.shape.k, phiT, plan.phi_ld, stream)
+    fa_build_basis(plan.M, plan.shape.k, phiT, plan.phi_ld, normalized=False, stream=stream)
     return phiT
 
 

@@ -122,7 +122,8 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) 
   return FA_OK;
 }
 
-int fa_build_basis(int32_t M, int32_t k, int32_t dtype, void* phiT, int64_t ld, void* stream) {
+int fa_build_basis(int32_t M, int32_t k, int32_t dtype, int32_t normalized, void* phiT,
+                   int64_t ld, void* stream) {
   if (M < 1 || k < 1 || k > M) return fail(FA_ERR_INVALID, "need 1 <= k <= M (k=%d, M=%d)", k, M);
   if (dtype != FA_BF16 && dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
   if (ld < M || ld % 8 != 0) return fail(FA_ERR_INVALID, "ld=%lld must be >= M and a multiple of 8", (long long)ld);
@@ -131,7 +132,8 @@ int fa_build_basis(int32_t M, int32_t k, int32_t dtype, void* phiT, int64_t ld, 
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e, "fa_build_basis: device query");
-  e = fa::launch_build_basis(M, k, ld, dtype, phiT, static_cast<cudaStream_t>(stream), sms);
+  e = fa::launch_build_basis(M, k, ld, dtype, normalized ? 1 : 0, phiT,
+                             static_cast<cudaStream_t>(stream), sms);
   if (e != cudaSuccess) return cuda_fail(e, "fa_build_basis: launch");
   return FA_OK;
 }
@@ -178,8 +180,11 @@ size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits) {
 }
 
 int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
-              void* workspace, size_t workspace_bytes, int32_t num_splits, void* stream) {
+              int32_t out_dtype, void* workspace, size_t workspace_bytes, int32_t num_splits,
+              void* stream) {
   if (int r = decode_checks(plan)) return r;
+  if (out_dtype != FA_BF16 && out_dtype != FA_F32)
+    return fail(FA_ERR_INVALID, "unknown out_dtype %d", out_dtype);
   if (!cache) return fail(FA_ERR_INVALID, "cache is NULL");
   if (int r = check_ptr(q, "q", true)) return r;
   if (int r = check_ptr(out, "out", true)) return r;
@@ -196,7 +201,8 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
   if (workspace_bytes < c.qw_bytes + c.rec_bytes)
     return fail(FA_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
                 workspace_bytes, c.qw_bytes + c.rec_bytes);
-  e = fa::launch_decode(plan, c, q, cache, out, workspace, static_cast<cudaStream_t>(stream));
+  e = fa::launch_decode(plan, c, q, cache, out, out_dtype, workspace,
+                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fa_decode: launch");
   return FA_OK;
 }

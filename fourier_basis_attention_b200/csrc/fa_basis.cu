@@ -4,7 +4,7 @@
 //   phi_0(t) = 1/sqrt(M);  phi_{2f-1}(t) = s_f cos(2 pi f t / M);  phi_{2f}(t) = s_f sin(2 pi f t / M)
 // with s_f = sqrt(2/M), except s_f = 1/sqrt(M) for the Nyquist cosine f = M/2 (M even).
 // The table is stored transposed, phiT[j][t], so that it is the K-major A operand of the
-// tensor-core projection in fa_compress.
+// tensor-core projection in fa_compress (which reads the unscaled variant: s_f = 1).
 #include "fa_host.h"
 #include "fa_internal.cuh"
 
@@ -18,6 +18,7 @@ template <typename T>
 __global__ void __launch_bounds__(256) build_basis_kernel(int M, int k, long long ld,
                                                           float norm_single, float norm_pair,
                                                           T* __restrict__ out) {
+  // norm_single = norm_pair = 1 gives the unscaled (unit-amplitude) table.
   const long long nchunk = ld / 8;
   const long long total = (long long)k * nchunk;
   for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
@@ -56,10 +57,10 @@ __global__ void __launch_bounds__(256) build_basis_kernel(int M, int k, long lon
   }
 }
 
-cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, void* out,
+cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, int normalized, void* out,
                                cudaStream_t stream, int num_sms) {
-  const float norm_single = (float)(1.0 / sqrt((double)M));
-  const float norm_pair = (float)sqrt(2.0 / (double)M);
+  const float norm_single = normalized ? (float)(1.0 / sqrt((double)M)) : 1.0f;
+  const float norm_pair = normalized ? (float)sqrt(2.0 / (double)M) : 1.0f;
   const long long total = (long long)k * (ld / 8);
   long long blocks = (total + 255) / 256;
   const long long cap = (long long)num_sms * 8;

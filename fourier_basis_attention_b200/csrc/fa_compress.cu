@@ -4,7 +4,7 @@
 // the middle span onto the leading Fourier functions; [abstract] restricts the
 // projection to the long-context-insensitive (masked) head dims. Per (batch b, KV head g,
 // X in {K, V}):
-//     C_X = Phi^T . X[S : S+M, compressed dims]          (k x dc, fp32 accumulate -> bf16)
+//     C_X = Phi^T . X[S : S+M, compressed dims]          (k x dc, fp32)
 //     E_X = X[S : S+M, retained dims]                     (bit-exact copy)
 //     F_X = X[sink and recent tokens, all dims]           (bit-exact copy)
 //
@@ -18,7 +18,8 @@
 // Warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread), warps 2-5 pack
 // the retained dims of every stage (coefficient tile 0 only) and run the epilogue.
 // Tokens past the middle span read a zero A (TMA out-of-bounds fill), so the ragged last
-// stage needs no masking.
+// stage needs no masking. A holds unit-amplitude cos / sin (DC = 1); each accumulator row
+// is scaled by its orthonormal factor (1/sqrt(M) or sqrt(2/M)) in fp32 in the epilogue.
 #include <cuda.h>
 
 #include "fa_host.h"
@@ -40,12 +41,13 @@ static_assert(CK_BM * CK_STAGE_LD * 4 <= CK_STAGES * CK_STAGE_BYTES, "staging fi
 
 struct CompressParams {
   int M, k, S, Hkv, n_ktiles;
+  float norm_single, norm_pair;
   long long c_batch, e_batch;
   long long c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
   int dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
   int de_ld[FA_MAX_KV_HEADS];
   unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
-  __nv_bfloat16* C[2];
+  float* C[2];
   __nv_bfloat16* E[2];
 };
 
@@ -221,7 +223,10 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
         if (lane == 0) mbar_arrive(&empty[s]);
       }
     }
-    if (!*abort_flag && dc > 0 && mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u)) {
+    // all four warps are done reading the stages before any staging write reuses them
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int acc_ready = (dc > 0 && !*abort_flag) ? (mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u) ? 1 : 0) : 0;
+    if (dc > 0 && bar1_and_128(acc_ready)) {
       tc_fence_after();
       float* stage_f = reinterpret_cast<float*>(stages);
       const int rb = warp & 3;  // TMEM lanes this warp may access: 32*rb .. 32*rb+31
@@ -239,23 +244,23 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const int dc_ld = p.dc_ld[g];
-      const int nchunk = dc_ld >> 3;
-      __nv_bfloat16* C = p.C[which] + (long long)b * p.c_batch + p.c_off[g];
+      const int nchunk = dc_ld >> 2;
+      float* C = p.C[which] + (long long)b * p.c_batch + p.c_off[g];
       const int rows = min(CK_BM, p.k - ktile * CK_BM);
       for (int c = et; c < rows * nchunk; c += 128) {
         const int r = c / nchunk;
         const int q = c - r * nchunk;
-        float v[8];
+        const int j = ktile * CK_BM + r;
+        const int f = (j + 1) >> 1;
+        const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+        float v[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int i = q * 8 + e;
-          v[e] = (i < dc) ? stage_f[r * CK_STAGE_LD + perm_s[i]] : 0.0f;
+        for (int e = 0; e < 4; ++e) {
+          const int i = q * 4 + e;
+          v[e] = (i < dc) ? nrm * stage_f[r * CK_STAGE_LD + perm_s[i]] : 0.0f;
         }
-        __nv_bfloat162 o[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[e] = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-        *reinterpret_cast<uint4*>(C + (long long)(ktile * CK_BM + r) * dc_ld + q * 8) =
-            *reinterpret_cast<uint4*>(o);
+        *reinterpret_cast<float4*>(C + (long long)j * dc_ld + q * 4) =
+            make_float4(v[0], v[1], v[2], v[3]);
       }
     }
   }
@@ -385,8 +390,10 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
     cp.de_ld[g] = plan->de_ld[g];
     memcpy(cp.perm[g], plan->perm[g], FA_HEAD_DIM);
   }
-  cp.C[0] = static_cast<__nv_bfloat16*>(cache->C_K);
-  cp.C[1] = static_cast<__nv_bfloat16*>(cache->C_V);
+  cp.C[0] = static_cast<float*>(cache->C_K);
+  cp.C[1] = static_cast<float*>(cache->C_V);
+  cp.norm_single = (float)(1.0 / sqrt((double)plan->M));
+  cp.norm_pair = (float)sqrt(2.0 / (double)plan->M);
   cp.E[0] = static_cast<__nv_bfloat16*>(cache->E_K);
   cp.E[1] = static_cast<__nv_bfloat16*>(cache->E_V);
 

@@ -19,7 +19,7 @@
 //             recent rows of each KV head. Every CTA writes a partial record
 //             (running max, running sum, value accumulator, u).
 //   combine   per KV head: merges the records, out_c = u C_V, scatters the dims back,
-//             normalises and stores bf16.
+//             normalises and stores fp32 or bf16.
 #include "fa_host.h"
 #include "fa_internal.cuh"
 
@@ -40,8 +40,10 @@ struct DecodeParams {
   long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
   int de[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS], dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
   unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
-  const __nv_bfloat16 *q, *FK, *FV, *EK, *EV, *CK, *CV;
-  __nv_bfloat16* out;
+  const __nv_bfloat16 *q, *FK, *FV, *EK, *EV;
+  const float *CK, *CV;
+  void* out;
+  int out_f32;
   float* qw;
   float* rec;
 };
@@ -86,22 +88,19 @@ __global__ void __launch_bounds__(DNT) decode_prologue_kernel(const __grid_const
     for (int i = tid; i < 2 * p.F_pad; i += DNT) rec[FA_HEAD_DIM + i] = 0.0f;
   }
   __syncthreads();
-  const __nv_bfloat16* CK = p.CK + (long long)b * p.c_batch + p.c_off[g];
+  const float* CK = p.CK + (long long)b * p.c_batch + p.c_off[g];
   for (int j = tid; j < p.k; j += DNT) {
     float acc[HL];
 #pragma unroll
     for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
-    const __nv_bfloat16* row = CK + (long long)j * dc_ld;
-    for (int c = 0; c < dc_ld; c += 8) {
-      float x[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c), x);
+    const float* row = CK + (long long)j * dc_ld;
+    for (int c = 0; c < dc_ld; c += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(row + c);
 #pragma unroll
       for (int h = 0; h < HL; ++h) {
         if (h < p.G) {
           const float4 q0 = *reinterpret_cast<const float4*>(qc_s + h * FA_HEAD_DIM + c);
-          const float4 q1 = *reinterpret_cast<const float4*>(qc_s + h * FA_HEAD_DIM + c + 4);
-          acc[h] += q0.x * x[0] + q0.y * x[1] + q0.z * x[2] + q0.w * x[3] + q1.x * x[4] +
-                    q1.y * x[5] + q1.z * x[6] + q1.w * x[7];
+          acc[h] += q0.x * x.x + q0.y * x.y + q0.z * x.z + q0.w * x.w;
         }
       }
     }
@@ -641,12 +640,12 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   }
   __syncthreads();
   if (tid < dc && p.n_splits > 0) {
-    const __nv_bfloat16* CV = p.CV + (long long)b * p.c_batch + p.c_off[g] + tid;
+    const float* CV = p.CV + (long long)b * p.c_batch + p.c_off[g] + tid;
     float acc[HL];
 #pragma unroll
     for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
     for (int j = 0; j < p.k; ++j) {
-      const float cv = __bfloat162float(CV[(long long)j * dc_ld]);
+      const float cv = CV[(long long)j * dc_ld];
 #pragma unroll
       for (int h = 0; h < HL; ++h)
         if (h < G) acc[h] += u[h * k_pad + j] * cv;
@@ -659,7 +658,11 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_consta
   __syncthreads();
   for (int h = 0; h < G; ++h) {
     const long long gh = (long long)b * p.Hq + g * G + h;
-    p.out[gh * FA_HEAD_DIM + tid] = __float2bfloat16_rn(oacc[h * FA_HEAD_DIM + tid] / lsum[h]);
+    const float o = oacc[h * FA_HEAD_DIM + tid] / lsum[h];
+    if (p.out_f32)
+      static_cast<float*>(p.out)[gh * FA_HEAD_DIM + tid] = o;
+    else
+      static_cast<__nv_bfloat16*>(p.out)[gh * FA_HEAD_DIM + tid] = __float2bfloat16_rn(o);
   }
 }
 
@@ -764,7 +767,8 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
 }
 
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
-                          const fa_cache* cache, void* out, void* workspace, cudaStream_t stream) {
+                          const fa_cache* cache, void* out, int out_dtype, void* workspace,
+                          cudaStream_t stream) {
   const fa_shape& sh = plan->shape;
   DecodeParams p;
   memset(&p, 0, sizeof(p));
@@ -812,9 +816,10 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   p.FV = static_cast<const __nv_bfloat16*>(cache->F_V);
   p.EK = static_cast<const __nv_bfloat16*>(cache->E_K);
   p.EV = static_cast<const __nv_bfloat16*>(cache->E_V);
-  p.CK = static_cast<const __nv_bfloat16*>(cache->C_K);
-  p.CV = static_cast<const __nv_bfloat16*>(cache->C_V);
-  p.out = static_cast<__nv_bfloat16*>(out);
+  p.CK = static_cast<const float*>(cache->C_K);
+  p.CV = static_cast<const float*>(cache->C_V);
+  p.out = out;
+  p.out_f32 = out_dtype == FA_F32 ? 1 : 0;
   p.qw = static_cast<float*>(workspace);
   p.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) + c.qw_bytes);
 

@@ -15,14 +15,14 @@ struct DecodeConfig {
   int rec_stride, qw_stride;
 };
 
-cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, void* out,
+cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, int normalized, void* out,
                                cudaStream_t stream, int num_sms);
 cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
                             const void* phiT, const fa_cache* cache, cudaStream_t stream,
                             const char** why);
 cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c);
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
-                          const fa_cache* cache, void* out, void* workspace,
+                          const fa_cache* cache, void* out, int out_dtype, void* workspace,
                           cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
 

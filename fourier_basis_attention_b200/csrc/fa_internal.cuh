@@ -89,6 +89,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// AND of `pred` over the 128 threads that use named barrier 1 (all of them get the result),
+// so a branch that follows is taken uniformly even if one thread's wait gave up.
+__device__ __forceinline__ int bar1_and_128(int pred) {
+  int out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(pred)
+      : "memory");
+  return out;
+}
+
 // ------------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, uint64_t* bar, int x,
                                             int y) {

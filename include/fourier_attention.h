@@ -71,16 +71,19 @@ typedef struct fa_shape {
  * head g, perm[g][0 .. dc[g]) lists the compressed dims in ascending order and
  * perm[g][dc[g] .. 128) the retained dims in ascending order.
  *
- * Hybrid cache layout (element offsets, bf16):
+ * Hybrid cache layout (element offsets; F and E bf16, C fp32):
  *   F (sink + recent rows, all dims): [B][Hkv][S + R][128]; row i < S is token i, row
  *     S + i is token L - R + i.
  *   E (middle rows, retained dims): block of KV head (b, g) starts at
  *     b * e_batch + e_off[g] and is [M][de_ld[g]] row-major; columns [de[g], de_ld[g])
  *     are zero.
- *   C (Fourier coefficients of the middle rows, compressed dims): block of (b, g) starts
- *     at b * c_batch + c_off[g] and is [kk][dc_ld[g]] row-major, kk = (M > 0 ? k : 0);
- *     columns [dc[g], dc_ld[g]) are zero. Row j is basis function j.
- * de_ld / dc_ld are de / dc rounded up to a multiple of 8 (16-byte rows).
+ *   C (Fourier coefficients of the middle rows, compressed dims, fp32): block of (b, g)
+ *     starts at b * c_batch + c_off[g] and is [kk][dc_ld[g]] row-major,
+ *     kk = (M > 0 ? k : 0); columns [dc[g], dc_ld[g]) are zero. Row j is basis function j.
+ *     C is kept in fp32: it holds k * dc values per head against M * de for E (about 2%
+ *     of the cache at k = M / 128), and a bf16 C would add a second rounding of up to
+ *     2^-8 relative to every reconstructed value.
+ * de_ld / dc_ld are de / dc rounded up to a multiple of 8 (rows of 16 / 32 bytes).
  *
  * Basis table (fa_build_basis) row stride: phi_ld = M rounded up to a multiple of 8.
  */
@@ -96,10 +99,10 @@ typedef struct fa_plan {
   uint8_t perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
 } fa_plan;
 
-/* The hybrid cache of one layer: six caller-allocated bf16 device buffers sized by the
- * plan (f_elems, e_elems, c_elems). This is the dict {initial, recent,
- * middle_compressed} of [skill] Step 3, with the retained dims of the middle (E) kept
- * beside the coefficients (C). */
+/* The hybrid cache of one layer: six caller-allocated device buffers sized by the plan
+ * (f_elems, e_elems, c_elems): F_K, F_V, E_K, E_V bf16; C_K, C_V fp32. This is the dict
+ * {initial, recent, middle_compressed} of [skill] Step 3, with the retained dims of the
+ * middle (E) kept beside the coefficients (C). */
 typedef struct fa_cache {
   void* F_K;
   void* F_V;
@@ -125,23 +128,30 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan);
  * fa_build_basis -- the orthonormal real Fourier basis over a span of M tokens, transposed.
  * ([abstract] "orthogonal Fourier bases"; [skill] Step 2 keeps the leading spectral
  * terms of a real FFT along the sequence.)
- *   phiT[j * ld + t] = phi_j(t) for j < k, t < M; columns [M, ld) are written as 0.
  *   phi_0(t) = 1/sqrt(M); for j >= 1, f = (j + 1) / 2 and phi_j is sqrt(2/M) cos(2 pi f t / M)
  *   (j odd) or sqrt(2/M) sin(2 pi f t / M) (j even); the cosine at f = M/2 (M even) uses
  *   1/sqrt(M). The phase f*t is reduced modulo M exactly in integers first.
- *   dtype FA_BF16 (table for fa_compress) or FA_F32. Requires 1 <= k <= M,
- *   ld >= M, ld * sizeof(dtype) a multiple of 16. phiT: device, k * ld elements.
+ *   normalized = 1: phiT[j * ld + t] = phi_j(t).
+ *   normalized = 0: the same functions without their scale (1 for DC, cos / sin of unit
+ *                   amplitude otherwise). This is the table fa_compress reads (dtype
+ *                   FA_BF16): the scales are applied in fp32 after accumulation, so the
+ *                   DC and Nyquist rows are exact in bf16 and no constant rounding error
+ *                   of 1/sqrt(M) or sqrt(2/M) biases the coefficients.
+ *   Columns [M, ld) are written as 0. dtype FA_BF16 or FA_F32. Requires 1 <= k <= M,
+ *   ld >= M, ld a multiple of 8. phiT: device, k * ld elements.
  */
-int fa_build_basis(int32_t M, int32_t k, int32_t dtype, void* phiT, int64_t ld, void* stream);
+int fa_build_basis(int32_t M, int32_t k, int32_t dtype, int32_t normalized, void* phiT,
+                   int64_t ld, void* stream);
 
 /*
  * fa_compress -- prefill compression of one layer ([skill] Steps 2-3; [abstract]).
  *   K, V   device bf16 [B][Hkv][L][128], the full-precision cache (read only).
- *   phiT   device bf16 [k][plan->phi_ld] from fa_build_basis(M, k, FA_BF16, ...); may be
- *          NULL only when M == 0.
+ *   phiT   device bf16 [k][plan->phi_ld] from fa_build_basis(M, k, FA_BF16, 0, ...) (the
+ *          unscaled table); may be NULL only when M == 0.
  *   cache  host struct of device output buffers (see fa_plan for layouts); written:
  *          F = sink/recent rows, E = retained dims of the middle (bit-exact copies),
- *          C = Phi^T X[S:S+M, compressed dims] with fp32 accumulation, rounded to bf16.
+ *          C = Phi^T X[S:S+M, compressed dims], fp32 (bf16 x bf16 products accumulated in
+ *          fp32 on the tensor cores, then scaled by the orthonormal factor of each row).
  * The projection runs on the tcgen05 tensor cores (TMA-fed, accumulator in TMEM).
  * Requires bf16 values to be finite (a non-finite recent-token value meets a zero basis
  * entry in the ragged last K tile).
@@ -161,7 +171,8 @@ size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits);
  * ([skill] Step 4, restore during decoding; [abstract].)
  *   q     device bf16 [B][Hq][128], one query per sequence and head.
  *   cache the hybrid cache written by fa_compress with the same plan.
- *   out   device bf16 [B][Hq][128].
+ *   out   device [B][Hq][128] of out_dtype: FA_F32, or FA_BF16 (the fp32 result rounded to
+ *         nearest even).
  * Scores of the compressed dims are Phi (C_K q_c) and their values (Phi^T p) C_V, with the
  * basis regenerated in-kernel (sincos recurrence), never read from memory; the exact dims,
  * sink and recent tokens use plain dot products. Softmax scale 1/sqrt(128); fp32 online
@@ -171,7 +182,8 @@ size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits);
  * Requires k <= FA_MAX_K_DECODE and M < 2^21 tokens.
  */
 int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
-              void* workspace, size_t workspace_bytes, int32_t num_splits, void* stream);
+              int32_t out_dtype, void* workspace, size_t workspace_bytes, int32_t num_splits,
+              void* stream);
 
 /*
  * fa_device_status -- synchronise `stream`, then read and clear the library's kernel

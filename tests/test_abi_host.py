@@ -108,11 +108,15 @@ def test_null_and_misaligned_pointers_rejected_on_host():
     assert r == fa.FA_ERR_INVALID and "K" in fa.fa_last_error()
     r = lib.fa_compress(ctypes.byref(p), 0x1008, 0x1000, 0x1000, ctypes.byref(cache), None)
     assert r == fa.FA_ERR_INVALID and "aligned" in fa.fa_last_error()
-    r = lib.fa_decode(ctypes.byref(p), 0x1000, ctypes.byref(cache), None, 0x1000, 1 << 20, 4, None)
+    r = lib.fa_decode(ctypes.byref(p), 0x1000, ctypes.byref(cache), None, fa.FA_BF16, 0x1000,
+                      1 << 20, 4, None)
     assert r == fa.FA_ERR_INVALID and "out" in fa.fa_last_error()
-    r = lib.fa_build_basis(100, 101, fa.FA_BF16, 0x1000, 104, None)
+    r = lib.fa_decode(ctypes.byref(p), 0x1000, ctypes.byref(cache), 0x1000, 7, 0x1000,
+                      1 << 20, 4, None)
+    assert r == fa.FA_ERR_INVALID and "out_dtype" in fa.fa_last_error()
+    r = lib.fa_build_basis(100, 101, fa.FA_BF16, 0, 0x1000, 104, None)
     assert r == fa.FA_ERR_INVALID
-    r = lib.fa_build_basis(100, 10, fa.FA_BF16, 0x1000, 100, None)  # ld not a multiple of 8
+    r = lib.fa_build_basis(100, 10, fa.FA_BF16, 0, 0x1000, 100, None)  # ld not a multiple of 8
     assert r == fa.FA_ERR_INVALID
     # a corrupted plan is rejected before any launch
     bad = fa.fa_plan_init(1, 4, 1, 300, 32, 64, 31, np.ones((1, 128)))
@@ -143,3 +147,13 @@ def test_workspace_size_formula():
     bhq = w.B * w.Hq
     expect = bhq * (128 + 2 * F_pad) * 4 + n_rec * bhq * (4 + 128 + 2 * F_pad) * 4
     assert fa.fa_decode_workspace_size(p, ns) == expect
+
+
+def test_gpu_test_shapes_have_valid_plans():
+    """Every workload the GPU parity tests and smoke() use must pass fa_plan_init."""
+    import __graft_entry__  # noqa: F401
+    import test_gpu_parity as tg
+    shapes = list(tg.SMALL) + list(tg.FULL)
+    shapes.append(wl.shrink(wl.LLAMA3_8B_GQA_32K, B=1, Hq=8, Hkv=2, L=2000))
+    for w in shapes:
+        fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
