@@ -26,7 +26,8 @@ FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE = range(5)
 FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode_workspace_size",
-            "fa_decode", "fa_device_status", "fa_last_error")
+            "fa_decode", "fa_decode_noalloc", "fa_device_status", "fa_last_error")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class FaError(RuntimeError):
@@ -75,10 +76,13 @@ def _load() -> ctypes.CDLL:
     lib.fa_decode_workspace_size.restype = SZ
     lib.fa_decode.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32, P, SZ,
                               I32, P]
+    lib.fa_decode_noalloc.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32,
+                                      I32, P]
     lib.fa_device_status.argtypes = [P]
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
-    for name in ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode", "fa_device_status"):
+    for name in ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode", "fa_decode_noalloc",
+                 "fa_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -151,6 +155,16 @@ def fa_decode(plan: fa_plan, q, cache: "Cache", out, workspace, num_splits: int 
     nbytes = workspace.numel() * workspace.element_size()
     _check(LIB.fa_decode(ctypes.byref(plan), _ptr(q), ctypes.byref(cache.c), _ptr(out),
                          out_dtype, _ptr(workspace), nbytes, num_splits, _stream(stream)))
+
+
+def fa_decode_noalloc(plan: fa_plan, q, cache: "Cache", out, num_splits: int = 0,
+                      stream=None) -> None:
+    """fa_decode without a workspace argument, for callers that cannot allocate device
+    memory: the library's own fixed scratch array is used (see the C header)."""
+    import torch
+    out_dtype = FA_F32 if out.dtype == torch.float32 else FA_BF16
+    _check(LIB.fa_decode_noalloc(ctypes.byref(plan), _ptr(q), ctypes.byref(cache.c), _ptr(out),
+                                 out_dtype, num_splits, _stream(stream)))
 
 
 def fa_device_status(stream=None) -> None:

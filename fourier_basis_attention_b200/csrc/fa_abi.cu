@@ -72,6 +72,8 @@ int check_plan(const fa_plan* plan) {
 
 }  // namespace
 
+int fa::set_last_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 extern "C" {
 
 const char* fa_last_error(void) { return g_last_error.c_str(); }

@@ -26,4 +26,7 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
                           cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
 
+// Records `msg` as the calling thread's fa_last_error() text and returns `code`.
+int set_last_error(int code, const char* msg);
+
 }  // namespace fa

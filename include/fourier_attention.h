@@ -186,6 +186,33 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
               void* stream);
 
 /*
+ * fa_decode_noalloc -- fa_decode for callers that cannot allocate device memory.
+ * (The paper has no counterpart; this is a deployment convenience of this library.)
+ *   Some callers cannot call cudaMalloc or hand over scratch memory: plug-ins running
+ *   inside a host framework that owns every device allocation and exposes no allocator
+ *   to them, serving loops that carved all of HBM into their own pools at start-up, and
+ *   latency-critical paths that must not take the implicit device synchronisation of
+ *   cudaMalloc / cudaFree. This entry point needs no workspace argument: its scratch is a
+ *   fixed array of FA_NOALLOC_SCRATCH_BYTES inside the library's device image, which
+ *   every GPU that loads the library holds until the process exits.
+ *   Arguments are those of fa_decode without workspace / workspace_bytes. num_splits <= 0
+ *   picks the split count fa_decode would pick, lowered until the scratch fits; a given
+ *   num_splits is used as is. If the scratch cannot hold even one split, the call
+ *   returns FA_ERR_UNSUPPORTED (message gives the bytes needed) and launches nothing.
+ *   Calls no cudaMalloc / cudaFree and no allocating library routine.
+ *   Set-up: the first call on each device (with that device current) looks up the
+ *   device address of the scratch array; make that first call before any stream
+ *   capture begins.
+ *   All calls in the process share one scratch array per device and it keeps the last
+ *   call's contents; the kernels write every scratch word before reading it, so nothing
+ *   needs clearing. Calls whose kernels overlap on the same GPU (different streams, no
+ *   ordering between them) race on the scratch and give wrong results.
+ */
+#define FA_NOALLOC_SCRATCH_BYTES (16u << 20)
+int fa_decode_noalloc(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
+                      int32_t out_dtype, int32_t num_splits, void* stream);
+
+/*
  * fa_device_status -- synchronise `stream`, then read and clear the library's kernel
  * watchdog word. Returns FA_OK if no kernel launched since the last call hit a wait
  * limit, FA_ERR_DEVICE (message names the kernel and wait) if one did, FA_ERR_CUDA if

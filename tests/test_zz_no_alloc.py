@@ -1,0 +1,79 @@
+"""fa_decode_noalloc: a decode step for callers that cannot allocate device memory.
+
+Some callers cannot call cudaMalloc or hand the library a scratch buffer: plug-ins inside
+a framework that owns every device allocation, serving loops that pooled all of HBM at
+start-up, and latency-critical paths that must not take cudaMalloc's implicit device
+synchronisation. fa_decode_noalloc serves them with a fixed scratch array built into the
+library. These tests call it through the C ABI and compare its output with fa_decode's
+(caller-provided workspace) on two calls in a row, so the second call runs on the scratch
+contents the first one left behind. The file is named to be collected last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import fourier_basis_attention_b200 as fa
+import workloads as wl
+
+pytestmark = pytest.mark.gpu
+TOL = 3e-3
+
+
+def _setup(w):
+    mask = wl.dim_mask(w)
+    dev = "cuda"
+    K = wl.kv_cache(w, "K", device=dev)
+    V = wl.kv_cache(w, "V", device=dev)
+    q = wl.queries(w, device=dev)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    cache = fa.Cache(p)
+    fa.fa_compress(p, K, V, fa.basis_table(p), cache)
+    return p, cache, q
+
+
+def _reference(p, cache, q, w, num_splits):
+    ws = torch.empty(fa.fa_decode_workspace_size(p, num_splits), dtype=torch.uint8, device="cuda")
+    ref = torch.empty(w.B, w.Hq, 128, dtype=torch.float32, device="cuda")
+    fa.fa_decode(p, q, cache, ref, ws, num_splits)
+    torch.cuda.synchronize()
+    return ref
+
+
+@pytest.mark.parametrize("w,num_splits", [
+    (wl.shrink(wl.LLAMA3_8B_GQA_32K, B=2, Hq=8, Hkv=2, L=2000), 0),
+    (wl.shrink(wl.LLAMA3_8B_GQA_32K, B=2, Hq=8, Hkv=2, L=2000), 5),
+    (wl.LLAMA2_7B_MHA_32K, 0),
+], ids=["small_auto", "small_forced_splits", "llama2_7b_full_auto"])
+def test_noalloc_matches_fa_decode_on_two_calls(w, num_splits):
+    p, cache, q = _setup(w)
+    ref = _reference(p, cache, q, w, num_splits)
+    scale = ref.abs().max().item()
+    for call in range(2):
+        out = torch.full((w.B, w.Hq, 128), float("nan"), dtype=torch.float32, device="cuda")
+        rc = fa.LIB.fa_decode_noalloc(ctypes.byref(p), q.data_ptr(), ctypes.byref(cache.c),
+                                      out.data_ptr(), fa.FA_F32, num_splits,
+                                      torch.cuda.current_stream().cuda_stream)
+        assert rc == fa.FA_OK, fa.fa_last_error()
+        fa.fa_device_status()
+        err = (out - ref).abs().max().item()
+        assert np.isfinite(err) and err <= TOL * scale, (call, err, scale)
+    # bf16 output through the same entry point
+    out_bf = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device="cuda")
+    fa.fa_decode_noalloc(p, q, cache, out_bf, num_splits)
+    torch.cuda.synchronize()
+    assert (out_bf.float() - ref).abs().max().item() <= 2.0 ** -8 * scale + TOL * scale
+
+
+def test_noalloc_rejects_oversized_request():
+    """A split count whose records exceed the built-in scratch is refused before launch."""
+    w = wl.LLAMA3_8B_GQA_128K
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    ns = 400
+    assert fa.fa_decode_workspace_size(p, ns) > fa.NOALLOC_SCRATCH_BYTES
+    cache = fa.fa_cache(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    rc = fa.LIB.fa_decode_noalloc(ctypes.byref(p), 0x1000, ctypes.byref(cache), 0x1000,
+                                  fa.FA_F32, ns, None)
+    assert rc == fa.FA_ERR_UNSUPPORTED
+    assert "bytes of scratch" in fa.fa_last_error()
