@@ -42,6 +42,9 @@ def parse():
     ap.add_argument("--workload", default="llama2_7b_mha_b8_L32768_k255")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
+    ap.add_argument("--no-clock-probe", action="store_true",
+                    help="skip the extra clock-sampling loop after a short timed region")
     return ap.parse_args()
 
 
@@ -246,6 +249,8 @@ def run_ours(args):
                                 device_id=torch.device("cuda", local))
 
     base = workload_by_name(args.workload)
+    if args.batch > 0:
+        base = wl.shrink(base, B=args.batch)
     w = wl.shrink(base, seed=base.seed + 1000 * rank) if rank else base
     mask = wl.dim_mask(base)
     dev = torch.device("cuda", local)
@@ -296,7 +301,7 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     rows = sampler.stop()
     clock_note = "sampled during the timed region"
-    if len([r for r in rows if r["power"] > 200.0]) < 3:
+    if len([r for r in rows if r["power"] > 200.0]) < 3 and not args.no_clock_probe:
         # timed region too short for the 100 ms sampler: sample the same step for ~1 s more
         sampler2 = ClockSampler(gpu_index)
         sampler2.start()

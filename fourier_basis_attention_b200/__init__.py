@@ -67,7 +67,11 @@ def _load() -> ctypes.CDLL:
         path = _build.build()
     if not os.path.exists(path):
         raise ImportError(f"{path} is missing; run fourier_basis_attention_b200._build.build()")
-    lib = ctypes.CDLL(path)
+    return configure(ctypes.CDLL(path))
+
+
+def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Declare the C signatures on a loaded copy of the library."""
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.fa_plan_init.argtypes = [ctypes.POINTER(fa_shape), P, ctypes.POINTER(fa_plan)]
     lib.fa_build_basis.argtypes = [I32, I32, I32, I32, P, I64, P]

@@ -8,15 +8,18 @@
 //     E_X = X[S : S+M, retained dims]                     (bit-exact copy)
 //     F_X = X[sink and recent tokens, all dims]           (bit-exact copy)
 //
-// GEMM mapping (one CTA per 128-coefficient tile x head x {K, V}):
-//   D[128 coefs x 128 dims] += A[128 coefs x 64 tokens] . B[64 tokens x 128 dims]
-//   A = Phi^T tile, K-major (tokens contiguous), loaded by TMA with 128-byte swizzle.
-//   B = cache rows, MN-major (dims contiguous, the cache's own layout), two 64-dim TMA
-//       boxes per stage. The full 128 dims are multiplied; the epilogue keeps the masked
-//       ones (a column gather on the B side is not expressible as a TMA box).
-//   D lives in tensor memory (128 lanes x 128 fp32 columns).
-// Warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread), warps 2-5 pack
-// the retained dims of every stage (coefficient tile 0 only) and run the epilogue.
+// GEMM mapping: one CTA per (batch b, KV head g, pair of 128-coefficient tiles) computes
+// the coefficients of K and V together:
+//   D_kt[128 coefs x 256] += A_kt[128 coefs x 64 tokens] . B[64 tokens x (128 K dims | 128 V dims)]
+//   A = unit-amplitude basis table tile, K-major (tokens contiguous), TMA, 128-byte swizzle.
+//   B = the cache rows of K and V, MN-major (dims contiguous: the cache's own layout), four
+//       64-dim TMA boxes per stage. One N = 256 MMA covers K and V, so a cache row is read
+//       from memory once for k <= 256 and the table tile feeds both.
+//   D lives in tensor memory: 2 tiles x 256 fp32 columns = all 512 columns of the SM.
+// All 128 dims are multiplied; the epilogue keeps the masked ones (a column gather on the
+// B side is not expressible as a TMA box).
+// Warp roles: warp 0 issues TMA, warp 1 issues tcgen05.mma (one thread), warps 2-9 pack
+// the retained dims of every stage (first tile pair only) and run the epilogue.
 // Tokens past the middle span read a zero A (TMA out-of-bounds fill), so the ragged last
 // stage needs no masking. A holds unit-amplitude cos / sin (DC = 1); each accumulator row
 // is scaled by its orthonormal factor (1/sqrt(M) or sqrt(2/M)) in fp32 in the epilogue.
@@ -27,20 +30,32 @@
 
 namespace fa {
 
-constexpr int CK_BM = 128;
-constexpr int CK_BN = 128;
-constexpr int CK_BK = 64;
-constexpr int CK_STAGES = 4;
-constexpr int CK_A_BYTES = CK_BM * CK_BK * 2;
-constexpr int CK_B_BYTES = CK_BN * CK_BK * 2;
-constexpr int CK_STAGE_BYTES = CK_A_BYTES + CK_B_BYTES;
-constexpr int CK_THREADS = 192;
-constexpr int CK_STAGE_LD = CK_BN + 4;  // fp32 staging row stride (bank-conflict free)
-constexpr int CK_SMEM = CK_STAGES * CK_STAGE_BYTES + 1024 /*align*/ + 1024 /*misc*/;
-static_assert(CK_BM * CK_STAGE_LD * 4 <= CK_STAGES * CK_STAGE_BYTES, "staging fits");
+constexpr int CK_BM = 128;                   // coefficient rows per tile (MMA M)
+constexpr int CK_BK = 64;                    // tokens per stage
+constexpr int CK_BN = 2 * FA_HEAD_DIM;       // K dims | V dims (MMA N)
+constexpr int CK_A_TILE = CK_BM * CK_BK * 2; // 16 KB per coefficient tile
+constexpr int CK_B_BOX = 64 * CK_BK * 2;     // 8 KB per 64-dim box
+constexpr int CK_B_BYTES = 4 * CK_B_BOX;     // 32 KB
+constexpr int CK_THREADS = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 pack + epilogue
+constexpr int CK_PACK_WARPS = 8;
+constexpr int CK_STAGE_LD = CK_BN + 4;       // fp32 staging row stride (bank-conflict free)
+constexpr int CK_PREFETCH = 8;               // stages of K / V rows prefetched into L2 ahead
+
+template <int KT>
+struct CkCfg {
+  static constexpr int A_BYTES = KT * CK_A_TILE;
+  static constexpr int STAGE_BYTES = A_BYTES + CK_B_BYTES;
+  static constexpr int STAGES = KT == 2 ? 3 : 4;
+  static constexpr int TMEM_COLS = KT * CK_BN;
+  static constexpr int BASE_SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*misc*/;
+  static_assert(CK_BM * CK_STAGE_LD * 4 <= STAGES * STAGE_BYTES, "staging fits");
+};
+
 
 struct CompressParams {
-  int M, k, S, Hkv, n_ktiles;
+  int M, k, S, L, Hkv, n_ktiles, n_pairs;
+  const void* K;
+  const void* V;
   float norm_single, norm_pair;
   long long c_batch, e_batch;
   long long c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
@@ -60,19 +75,22 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+template <int KT>
 __global__ void __launch_bounds__(CK_THREADS, 1)
     compress_kernel(const __grid_constant__ CUtensorMap tm_phi,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CompressParams p) {
+  using Cfg = CkCfg<KT>;
+  constexpr int STAGES = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* misc = smem + CK_STAGES * CK_STAGE_BYTES;
+  uint8_t* misc = smem + STAGES * Cfg::STAGE_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(misc);
-  uint64_t* empty = full + CK_STAGES;
-  uint64_t* accum = empty + CK_STAGES;
+  uint64_t* empty = full + STAGES;
+  uint64_t* accum = empty + STAGES;
   uint64_t* drain = accum + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -80,33 +98,34 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int ktile = blockIdx.x % p.n_ktiles;
-  const int rest = blockIdx.x / p.n_ktiles;
-  const int which = rest & 1;  // 0 = K, 1 = V
-  const int head = rest >> 1;  // flattened b * Hkv + g
+  const int pair = blockIdx.x % p.n_pairs;
+  const int head = blockIdx.x / p.n_pairs;  // flattened b * Hkv + g
   const int b = head / p.Hkv;
   const int g = head - b * p.Hkv;
   const int dc = p.dc[g];
-  const bool do_pack = (ktile == 0);
+  const int kt0 = pair * KT;                       // first coefficient tile of this CTA
+  const int kt_n = min(KT, p.n_ktiles - kt0);       // tiles present (>= 1)
+  const bool do_pack = (pair == 0);
   const int nk = (p.M + CK_BK - 1) / CK_BK;
-  // A head with no compressed dims needs only the packing pass of tile 0.
-  if (dc == 0 && ktile != 0) return;
+  // A head with no compressed dims needs only the packing pass of the first pair.
+  if (dc == 0 && pair != 0) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < CK_STAGES; ++s) {
+    for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + (do_pack ? 4 : 0));
+      mbar_init(&empty[s], 1 + (do_pack ? CK_PACK_WARPS : 0));
     }
     mbar_init(accum, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_phi);
-    prefetch_tmap(which ? &tm_v : &tm_k);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
   }
   if (threadIdx.x < FA_HEAD_DIM) perm_s[threadIdx.x] = p.perm[g][threadIdx.x];
   if (warp == 1) {
-    tmem_alloc(tmem_slot, CK_BN);
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -117,30 +136,48 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      const CUtensorMap* tm_x = which ? &tm_v : &tm_k;
+      const uint32_t tx = (uint32_t)(kt_n * CK_A_TILE + CK_B_BYTES);
+      // K / V rows of this head are contiguous (256 bytes per token): pull them into L2
+      // CK_PREFETCH stages ahead of their TMA loads so that those see L2, not DRAM, latency.
+      const char* k_rows = static_cast<const char*>(p.K) + (long long)head * p.L * (FA_HEAD_DIM * 2);
+      const char* v_rows = static_cast<const char*>(p.V) + (long long)head * p.L * (FA_HEAD_DIM * 2);
+      auto prefetch_stage = [&](int st) {
+        const int t = p.S + st * CK_BK;
+        const int n = min(CK_BK, p.L - t);
+        if (n > 0) {
+          prefetch_l2_bulk(k_rows + (long long)t * (FA_HEAD_DIM * 2), (uint32_t)n * (FA_HEAD_DIM * 2));
+          prefetch_l2_bulk(v_rows + (long long)t * (FA_HEAD_DIM * 2), (uint32_t)n * (FA_HEAD_DIM * 2));
+        }
+      };
+      for (int st = 0; st < CK_PREFETCH && st < nk; ++st) prefetch_stage(st);
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
-        const int s = it % CK_STAGES;
-        const uint32_t use = (uint32_t)(it / CK_STAGES);
-        if (it >= CK_STAGES &&
+        if (it + CK_PREFETCH < nk) prefetch_stage(it + CK_PREFETCH);
+        const int s = it % STAGES;
+        const uint32_t use = (uint32_t)(it / STAGES);
+        if (it >= STAGES &&
             !mbar_wait(&empty[s], (use & 1u) ^ 1u, abort_flag, WD_COMPRESS | 1u))
           break;
-        uint8_t* a_s = stages + s * CK_STAGE_BYTES;
-        uint8_t* b_s = a_s + CK_A_BYTES;
-        mbar_arrive_expect_tx(&full[s], CK_STAGE_BYTES);
-        tma_load_2d(a_s, &tm_phi, &full[s], it * CK_BK, ktile * CK_BM);
-        tma_load_3d(b_s, tm_x, &full[s], 0, p.S + it * CK_BK, head);
-        tma_load_3d(b_s + CK_B_BYTES / 2, tm_x, &full[s], 64, p.S + it * CK_BK, head);
+        uint8_t* a_s = stages + s * Cfg::STAGE_BYTES;
+        uint8_t* b_s = a_s + Cfg::A_BYTES;
+        const int t = p.S + it * CK_BK;
+        mbar_arrive_expect_tx(&full[s], tx);
+        for (int kt = 0; kt < kt_n; ++kt)
+          tma_load_2d(a_s + kt * CK_A_TILE, &tm_phi, &full[s], it * CK_BK, (kt0 + kt) * CK_BM);
+        tma_load_3d(b_s, &tm_k, &full[s], 0, t, head);
+        tma_load_3d(b_s + CK_B_BOX, &tm_k, &full[s], 64, t, head);
+        tma_load_3d(b_s + 2 * CK_B_BOX, &tm_v, &full[s], 0, t, head);
+        tma_load_3d(b_s + 3 * CK_B_BOX, &tm_v, &full[s], 64, t, head);
         ++issued;
       }
       if (*abort_flag) {
         // let the copies already issued land before shared memory goes away
-        for (int it = (issued > CK_STAGES ? issued - CK_STAGES : 0); it < issued; ++it)
-          drain_wait(&full[it % CK_STAGES], (uint32_t)(it / CK_STAGES) & 1u);
+        for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
+          drain_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u);
       } else {
         // tail: every stage's last release (MMA commit + pack arrivals) has landed
-        for (int it = (nk > CK_STAGES ? nk - CK_STAGES : 0); it < nk; ++it)
-          mbar_wait(&empty[it % CK_STAGES], (uint32_t)(it / CK_STAGES) & 1u, abort_flag,
+        for (int it = (nk > STAGES ? nk - STAGES : 0); it < nk; ++it)
+          mbar_wait(&empty[it % STAGES], (uint32_t)(it / STAGES) & 1u, abort_flag,
                     WD_COMPRESS | 5u);
       }
     }
@@ -150,22 +187,27 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(CK_BM, CK_BN, /*b_mn_major=*/true);
       bool ok = true;
       for (int it = 0; it < nk; ++it) {
-        const int s = it % CK_STAGES;
-        if (!mbar_wait(&full[s], (uint32_t)(it / CK_STAGES) & 1u, abort_flag, WD_COMPRESS | 2u)) {
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(it / STAGES) & 1u, abort_flag, WD_COMPRESS | 2u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(stages + s * CK_STAGE_BYTES);
-        const uint32_t b_addr = a_addr + CK_A_BYTES;
+        const uint32_t a_addr = smem_u32(stages + s * Cfg::STAGE_BYTES);
+        const uint32_t b_addr = a_addr + Cfg::A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < CK_BK / 16; ++kk) {
-          // A: 16 tokens = 32 bytes further along the swizzled 128-byte row.
-          const uint64_t ad = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
-          // B: 16 tokens = two 8-row groups of 128-byte rows; the 64-dim halves are
-          // CK_B_BYTES/2 apart (leading byte offset).
-          const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, CK_B_BYTES / 2, 1024);
-          mma_bf16(tmem_d, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+          // B: 16 tokens = two 8-row groups of 128-byte rows; the four 64-dim boxes are
+          // CK_B_BOX apart (leading byte offset).
+          const uint64_t bd = smem_desc_sw128(b_addr + kk * 2048, CK_B_BOX, 1024);
+#pragma unroll
+          for (int kt = 0; kt < KT; ++kt) {
+            if (kt < kt_n) {
+              // A: 16 tokens = 32 bytes further along the swizzled 128-byte row.
+              const uint64_t ad = smem_desc_sw128(a_addr + kt * CK_A_TILE + kk * 32, 16, 1024);
+              mma_bf16(tmem_d + kt * CK_BN, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+            }
+          }
         }
         mma_commit(&empty[s]);
       }
@@ -180,87 +222,114 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
     }
   } else {
     // ---------------------------------------------------------------- pack + epilogue
-    const int et = threadIdx.x - 64;  // 0..127
+    const int et = threadIdx.x - 64;  // 0..255
+    const int pw = warp - 2;          // 0..7
     if (do_pack) {
+      // Lane i of every pack warp owns retained dims i, i + 32, ... of the head; warp pw
+      // owns tokens pw, pw + 8, ... of each stage. Source offsets inside the swizzled B
+      // boxes are fixed per dim; only the row and its swizzle phase change per token.
+      // Shared memory is close to saturated by the MMA operand reads and the TMA fills,
+      // so each warp issues all of a stage's loads back to back (one exposed latency per
+      // stage), then writes the rows as coalesced 64-byte global stores.
       const int de = FA_HEAD_DIM - dc;
       const int de_ld = p.de_ld[g];
-      const int nchunk = de_ld >> 3;
-      __nv_bfloat16* E = p.E[which] + (long long)b * p.e_batch + p.e_off[g];
+      const int ngrp = (de_ld + 31) >> 5;  // 32-dim groups per row
+      __nv_bfloat16* const E0 = p.E[0] + (long long)b * p.e_batch + p.e_off[g];
+      __nv_bfloat16* const E1 = p.E[1] + (long long)b * p.e_batch + p.e_off[g];
+      constexpr int TPW = CK_BK / CK_PACK_WARPS;  // tokens per warp per stage
       for (int it = 0; it < nk; ++it) {
-        const int s = it % CK_STAGES;
-        if (!mbar_wait(&full[s], (uint32_t)(it / CK_STAGES) & 1u, abort_flag, WD_COMPRESS | 3u))
+        const int s = it % STAGES;
+        if (!mbar_wait(&full[s], (uint32_t)(it / STAGES) & 1u, abort_flag, WD_COMPRESS | 3u))
           break;
-        const uint8_t* b_s = stages + s * CK_STAGE_BYTES + CK_A_BYTES;
+        const uint8_t* b_s = stages + s * Cfg::STAGE_BYTES + Cfg::A_BYTES;
         const int ntok = min(CK_BK, p.M - it * CK_BK);
-        for (int c = et; c < ntok * nchunk; c += 128) {
-          const int tau = c / nchunk;
-          const int q = c - tau * nchunk;
-          uint32_t w[4];
-#pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            uint32_t lohi[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int i = q * 8 + e2 * 2 + h;
-              uint32_t bits = 0;
-              if (i < de) {
-                const int d = perm_s[dc + i];
-                const int half = d >> 6;
-                const int col = d & 63;
-                // 128-byte swizzle: 16-byte chunk index XOR (row mod 8)
-                const int off = half * (CK_B_BYTES / 2) + tau * 128 +
-                                ((((col >> 3) ^ (tau & 7)) << 4) | ((col & 7) << 1));
-                bits = *reinterpret_cast<const unsigned short*>(b_s + off);
-              }
-              lohi[h] = bits;
-            }
-            w[e2] = lohi[0] | (lohi[1] << 16);
+        for (int c = 0; c < ngrp; ++c) {
+          const int i = lane + 32 * c;
+          int boff = -1, cbit = 0;
+          if (i < de) {
+            const int d = perm_s[dc + i];
+            boff = (d >> 6) * CK_B_BOX + ((d & 7) << 1);
+            cbit = (d & 63) >> 3;
           }
-          *reinterpret_cast<uint4*>(E + (long long)(it * CK_BK + tau) * de_ld + q * 8) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+          unsigned short v[2][TPW];
+#pragma unroll
+          for (int x = 0; x < 2; ++x)
+#pragma unroll
+            for (int j = 0; j < TPW; ++j) {
+              const int tau = pw + j * CK_PACK_WARPS;
+              v[x][j] = 0;
+              if (boff >= 0 && tau < ntok)
+                v[x][j] = *reinterpret_cast<const unsigned short*>(
+                    b_s + x * 2 * CK_B_BOX + tau * 128 + boff + ((cbit ^ (tau & 7)) << 4));
+            }
+          if (i < de_ld) {
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+              for (int j = 0; j < TPW; ++j) {
+                const int tau = pw + j * CK_PACK_WARPS;
+                if (tau < ntok)
+                  reinterpret_cast<unsigned short*>((x ? E1 : E0) +
+                                                    (long long)(it * CK_BK + tau) * de_ld)[i] =
+                      v[x][j];
+              }
+          }
         }
+        // the stage's shared-memory values have been consumed: it may be refilled
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (lane == 0) mbar_arrive_relaxed(&empty[s]);
       }
     }
-    // all four warps are done reading the stages before any staging write reuses them
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    const int acc_ready = (dc > 0 && !*abort_flag) ? (mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u) ? 1 : 0) : 0;
-    if (dc > 0 && bar1_and_128(acc_ready)) {
+    // all pack warps are done reading the stages before any staging write reuses them
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const int acc_ready =
+        (dc > 0 && !*abort_flag) ? (mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u) ? 1 : 0) : 0;
+    if (dc > 0 && bar1_and_256(acc_ready)) {
       tc_fence_after();
       float* stage_f = reinterpret_cast<float*>(stages);
-      const int rb = warp & 3;  // TMEM lanes this warp may access: 32*rb .. 32*rb+31
+      const int rb = warp & 3;       // TMEM lanes this warp may access: 32*rb .. 32*rb+31
+      const int half = pw >> 2;      // warps 2-5: K columns, warps 6-9: V columns
       const int row = rb * 32 + lane;
-#pragma unroll
-      for (int cb = 0; cb < CK_BN / 32; ++cb) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(rb * 32) << 16) + cb * 32, r);
-        tmem_ld_wait();
-        float4* dst = reinterpret_cast<float4*>(stage_f + row * CK_STAGE_LD + cb * 32);
-#pragma unroll
-        for (int v = 0; v < 8; ++v)
-          dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                               __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-      }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
       const int dc_ld = p.dc_ld[g];
       const int nchunk = dc_ld >> 2;
-      float* C = p.C[which] + (long long)b * p.c_batch + p.c_off[g];
-      const int rows = min(CK_BM, p.k - ktile * CK_BM);
-      for (int c = et; c < rows * nchunk; c += 128) {
-        const int r = c / nchunk;
-        const int q = c - r * nchunk;
-        const int j = ktile * CK_BM + r;
-        const int f = (j + 1) >> 1;
-        const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
-        float v[4];
+      const int per_x = CK_BM * nchunk;
+      float* const C0 = p.C[0] + (long long)b * p.c_batch + p.c_off[g];
+      float* const C1 = p.C[1] + (long long)b * p.c_batch + p.c_off[g];
+      for (int kt = 0; kt < kt_n; ++kt) {
+        if (kt > 0) asm volatile("bar.sync 1, 256;" ::: "memory");  // staging reads done
+#pragma unroll 1
+        for (int cb = 0; cb < FA_HEAD_DIM / 32; ++cb) {
+          uint32_t r[32];
+          const int col = half * FA_HEAD_DIM + cb * 32;
+          tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(rb * 32) << 16) + kt * CK_BN + col, r);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(stage_f + row * CK_STAGE_LD + col);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = q * 4 + e;
-          v[e] = (i < dc) ? nrm * stage_f[r * CK_STAGE_LD + perm_s[i]] : 0.0f;
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
         }
-        *reinterpret_cast<float4*>(C + (long long)j * dc_ld + q * 4) =
-            make_float4(v[0], v[1], v[2], v[3]);
+        asm volatile("bar.sync 1, 256;" ::: "memory");
+        const int jt = (kt0 + kt) * CK_BM;
+        const int rows = min(CK_BM, p.k - jt);
+        for (int c = et; c < 2 * per_x; c += 256) {
+          const int x = c >= per_x ? 1 : 0;
+          const int rem = c - x * per_x;
+          const int r = rem / nchunk;
+          const int q = rem - r * nchunk;
+          if (r >= rows) continue;
+          const int j = jt + r;
+          const int f = (j + 1) >> 1;
+          const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+          float v[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = q * 4 + e;
+            v[e] = (i < dc) ? nrm * stage_f[r * CK_STAGE_LD + x * FA_HEAD_DIM + perm_s[i]] : 0.0f;
+          }
+          *reinterpret_cast<float4*>((x ? C1 : C0) + (long long)j * dc_ld + q * 4) =
+              make_float4(v[0], v[1], v[2], v[3]);
+        }
       }
     }
   }
@@ -269,7 +338,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_d, CK_BN);
+    tmem_dealloc(tmem_d, Cfg::TMEM_COLS);
   }
 }
 
@@ -378,6 +447,9 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   cp.M = plan->M;
   cp.k = sh.k;
   cp.S = plan->S;
+  cp.L = sh.L;
+  cp.K = K;
+  cp.V = V;
   cp.Hkv = sh.Hkv;
   cp.n_ktiles = (sh.k + CK_BM - 1) / CK_BM;
   cp.c_batch = plan->c_batch;
@@ -397,11 +469,21 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   cp.E[0] = static_cast<__nv_bfloat16*>(cache->E_K);
   cp.E[1] = static_cast<__nv_bfloat16*>(cache->E_V);
 
-  cudaError_t e = cudaFuncSetAttribute(compress_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, CK_SMEM);
-  if (e != cudaSuccess) return e;
-  const long long grid = (long long)cp.n_ktiles * 2 * n_heads;
-  compress_kernel<<<(unsigned)grid, CK_THREADS, CK_SMEM, stream>>>(tm_phi, tm_k, tm_v, cp);
+  // One tile per CTA when k <= 128, else pairs of tiles (512 TMEM columns).
+  const int KT = cp.n_ktiles >= 2 ? 2 : 1;
+  cp.n_pairs = (cp.n_ktiles + KT - 1) / KT;
+  const long long grid = (long long)cp.n_pairs * n_heads;
+  const int smem = KT == 2 ? CkCfg<2>::BASE_SMEM : CkCfg<1>::BASE_SMEM;
+  cudaError_t e;
+  if (KT == 2) {
+    e = cudaFuncSetAttribute(compress_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    compress_kernel<2><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
+  } else {
+    e = cudaFuncSetAttribute(compress_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    compress_kernel<1><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
+  }
   return cudaGetLastError();
 }
 
