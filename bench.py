@@ -45,6 +45,11 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--no-clock-probe", action="store_true",
                     help="skip the extra clock-sampling loop after a short timed region")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time every single-layer workload and the 32-layer LLaMA-3-8B decode "
+                         "sweep (one JSON line each) instead of the default bench line")
+    ap.add_argument("--sweep-points", default="",
+                    help="comma list of BxL points for the 32-layer sweep (default: all 12)")
     return ap.parse_args()
 
 
@@ -431,10 +436,132 @@ def K_bytes(w):
     return w.B * w.Hkv * w.L * 128 * 2
 
 
+def _time(fn, n, stream):
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def run_sweep(args):
+    """Per-workload timings (1 GPU): the four single-layer workloads, then the 32-layer
+    LLaMA-3-8B-shaped cache: compress every layer (distinct seeded masks), and time one
+    decode step over all 32 layers for each batch x context point."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, _ = load_peaks()
+    hbm = peaks["hbm_gbs"]
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    for w in wl.CONFIGS:
+        mask = wl.dim_mask(w)
+        K = wl.kv_cache(w, "K", device=dev)
+        V = wl.kv_cache(w, "V", device=dev)
+        q = wl.queries(w, device=dev)
+        plan = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+        cache = fa.Cache(plan, device=dev)
+        phiT = torch.empty(w.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(fa.fa_decode_workspace_size(plan), dtype=torch.uint8, device=dev)
+        out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+        basis = lambda: fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
+        comp = lambda: fa.fa_compress(plan, K, V, phiT, cache, stream)
+        dec = lambda: fa.fa_decode(plan, q, cache, out, ws, 0, stream)
+        for f in (basis, comp, dec):
+            f(); f(); f()
+        tb = _time(basis, 10, stream)
+        tcmp = _time(comp, 10, stream)
+        td = _time(dec, 20, stream)
+        fa.fa_device_status(stream)
+        wm = work_model(w, plan)
+        print(json.dumps({"sweep": "single_layer", "workload": w.name, "basis_us": tb * 1e3,
+                          "compress_us": tcmp * 1e3,
+                          "compress_tflops": wm["compress_flops"] / tcmp / 1e9,
+                          "compress_hbm_gbs": wm["compress_bytes"] / tcmp / 1e6,
+                          "compress_frac_tensor": wm["compress_flops"] / tcmp / 1e9 / tc,
+                          "compress_frac_hbm": wm["compress_bytes"] / tcmp / 1e6 / hbm,
+                          "decode_us": td * 1e3, "decode_hbm_gbs": wm["decode_bytes"] / td / 1e6,
+                          "decode_frac_hbm": wm["decode_bytes"] / td / 1e6 / hbm,
+                          "decode_fp32_tflops": wm["decode_flops"] / td / 1e9}), flush=True)
+        del K, V, cache, ws, out, phiT
+        torch.cuda.empty_cache()
+
+    points = [(B, L) for L in wl.SWEEP_L for B in wl.SWEEP_BATCH]
+    if args.sweep_points:
+        points = [tuple(int(x) for x in p.split("x")) for p in args.sweep_points.split(",")]
+    for B, L in points:
+        w0 = wl.llama3_8b_layer(B, L, 0)
+        K = wl.kv_cache(w0, "K", device=dev)
+        V = wl.kv_cache(w0, "V", device=dev)
+        q = wl.queries(w0, device=dev)
+        plans, caches, t_comp = [], [], []
+        free, _ = torch.cuda.mem_get_info(dev)
+        phiT = None
+        resident = 0
+        for layer in range(32):
+            wlay = wl.llama3_8b_layer(B, L, layer)
+            plan = fa.fa_plan_init(B, 32, 8, L, wlay.S, wlay.R, wlay.k, wl.dim_mask(wlay))
+            need = 2 * (plan.f_elems * 2 + plan.e_elems * 2 + plan.c_elems * 4)
+            free, _ = torch.cuda.mem_get_info(dev)
+            if need > free - (4 << 30) and resident > 0:
+                plans.append(plan)  # cycled: reuses an earlier layer's buffers
+                caches.append(caches[layer % resident])
+            else:
+                cache = fa.Cache(plan, device=dev)
+                plans.append(plan)
+                caches.append(cache)
+                resident += 1
+            if phiT is None:
+                phiT = torch.empty(wlay.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
+                fa.fa_build_basis(plan.M, wlay.k, phiT, plan.phi_ld, False, stream)
+            # the K / V of every layer are the same synthetic draw (its mask differs); the
+            # compress cost does not depend on the values
+            fa.fa_compress(plan, K, V, phiT, caches[-1], stream)
+            t_comp.append(_time(lambda: fa.fa_compress(plan, K, V, phiT, caches[-1], stream), 1, stream))
+        del K, V
+        torch.cuda.empty_cache()
+        ws = torch.empty(max(fa.fa_decode_workspace_size(p) for p in plans), dtype=torch.uint8, device=dev)
+        out = torch.empty(B, 32, 128, dtype=torch.bfloat16, device=dev)
+
+        def step():
+            for p, c in zip(plans, caches):
+                fa.fa_decode(p, q, c, out, ws, 0, stream)
+        step()
+        n = 3 if B * L >= 32 * 131072 else 10
+        td = _time(step, n, stream)
+        fa.fa_device_status(stream)
+        wms = [work_model(wl.llama3_8b_layer(B, L, l), p) for l, p in enumerate(plans)]
+        dbytes = sum(m["decode_bytes"] for m in wms)
+        cflops = sum(m["compress_flops"] for m in wms)
+        cbytes = sum(m["compress_bytes"] for m in wms)
+        tcomp = sum(t_comp)
+        print(json.dumps({"sweep": "llama3_8b_32_layers", "B": B, "L": L, "k": w0.k,
+                          "layers_resident": resident, "layers": 32,
+                          "compress_us_32_layers": tcomp * 1e3,
+                          "compress_tflops": cflops / tcomp / 1e9,
+                          "compress_frac_hbm": cbytes / tcomp / 1e6 / hbm,
+                          "decode_us_per_step": td * 1e3,
+                          "decode_hbm_gbs": dbytes / td / 1e6,
+                          "decode_frac_hbm": dbytes / td / 1e6 / hbm}), flush=True)
+        del caches, plans, ws, out, q, phiT
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.sweep:
+        run_sweep(args)
     else:
         run_ours(args)
 

@@ -26,7 +26,8 @@ FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE = range(5)
 FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode_workspace_size",
-            "fa_decode", "fa_decode_noalloc", "fa_device_status", "fa_last_error")
+            "fa_decode", "fa_decode_noalloc", "fa_device_status", "fa_watchdog_selftest",
+            "fa_last_error")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -83,10 +84,11 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_decode_noalloc.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32,
                                       I32, P]
     lib.fa_device_status.argtypes = [P]
+    lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint32, P]
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
     for name in ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode", "fa_decode_noalloc",
-                 "fa_device_status"):
+                 "fa_device_status", "fa_watchdog_selftest"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -173,6 +175,11 @@ def fa_decode_noalloc(plan: fa_plan, q, cache: "Cache", out, num_splits: int = 0
 
 def fa_device_status(stream=None) -> None:
     _check(LIB.fa_device_status(_stream(stream)))
+
+
+def fa_watchdog_selftest(wait_ns: int = 20_000_000, stream=None) -> None:
+    """Launch a kernel whose bounded wait must expire (see the C header)."""
+    _check(LIB.fa_watchdog_selftest(wait_ns, _stream(stream)))
 
 
 # ----------------------------------------------------------------------------- marshalling helpers

@@ -209,6 +209,14 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
   return FA_OK;
 }
 
+int fa_watchdog_selftest(uint32_t wait_ns, void* stream) {
+  if (wait_ns < 1000u || wait_ns > 1000000000u)
+    return fail(FA_ERR_INVALID, "wait_ns=%u outside [1 us, 1 s]", wait_ns);
+  cudaError_t e = fa::launch_watchdog_selftest(wait_ns, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_watchdog_selftest: launch");
+  return FA_OK;
+}
+
 int fa_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: stream");

@@ -361,7 +361,25 @@ __global__ void __launch_bounds__(256) copy_sink_recent_kernel(
   }
 }
 
+// One thread waits on an mbarrier that expects an arrival nobody makes; the bounded wait
+// expires after `limit_ns`, records WD_SELFTEST and the kernel returns.
+__global__ void watchdog_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+    mbar_wait(&bar, 0, &abort_flag, WD_SELFTEST | 1u, limit_ns);
+  }
+}
+
 // ------------------------------------------------------------------------- host side
+cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream) {
+  watchdog_selftest_kernel<<<1, 32, 0, stream>>>((unsigned long long)wait_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t read_and_clear_watchdog(unsigned int* word) {
   cudaError_t e = cudaMemcpyFromSymbol(word, g_watchdog, sizeof(unsigned int));
   if (e != cudaSuccess) return e;

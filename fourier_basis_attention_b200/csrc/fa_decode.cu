@@ -126,7 +126,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   const int hi = min(p.M, lo + p.split_len);
   const int M = p.M;
 
-  float* Ws = sm;                           // [F_pad][HL][2]
+  float* Ws = sm;                           // [F_pad][cos | sin][HL]
   float* qes = Ws + p.F_pad * HL * 2;       // [HL][128]
   float* ps = qes + HL * FA_HEAD_DIM;       // [DT][HL]
   float* red = ps + DT * HL;                // [4][DT][HL]
@@ -156,7 +156,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   }
   __syncthreads();
   for (int idx = tid; idx < p.F_pad * HL * 2; idx += DNT) {
-    const int f = idx >> 4, i = (idx >> 1) & 7, c = idx & 1;
+    const int f = idx >> 4, c = (idx >> 3) & 1, i = idx & 7;  // [f][cos | sin][head]
     const int gh = gh_s[i];
     Ws[idx] = (gh >= 0 && f < p.F) ? p.qw[(long long)gh * p.qw_stride + FA_HEAD_DIM + 2 * f + c]
                                    : 0.0f;
@@ -183,24 +183,26 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   // u role: slots ui + j * NTU, token group uq
   const int ui = tid % p.NTU, uq = tid / p.NTU;
   const int UT = DT / p.TG;
-  float uacc[SPT][HL][2];
+  // u accumulators, heads in pairs (paired fp32 FMA): ucs[j][hp] = cos sums of heads 2hp, 2hp+1,
+  // uss[j][hp] = sin sums
+  float2 ucs[SPT][HL / 2], uss[SPT][HL / 2];
   float cb[SPT], sb[SPT];
 #pragma unroll
   for (int j = 0; j < SPT; ++j) {
     phase_sincos((long long)(ui + j * p.NTU) % M, M, p.two_over_M, &sb[j], &cb[j]);
 #pragma unroll
-    for (int h = 0; h < HL; ++h) uacc[j][h][0] = uacc[j][h][1] = 0.0f;
+    for (int hp = 0; hp < HL / 2; ++hp) ucs[j][hp] = uss[j][hp] = make_float2(0.0f, 0.0f);
   }
   // exact-dim value role: head ie, 8-dim chunk ce, token group qg
   const int ei = tid % (HL * p.DEC), qg = tid / (HL * p.DEC);
   const int ie = ei / p.DEC, ce = ei - (ei / p.DEC) * p.DEC;
   const bool e_on = gh_s[ie] >= 0 && ce * 8 < deld_s[ie];
-  const long long ebe = ebase_s[ie];
   const int dle = deld_s[ie];
   const int ET = DT / p.TGE;
   float acce[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acce[e] = 0.0f;
+  const long long ebe = ebase_s[ie];
 
   for (int t0 = lo; t0 < hi; t0 += DT) {
     const int nt = min(DT, hi - t0);
@@ -208,18 +210,28 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     if (tid < 2 * HL) {
       const int i = (tid & 7);
       const int tn = t0 + DT;
-      if (gh_s[i] >= 0 && (i % p.G) == 0 && tn < hi) {
+      if (gh_s[i] >= 0 && (i % p.G) == 0 && tn < hi && deld_s[i] > 0) {
         const int nb = min(DT, hi - tn);
         const __nv_bfloat16* base = (tid < HL ? p.EK : p.EV) + ebase_s[i] + (long long)tn * deld_s[i];
         prefetch_l2_bulk(base, (uint32_t)(nb * deld_s[i] * 2));
       }
     }
     // ---------------------------------------------------------------- scores
-    float part[HL];
+    float2 part2[HL / 2];
 #pragma unroll
-    for (int h = 0; h < HL; ++h) part[h] = 0.0f;
+    for (int hp = 0; hp < HL / 2; ++hp) part2[hp] = make_float2(0.0f, 0.0f);
     const int tm = t0 + tau;
     if (tau < nt) {
+      // the first 32 exact dims of both rows are loaded up front so that their latency
+      // hides behind the basis loop
+      uint4 ek0[4], ek1[4];
+      const __nv_bfloat16* row0 = p.EK + eb0 + (long long)tm * dl0;
+      const __nv_bfloat16* row1 = p.EK + eb1 + (long long)tm * dl1;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        ek0[c8] = (v0 && c8 * 8 < dl0) ? *reinterpret_cast<const uint4*>(row0 + c8 * 8) : make_uint4(0, 0, 0, 0);
+        ek1[c8] = (v1 && c8 * 8 < dl1) ? *reinterpret_cast<const uint4*>(row1 + c8 * 8) : make_uint4(0, 0, 0, 0);
+      }
       if (fb < fe) {
         float sa, ca;
         phase_sincos(tm, M, p.two_over_M, &sa, &ca);
@@ -229,15 +241,16 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
           const int f1 = min(fe, f0 + 32);
           for (int f = f0; f < f1; ++f) {
             const float4* w4 = reinterpret_cast<const float4*>(Ws + f * (HL * 2));
-            const float4 a = w4[0], bq = w4[1], cq = w4[2], dq = w4[3];
-            part[0] += c * a.x + s * a.y;
-            part[1] += c * a.z + s * a.w;
-            part[2] += c * bq.x + s * bq.y;
-            part[3] += c * bq.z + s * bq.w;
-            part[4] += c * cq.x + s * cq.y;
-            part[5] += c * cq.z + s * cq.w;
-            part[6] += c * dq.x + s * dq.y;
-            part[7] += c * dq.z + s * dq.w;
+            const float4 wc0 = w4[0], wc1 = w4[1], ws0 = w4[2], ws1 = w4[3];
+            const float2 cc = make_float2(c, c), ss = make_float2(s, s);
+            part2[0] = __ffma2_rn(cc, make_float2(wc0.x, wc0.y), part2[0]);
+            part2[1] = __ffma2_rn(cc, make_float2(wc0.z, wc0.w), part2[1]);
+            part2[2] = __ffma2_rn(cc, make_float2(wc1.x, wc1.y), part2[2]);
+            part2[3] = __ffma2_rn(cc, make_float2(wc1.z, wc1.w), part2[3]);
+            part2[0] = __ffma2_rn(ss, make_float2(ws0.x, ws0.y), part2[0]);
+            part2[1] = __ffma2_rn(ss, make_float2(ws0.z, ws0.w), part2[1]);
+            part2[2] = __ffma2_rn(ss, make_float2(ws1.x, ws1.y), part2[2]);
+            part2[3] = __ffma2_rn(ss, make_float2(ws1.z, ws1.w), part2[3]);
             const float cn = c * ca - s * sa;
             s = s * ca + c * sa;
             c = cn;
@@ -246,11 +259,24 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
       }
       // exact dims of the middle tokens for heads i0, i1
       float e0 = 0.0f, e1 = 0.0f;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float x[8], y[8];
+        bf16x8_to_f32(ek0[c8], x);
+        bf16x8_to_f32(ek1[c8], y);
+        const float4 qa = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8 * 8);
+        const float4 qb = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8 * 8 + 4);
+        const float4 ra = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8 * 8);
+        const float4 rb = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8 * 8 + 4);
+        e0 += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] + qb.y * x[5] +
+              qb.z * x[6] + qb.w * x[7];
+        e1 += ra.x * y[0] + ra.y * y[1] + ra.z * y[2] + ra.w * y[3] + rb.x * y[4] + rb.y * y[5] +
+              rb.z * y[6] + rb.w * y[7];
+      }
       if (v0) {
-        const __nv_bfloat16* row = p.EK + eb0 + (long long)tm * dl0;
-        for (int c8 = 0; c8 < dl0; c8 += 8) {
+        for (int c8 = 32; c8 < dl0; c8 += 8) {
           float x[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c8), x);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row0 + c8), x);
           const float4 qa = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8);
           const float4 qb = *reinterpret_cast<const float4*>(qes + i0 * FA_HEAD_DIM + c8 + 4);
           e0 += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
@@ -258,26 +284,27 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
         }
       }
       if (v1) {
-        const __nv_bfloat16* row = p.EK + eb1 + (long long)tm * dl1;
-        for (int c8 = 0; c8 < dl1; c8 += 8) {
+        for (int c8 = 32; c8 < dl1; c8 += 8) {
           float x[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c8), x);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(row1 + c8), x);
           const float4 qa = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8);
           const float4 qb = *reinterpret_cast<const float4*>(qes + i1 * FA_HEAD_DIM + c8 + 4);
           e1 += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
                 qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
         }
       }
+      // heads i0 = 2 qf, i1 = 2 qf + 1 form pair qf
 #pragma unroll
-      for (int h = 0; h < HL; ++h) {
-        if (h == i0) part[h] += e0;
-        if (h == i1) part[h] += e1;
-      }
+      for (int hp = 0; hp < HL / 2; ++hp)
+        if (hp == qf) {
+          part2[hp].x += e0;
+          part2[hp].y += e1;
+        }
     }
     {
       float4* dst = reinterpret_cast<float4*>(red + (qf * DT + tau) * HL);
-      dst[0] = make_float4(part[0], part[1], part[2], part[3]);
-      dst[1] = make_float4(part[4], part[5], part[6], part[7]);
+      dst[0] = make_float4(part2[0].x, part2[0].y, part2[1].x, part2[1].y);
+      dst[1] = make_float4(part2[2].x, part2[2].y, part2[3].x, part2[3].y);
     }
     __syncthreads();
     // ---------------------------------------------------------------- online softmax
@@ -322,15 +349,15 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     __syncthreads();
     // ---------------------------------------------------------------- u += p phi
     {
-      float al[HL];
+      float2 al[HL / 2];
 #pragma unroll
-      for (int h = 0; h < HL; ++h) al[h] = alpha_s[h];
+      for (int hp = 0; hp < HL / 2; ++hp) al[hp] = make_float2(alpha_s[2 * hp], alpha_s[2 * hp + 1]);
 #pragma unroll
       for (int j = 0; j < SPT; ++j)
 #pragma unroll
-        for (int h = 0; h < HL; ++h) {
-          uacc[j][h][0] *= al[h];
-          uacc[j][h][1] *= al[h];
+        for (int hp = 0; hp < HL / 2; ++hp) {
+          ucs[j][hp] = __fmul2_rn(ucs[j][hp], al[hp]);
+          uss[j][hp] = __fmul2_rn(uss[j][hp], al[hp]);
         }
       const int tb = uq * UT, te = min(nt, tb + UT);
       if (tb < te) {
@@ -342,13 +369,15 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
         for (int t = tb; t < te; ++t) {
           const float4 pa = *reinterpret_cast<const float4*>(ps + t * HL);
           const float4 pb = *reinterpret_cast<const float4*>(ps + t * HL + 4);
-          const float pr[HL] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+          const float2 pr[HL / 2] = {make_float2(pa.x, pa.y), make_float2(pa.z, pa.w),
+                                     make_float2(pb.x, pb.y), make_float2(pb.z, pb.w)};
 #pragma unroll
           for (int j = 0; j < SPT; ++j) {
+            const float2 cc = make_float2(c[j], c[j]), ss = make_float2(s[j], s[j]);
 #pragma unroll
-            for (int h = 0; h < HL; ++h) {
-              uacc[j][h][0] += pr[h] * c[j];
-              uacc[j][h][1] += pr[h] * s[j];
+            for (int hp = 0; hp < HL / 2; ++hp) {
+              ucs[j][hp] = __ffma2_rn(pr[hp], cc, ucs[j][hp]);
+              uss[j][hp] = __ffma2_rn(pr[hp], ss, uss[j][hp]);
             }
             const float cn = c[j] * cb[j] - s[j] * sb[j];
             s[j] = s[j] * cb[j] + c[j] * sb[j];
@@ -396,11 +425,11 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     dst[1] = make_float4(acce[4], acce[5], acce[6], acce[7]);
   }
   if (p.TG > 1) {
-    // SPT == 1 whenever TG > 1
+    // SPT == 1 whenever TG > 1; per thread [head][cos, sin]
     float4* dst = reinterpret_cast<float4*>(ured + tid * 16);
 #pragma unroll
-    for (int h = 0; h < HL; h += 2)
-      dst[h / 2] = make_float4(uacc[0][h][0], uacc[0][h][1], uacc[0][h + 1][0], uacc[0][h + 1][1]);
+    for (int hp = 0; hp < HL / 2; ++hp)
+      dst[hp] = make_float4(ucs[0][hp].x, uss[0][hp].x, ucs[0][hp].y, uss[0][hp].y);
   }
   __syncthreads();
   if (tid < HL && gh_s[tid] >= 0) {
@@ -451,7 +480,9 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
         for (int h = 0; h < HL; ++h) {
           if (gh_s[h] >= 0) {
             float* rec = p.rec + ((long long)sp * bhq + gh_s[h]) * p.rec_stride + 4 + FA_HEAD_DIM;
-            *reinterpret_cast<float2*>(rec + 2 * f) = make_float2(uacc[j][h][0], uacc[j][h][1]);
+            const float uc = (h & 1) ? ucs[j][h >> 1].y : ucs[j][h >> 1].x;
+            const float us = (h & 1) ? uss[j][h >> 1].y : uss[j][h >> 1].x;
+            *reinterpret_cast<float2*>(rec + 2 * f) = make_float2(uc, us);
           }
         }
       }
@@ -579,7 +610,8 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
 }
 
 template <int SPT>
-__global__ void __launch_bounds__(DNT, 1) decode_main_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(DNT, SPT == 1 ? 2 : 1)
+    decode_main_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ __align__(16) float sm[];
   const int cta = blockIdx.x;
   if (cta < p.n_mid)

@@ -25,6 +25,7 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
                           const fa_cache* cache, void* out, int out_dtype, void* workspace,
                           cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
+cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream);
 
 // Records `msg` as the calling thread's fa_last_error() text and returns `code`.
 int set_last_error(int code, const char* msg);

@@ -22,6 +22,8 @@ static __device__ unsigned int g_watchdog = 0;
 
 enum : unsigned int {
   WD_COMPRESS = 1u << 8,
+  WD_DECODE = 2u << 8,
+  WD_SELFTEST = 15u << 8,
 };
 
 // Wall-time bound of one mbarrier wait (ns). Legitimate waits in these kernels last at
@@ -81,14 +83,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // `site` in the watchdog word and raising *abort) if the wall-time limit passed or
 // another thread of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          unsigned int site) {
+                                          unsigned int site,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicCAS(&g_watchdog, 0u, site);
         *abort = 1;
         return false;
@@ -128,6 +131,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const void* tmap, uint64_
       "cp.async.bulk.tensor.3d.shared::cta.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// Bulk copy global -> shared (both 16-byte aligned, bytes a multiple of 16), completing on
+// an mbarrier's transaction count.
+__device__ __forceinline__ void bulk_load(void* sdst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(sdst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -221,6 +221,15 @@ int fa_decode_noalloc(const fa_plan* plan, const void* q, const fa_cache* cache,
  */
 int fa_device_status(void* stream);
 
+/*
+ * fa_watchdog_selftest -- diagnostics for the bounded-wait path (no counterpart in the
+ * paper). Launches one CTA whose thread waits on an mbarrier that nothing ever completes,
+ * with a wall-time bound of `wait_ns` (1 us .. 1 s). The wait expires, the kernel records a
+ * watchdog code and returns normally; the next fa_device_status(stream) must then report
+ * FA_ERR_DEVICE and clear it. Nothing faults, traps or hangs.
+ */
+int fa_watchdog_selftest(uint32_t wait_ns, void* stream);
+
 /* Message of the last non-FA_OK return on the calling thread ("" if none). */
 const char* fa_last_error(void);
 

@@ -227,3 +227,16 @@ def test_full_size_sampled_heads(w):
     assert torch.isfinite(out.float()).all().item()
     idx = torch.cat([torch.arange(p.S), torch.arange(w.L - p.R, w.L)]).cuda()
     assert torch.equal(cache.F("K"), K[:, :, idx]) and torch.equal(cache.F("V"), V[:, :, idx])
+
+
+# ----------------------------------------------------------------------------- failure detection
+
+def test_bounded_wait_reports_and_context_survives():
+    """A kernel waiting on a barrier nothing completes gives up after its bound, the host
+    reads FA_ERR_DEVICE, the word is cleared, and the next compress + decode still run."""
+    fa.fa_watchdog_selftest(20_000_000)
+    with pytest.raises(fa.FaError) as e:
+        fa.fa_device_status()
+    assert e.value.code == fa.FA_ERR_DEVICE and "kernel 15" in str(e.value)
+    fa.fa_device_status()  # cleared
+    run_small(wl.shrink(wl.SINGLE_HEAD_2K, L=600))
