@@ -205,7 +205,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
             if (kt < kt_n) {
               // A: 16 tokens = 32 bytes further along the swizzled 128-byte row.
               const uint64_t ad = smem_desc_sw128(a_addr + kt * CK_A_TILE + kk * 32, 16, 1024);
-              mma_bf16(tmem_d + kt * CK_BN, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
+              mma_f16(tmem_d + kt * CK_BN, ad, bd, idesc, (it > 0 || kk > 0) ? 1u : 0u);
             }
           }
         }

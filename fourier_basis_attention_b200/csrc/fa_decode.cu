@@ -20,49 +20,9 @@
 //             (running max, running sum, value accumulator, u).
 //   combine   per KV head: merges the records, out_c = u C_V, scatters the dims back,
 //             normalises and stores fp32 or bf16.
-#include "fa_host.h"
-#include "fa_internal.cuh"
+#include "fa_decode_common.cuh"
 
 namespace fa {
-
-constexpr int DT = 64;    // tokens per tile
-constexpr int DNT = 256;  // threads per CTA
-constexpr int HL = 8;     // query heads per CTA (zero-padded)
-constexpr int FT = 256;   // sink/recent rows per CTA
-
-struct DecodeParams {
-  int B, Hq, Hkv, G, M, k, F, F_pad, nF;
-  int n_splits, split_len, n_fsplits, NKV, n_mid, n_rec;
-  int rec_stride, qw_stride;
-  int NTU, TG, DEC, TGE;
-  float qscale, norm_single, norm_pair, two_over_M;
-  long long e_batch, c_batch;
-  long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
-  int de[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS], dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
-  unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
-  const __nv_bfloat16 *q, *FK, *FV, *EK, *EV;
-  const float *CK, *CV;
-  void* out;
-  int out_f32;
-  float* qw;
-  float* rec;
-};
-
-// cos / sin of 2 pi r / M for an exactly reduced integer phase 0 <= r < M.
-__device__ __forceinline__ void phase_sincos(long long r, int M, float two_over_M, float* s,
-                                             float* c) {
-  const long long rr = (2 * r > M) ? r - M : r;  // (-M/2, M/2]
-  sincospif((float)rr * two_over_M, s, c);
-}
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&x)[8]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
 
 // ------------------------------------------------------------------------- prologue
 __global__ void __launch_bounds__(DNT) decode_prologue_kernel(const __grid_constant__ DecodeParams p) {
@@ -191,7 +151,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   for (int j = 0; j < SPT; ++j) {
     phase_sincos((long long)(ui + j * p.NTU) % M, M, p.two_over_M, &sb[j], &cb[j]);
 #pragma unroll
-    for (int hp = 0; hp < HL / 2; ++hp) ucs[j][hp] = uss[j][hp] = make_float2(0.0f, 0.0f);
+    for (int pr2 = 0; pr2 < HL / 2; ++pr2) ucs[j][pr2] = uss[j][pr2] = make_float2(0.0f, 0.0f);
   }
   // exact-dim value role: head ie, 8-dim chunk ce, token group qg
   const int ei = tid % (HL * p.DEC), qg = tid / (HL * p.DEC);
@@ -219,7 +179,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     // ---------------------------------------------------------------- scores
     float2 part2[HL / 2];
 #pragma unroll
-    for (int hp = 0; hp < HL / 2; ++hp) part2[hp] = make_float2(0.0f, 0.0f);
+    for (int pr2 = 0; pr2 < HL / 2; ++pr2) part2[pr2] = make_float2(0.0f, 0.0f);
     const int tm = t0 + tau;
     if (tau < nt) {
       // the first 32 exact dims of both rows are loaded up front so that their latency
@@ -295,10 +255,10 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
       }
       // heads i0 = 2 qf, i1 = 2 qf + 1 form pair qf
 #pragma unroll
-      for (int hp = 0; hp < HL / 2; ++hp)
-        if (hp == qf) {
-          part2[hp].x += e0;
-          part2[hp].y += e1;
+      for (int pr2 = 0; pr2 < HL / 2; ++pr2)
+        if (pr2 == qf) {
+          part2[pr2].x += e0;
+          part2[pr2].y += e1;
         }
     }
     {
@@ -351,13 +311,14 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     {
       float2 al[HL / 2];
 #pragma unroll
-      for (int hp = 0; hp < HL / 2; ++hp) al[hp] = make_float2(alpha_s[2 * hp], alpha_s[2 * hp + 1]);
+      for (int pr2 = 0; pr2 < HL / 2; ++pr2)
+        al[pr2] = make_float2(alpha_s[2 * pr2], alpha_s[2 * pr2 + 1]);
 #pragma unroll
       for (int j = 0; j < SPT; ++j)
 #pragma unroll
-        for (int hp = 0; hp < HL / 2; ++hp) {
-          ucs[j][hp] = __fmul2_rn(ucs[j][hp], al[hp]);
-          uss[j][hp] = __fmul2_rn(uss[j][hp], al[hp]);
+        for (int pr2 = 0; pr2 < HL / 2; ++pr2) {
+          ucs[j][pr2] = __fmul2_rn(ucs[j][pr2], al[pr2]);
+          uss[j][pr2] = __fmul2_rn(uss[j][pr2], al[pr2]);
         }
       const int tb = uq * UT, te = min(nt, tb + UT);
       if (tb < te) {
@@ -375,9 +336,9 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
           for (int j = 0; j < SPT; ++j) {
             const float2 cc = make_float2(c[j], c[j]), ss = make_float2(s[j], s[j]);
 #pragma unroll
-            for (int hp = 0; hp < HL / 2; ++hp) {
-              ucs[j][hp] = __ffma2_rn(pr[hp], cc, ucs[j][hp]);
-              uss[j][hp] = __ffma2_rn(pr[hp], ss, uss[j][hp]);
+            for (int pr2 = 0; pr2 < HL / 2; ++pr2) {
+              ucs[j][pr2] = __ffma2_rn(pr[pr2], cc, ucs[j][pr2]);
+              uss[j][pr2] = __ffma2_rn(pr[pr2], ss, uss[j][pr2]);
             }
             const float cn = c[j] * cb[j] - s[j] * sb[j];
             s[j] = s[j] * cb[j] + c[j] * sb[j];
@@ -428,8 +389,8 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
     // SPT == 1 whenever TG > 1; per thread [head][cos, sin]
     float4* dst = reinterpret_cast<float4*>(ured + tid * 16);
 #pragma unroll
-    for (int hp = 0; hp < HL / 2; ++hp)
-      dst[hp] = make_float4(ucs[0][hp].x, uss[0][hp].x, ucs[0][hp].y, uss[0][hp].y);
+    for (int pr2 = 0; pr2 < HL / 2; ++pr2)
+      dst[pr2] = make_float4(ucs[0][pr2].x, uss[0][pr2].x, ucs[0][pr2].y, uss[0][pr2].y);
   }
   __syncthreads();
   if (tid < HL && gh_s[tid] >= 0) {
@@ -742,9 +703,18 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   c->TGE = DNT / (HL * c->DEC);
   c->NKV = HL / plan->G;
   const int n_heads = sh.B * sh.Hkv;
-  const int n_headsets = (n_heads + c->NKV - 1) / c->NKV;
   c->smem_main = main_smem_bytes(c->F_pad);
-  const int ntiles = (M + DT - 1) / DT;
+  c->de_ld_max = de_ld_max;
+  // The tensor-core split kernel holds W and U for 128 heads x 2F slots on chip: it takes
+  // k <= 255 (2F <= 256 slots, in 64-slot swizzle atoms) and up to 64 exact dims per head.
+  c->tc_F2 = ((2 * c->F + 63) / 64) * 64;
+  c->tc = (M > 0 && c->tc_F2 <= 256 && de_ld_max <= 64) ? 1 : 0;
+  int cols = 32;
+  while (cols < c->tc_F2 + 64) cols <<= 1;
+  c->tc_tmem_cols = cols;
+  const int unit_tokens = c->tc ? 32 : DT;  // tokens per tile
+  const int n_headsets = c->tc ? (sh.B * sh.Hq + 127) / 128 : (n_heads + c->NKV - 1) / c->NKV;
+  const int ntiles = (M + unit_tokens - 1) / unit_tokens;
   if (M == 0) {
     c->n_splits = 0;
     c->split_len = 0;
@@ -758,9 +728,13 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
       if (e != cudaSuccess) return e;
       e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
       if (e != cudaSuccess) return e;
-      e = c->SPT == 1 ? occupancy<1>(&occ, c->smem_main)
-                      : (c->SPT == 2 ? occupancy<2>(&occ, c->smem_main) : occupancy<4>(&occ, c->smem_main));
-      if (e != cudaSuccess) return e;
+      if (c->tc) {
+        occ = 1;  // one CTA per SM (shared memory)
+      } else {
+        e = c->SPT == 1 ? occupancy<1>(&occ, c->smem_main)
+                        : (c->SPT == 2 ? occupancy<2>(&occ, c->smem_main) : occupancy<4>(&occ, c->smem_main));
+        if (e != cudaSuccess) return e;
+      }
       if (occ < 1) occ = 1;
       const long long slots = (long long)sms * occ;
       // cost = waves x tiles per CTA, plus a small per-split charge for the record
@@ -782,7 +756,7 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
     }
     const int per = (ntiles + ns - 1) / ns;
     c->n_splits = (ntiles + per - 1) / per;
-    c->split_len = per * DT;
+    c->split_len = per * unit_tokens;
   }
   const int nF = plan->S + plan->R;
   c->n_fsplits = (nF + FT - 1) / FT;
@@ -825,6 +799,8 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   p.qw_stride = c.qw_stride;
   p.NTU = c.NTU;
   p.TG = c.TG;
+  p.tc_F2 = c.tc_F2;
+  p.tc_tmem_cols = c.tc_tmem_cols;
   p.DEC = c.DEC;
   p.TGE = c.TGE;
   p.qscale = (float)(1.4426950408889634 / sqrt((double)FA_HEAD_DIM));
@@ -859,6 +835,12 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   if (p.M > 0) {
     decode_prologue_kernel<<<n_heads, DNT, plan->G * FA_HEAD_DIM * 4, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (c.tc && p.n_splits > 0) {
+    // middle span on the tensor cores; the CUDA-core kernel below then only runs the
+    // sink / recent CTAs
+    if ((e = launch_decode_tc(p, c.de_ld_max, stream)) != cudaSuccess) return e;
+    p.n_mid = 0;
   }
   const int grid = p.n_mid + n_heads * c.n_fsplits;
   if (grid > 0) {

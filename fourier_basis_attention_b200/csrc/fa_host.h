@@ -11,6 +11,7 @@ namespace fa {
 // Launch configuration of one fa_decode call (derived by decode_configure).
 struct DecodeConfig {
   int n_splits, split_len, n_fsplits, n_rec, F, F_pad, SPT, NTU, TG, DEC, TGE, NKV;
+  int tc, tc_F2, tc_tmem_cols, de_ld_max;  // tensor-core split kernel chosen, its slots / TMEM
   size_t qw_bytes, rec_bytes, smem_main, smem_combine;
   int rec_stride, qw_stride;
 };
