@@ -412,7 +412,7 @@ def run_ours(args):
         },
         "roofline": roof,
         "clocks": {**summarize_clocks(rows), "note": clock_note},
-        "gpu_launches": 6 * args.steps,
+        "gpu_launches": launches_per_step(w, plan) * args.steps,
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
     }
@@ -432,6 +432,18 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def launches_per_step(w, plan):
+    """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel and
+    compress_kernel; then fa_decode's prologue (middle span present), one split kernel (the
+    tensor-core one when the plan laid E out token-major, else the CUDA-core one; either
+    also covers the sink / recent rows), and the combine."""
+    n = 1 + 2
+    n += 1 if plan.M > 0 else 0          # prologue
+    if plan.M > 0 or plan.S + plan.R > 0:
+        n += 1                           # split kernel
+    return n + 1                         # combine
+
+
 def K_bytes(w):
     return w.B * w.Hkv * w.L * 128 * 2
 
@@ -445,6 +457,34 @@ def _time(fn, n, stream):
         fn()
     b.record(stream)
     torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def _time_graph(fn, n):
+    """Per-replay device time of fn(stream) captured once in a CUDA graph (the way a serving
+    loop runs a launch-bound step); CUDA events on the replaying stream."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn(side)
+        fn(side)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn(torch.cuda.current_stream())
+    g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    del g
     return a.elapsed_time(b) / n
 
 
@@ -480,7 +520,8 @@ def run_sweep(args):
             f(); f(); f()
         tb = _time(basis, 10, stream)
         tcmp = _time(comp, 10, stream)
-        td = _time(dec, 20, stream)
+        td_eager = _time(dec, 20, stream)
+        td = _time_graph(lambda s: fa.fa_decode(plan, q, cache, out, ws, 0, s), 20)
         fa.fa_device_status(stream)
         wm = work_model(w, plan)
         print(json.dumps({"sweep": "single_layer", "workload": w.name, "basis_us": tb * 1e3,
@@ -489,7 +530,9 @@ def run_sweep(args):
                           "compress_hbm_gbs": wm["compress_bytes"] / tcmp / 1e6,
                           "compress_frac_tensor": wm["compress_flops"] / tcmp / 1e9 / tc,
                           "compress_frac_hbm": wm["compress_bytes"] / tcmp / 1e6 / hbm,
-                          "decode_us": td * 1e3, "decode_hbm_gbs": wm["decode_bytes"] / td / 1e6,
+                          "decode_us": td * 1e3, "decode_us_eager": td_eager * 1e3,
+                          "decode_timing": "CUDA graph replay (eager launches in decode_us_eager)",
+                          "decode_hbm_gbs": wm["decode_bytes"] / td / 1e6,
                           "decode_frac_hbm": wm["decode_bytes"] / td / 1e6 / hbm,
                           "decode_fp32_tflops": wm["decode_flops"] / td / 1e9}), flush=True)
         del K, V, cache, ws, out, phiT
@@ -532,12 +575,13 @@ def run_sweep(args):
         ws = torch.empty(max(fa.fa_decode_workspace_size(p) for p in plans), dtype=torch.uint8, device=dev)
         out = torch.empty(B, 32, 128, dtype=torch.bfloat16, device=dev)
 
-        def step():
+        def step(s=stream):
             for p, c in zip(plans, caches):
-                fa.fa_decode(p, q, c, out, ws, 0, stream)
+                fa.fa_decode(p, q, c, out, ws, 0, s)
         step()
         n = 3 if B * L >= 32 * 131072 else 10
-        td = _time(step, n, stream)
+        td_eager = _time(step, n, stream)
+        td = _time_graph(step, n)
         fa.fa_device_status(stream)
         wms = [work_model(wl.llama3_8b_layer(B, L, l), p) for l, p in enumerate(plans)]
         dbytes = sum(m["decode_bytes"] for m in wms)
@@ -550,6 +594,8 @@ def run_sweep(args):
                           "compress_tflops": cflops / tcomp / 1e9,
                           "compress_frac_hbm": cbytes / tcomp / 1e6 / hbm,
                           "decode_us_per_step": td * 1e3,
+                          "decode_us_per_step_eager": td_eager * 1e3,
+                          "decode_timing": "CUDA graph replay of the 32 layer calls",
                           "decode_hbm_gbs": dbytes / td / 1e6,
                           "decode_frac_hbm": dbytes / td / 1e6 / hbm}), flush=True)
         del caches, plans, ws, out, q, phiT

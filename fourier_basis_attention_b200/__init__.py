@@ -49,8 +49,10 @@ class fa_plan(ctypes.Structure):
         ("shape", fa_shape),
         ("S", ctypes.c_int32), ("R", ctypes.c_int32), ("M", ctypes.c_int32),
         ("kk", ctypes.c_int32), ("G", ctypes.c_int32), ("phi_ld", ctypes.c_int32),
+        ("e_token_major", ctypes.c_int32),
         ("dc", ctypes.c_int32 * _H), ("de", ctypes.c_int32 * _H),
         ("dc_ld", ctypes.c_int32 * _H), ("de_ld", ctypes.c_int32 * _H),
+        ("e_pitch", ctypes.c_int32 * _H),
         ("c_off", ctypes.c_int64 * _H), ("e_off", ctypes.c_int64 * _H),
         ("c_batch", ctypes.c_int64), ("e_batch", ctypes.c_int64),
         ("f_elems", ctypes.c_int64), ("e_elems", ctypes.c_int64), ("c_elems", ctypes.c_int64),
@@ -208,10 +210,7 @@ class Cache:
         return t[:p.f_elems].view(p.shape.B, p.shape.Hkv, p.S + p.R, HEAD_DIM)
 
     def E(self, which: str, b: int, g: int):
-        p = self.plan
-        t = self.E_K if which == "K" else self.E_V
-        off = b * p.e_batch + p.e_off[g]
-        return t[off:off + p.M * p.de_ld[g]].view(p.M, p.de_ld[g])[:, :p.de[g]]
+        return self.E_raw(which, b, g)[:, :self.plan.de[g]]
 
     def C(self, which: str, b: int, g: int):
         p = self.plan
@@ -220,10 +219,11 @@ class Cache:
         return t[off:off + p.kk * p.dc_ld[g]].view(p.kk, p.dc_ld[g])[:, :p.dc[g]]
 
     def E_raw(self, which: str, b: int, g: int):
+        """[M, de_ld] view of KV head (b, g)'s rows (strided when E is token-major)."""
         p = self.plan
         t = self.E_K if which == "K" else self.E_V
         off = b * p.e_batch + p.e_off[g]
-        return t[off:off + p.M * p.de_ld[g]].view(p.M, p.de_ld[g])
+        return t.as_strided((p.M, p.de_ld[g]), (p.e_pitch[g], 1), t.storage_offset() + off)
 
     def C_raw(self, which: str, b: int, g: int):
         p = self.plan

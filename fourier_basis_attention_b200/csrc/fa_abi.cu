@@ -37,6 +37,45 @@ int check_ptr(const void* p, const char* name, bool required) {
   return FA_OK;
 }
 
+// Fills the layout fields of a plan (everything below the dim split) from shape, S, R, M,
+// kk, G, dc and de. E is token-major exactly when the tensor-core decode is used: it can
+// run when k <= 255, G is 1, 2 or 4 and every KV head keeps at most 32 dims, and it is
+// chosen when the k-length work per token and KV head (k G) is at least 500 and there are
+// at least 128 query heads (one full tensor-core head set); below that the CUDA-core
+// decode, whose time is then mostly the exact-dim rows, is the faster of the two.
+void derive_layout(fa_plan* plan) {
+  const fa_shape& s = plan->shape;
+  int max_de = 0;
+  for (int g = 0; g < s.Hkv; ++g) max_de = plan->de[g] > max_de ? plan->de[g] : max_de;
+  const int G = plan->G;
+  const bool tm = plan->M > 0 && s.k <= 255 && (G == 1 || G == 2 || G == 4) && max_de <= 32 &&
+                  s.k * G >= 500 && (long long)s.B * s.Hq >= 128;
+  const int w = max_de == 0 ? 0 : (max_de <= 8 ? 8 : (max_de <= 16 ? 16 : 32));
+  plan->e_token_major = tm ? 1 : 0;
+  long long ce = 0, ee = 0;
+  for (int g = 0; g < s.Hkv; ++g) {
+    plan->dc_ld[g] = round8(plan->dc[g]);
+    plan->c_off[g] = ce;
+    ce += (long long)plan->kk * plan->dc_ld[g];
+    if (tm) {
+      plan->de_ld[g] = w;
+      plan->e_off[g] = (long long)g * w;
+      plan->e_pitch[g] = s.Hkv * w;
+    } else {
+      plan->de_ld[g] = round8(plan->de[g]);
+      plan->e_off[g] = ee;
+      plan->e_pitch[g] = plan->de_ld[g];
+      ee += (long long)plan->M * plan->de_ld[g];
+    }
+  }
+  if (tm) ee = (long long)plan->M * s.Hkv * w;
+  plan->c_batch = ce;
+  plan->e_batch = ee;
+  plan->f_elems = (long long)s.B * s.Hkv * (plan->S + plan->R) * FA_HEAD_DIM;
+  plan->e_elems = (long long)s.B * ee;
+  plan->c_elems = (long long)s.B * ce;
+}
+
 // Re-checks the fields kernels rely on, so a plan edited by hand cannot drive a launch
 // out of bounds.
 int check_plan(const fa_plan* plan) {
@@ -49,11 +88,9 @@ int check_plan(const fa_plan* plan) {
   if (plan->S < 0 || plan->R < 0 || plan->M < 0 || plan->S + plan->M + plan->R != s.L)
     return fail(FA_ERR_INVALID, "plan token partition is inconsistent");
   if (plan->G != s.Hq / s.Hkv) return fail(FA_ERR_INVALID, "plan G is inconsistent");
-  long long ce = 0, ee = 0;
+  if (plan->kk != (plan->M > 0 ? s.k : 0)) return fail(FA_ERR_INVALID, "plan kk is inconsistent");
   for (int g = 0; g < s.Hkv; ++g) {
-    if (plan->dc[g] < 0 || plan->dc[g] > FA_HEAD_DIM || plan->de[g] != FA_HEAD_DIM - plan->dc[g] ||
-        plan->dc_ld[g] != round8(plan->dc[g]) || plan->de_ld[g] != round8(plan->de[g]) ||
-        plan->c_off[g] != ce || plan->e_off[g] != ee)
+    if (plan->dc[g] < 0 || plan->dc[g] > FA_HEAD_DIM || plan->de[g] != FA_HEAD_DIM - plan->dc[g])
       return fail(FA_ERR_INVALID, "plan dims of KV head %d are inconsistent", g);
     bool seen[FA_HEAD_DIM] = {false};
     for (int i = 0; i < FA_HEAD_DIM; ++i) {
@@ -62,11 +99,17 @@ int check_plan(const fa_plan* plan) {
         return fail(FA_ERR_INVALID, "plan perm of KV head %d is not a permutation", g);
       seen[d] = true;
     }
-    ce += (long long)plan->kk * plan->dc_ld[g];
-    ee += (long long)plan->M * plan->de_ld[g];
   }
-  if (plan->c_batch != ce || plan->e_batch != ee)
-    return fail(FA_ERR_INVALID, "plan batch strides are inconsistent");
+  fa_plan ref = *plan;
+  derive_layout(&ref);
+  bool same = ref.e_token_major == plan->e_token_major && ref.c_batch == plan->c_batch &&
+              ref.e_batch == plan->e_batch && ref.f_elems == plan->f_elems &&
+              ref.e_elems == plan->e_elems && ref.c_elems == plan->c_elems;
+  for (int g = 0; g < s.Hkv && same; ++g)
+    same = ref.dc_ld[g] == plan->dc_ld[g] && ref.de_ld[g] == plan->de_ld[g] &&
+           ref.e_pitch[g] == plan->e_pitch[g] && ref.c_off[g] == plan->c_off[g] &&
+           ref.e_off[g] == plan->e_off[g];
+  if (!same) return fail(FA_ERR_INVALID, "plan layout fields are inconsistent");
   return FA_OK;
 }
 
@@ -97,7 +140,6 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) 
   plan->G = s.Hq / s.Hkv;
   plan->phi_ld = round8(plan->M > 8 ? plan->M : 8);
   bool any_dc = false;
-  long long ce = 0, ee = 0;
   for (int g = 0; g < s.Hkv; ++g) {
     int n = 0;
     for (int d = 0; d < FA_HEAD_DIM; ++d)
@@ -106,21 +148,11 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) 
     for (int d = 0; d < FA_HEAD_DIM; ++d)
       if (!dim_mask[g * FA_HEAD_DIM + d]) plan->perm[g][n++] = (uint8_t)d;
     plan->de[g] = FA_HEAD_DIM - plan->dc[g];
-    plan->dc_ld[g] = round8(plan->dc[g]);
-    plan->de_ld[g] = round8(plan->de[g]);
-    plan->c_off[g] = ce;
-    plan->e_off[g] = ee;
-    ce += (long long)plan->kk * plan->dc_ld[g];
-    ee += (long long)plan->M * plan->de_ld[g];
     any_dc = any_dc || plan->dc[g] > 0;
   }
   if (plan->M > 0 && any_dc && s.k > plan->M)
     return fail(FA_ERR_UNSUPPORTED, "k=%d exceeds the middle span M=%d", s.k, plan->M);
-  plan->c_batch = ce;
-  plan->e_batch = ee;
-  plan->f_elems = (long long)s.B * s.Hkv * (plan->S + plan->R) * FA_HEAD_DIM;
-  plan->e_elems = (long long)s.B * ee;
-  plan->c_elems = (long long)s.B * ce;
+  derive_layout(plan);
   return FA_OK;
 }
 
@@ -130,9 +162,8 @@ int fa_build_basis(int32_t M, int32_t k, int32_t dtype, int32_t normalized, void
   if (dtype != FA_BF16 && dtype != FA_F32) return fail(FA_ERR_INVALID, "unknown dtype %d", dtype);
   if (ld < M || ld % 8 != 0) return fail(FA_ERR_INVALID, "ld=%lld must be >= M and a multiple of 8", (long long)ld);
   if (int r = check_ptr(phiT, "phiT", true)) return r;
-  int dev = 0, sms = 148;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = 148;
+  cudaError_t e = fa::device_sm_count(&sms);
   if (e != cudaSuccess) return cuda_fail(e, "fa_build_basis: device query");
   e = fa::launch_build_basis(M, k, ld, dtype, normalized ? 1 : 0, phiT,
                              static_cast<cudaStream_t>(stream), sms);

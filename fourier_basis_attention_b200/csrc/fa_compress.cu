@@ -60,7 +60,7 @@ struct CompressParams {
   long long c_batch, e_batch;
   long long c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
   int dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
-  int de_ld[FA_MAX_KV_HEADS];
+  int de_ld[FA_MAX_KV_HEADS], e_pitch[FA_MAX_KV_HEADS];
   unsigned char perm[FA_MAX_KV_HEADS][FA_HEAD_DIM];
   float* C[2];
   __nv_bfloat16* E[2];
@@ -233,6 +233,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       // stage), then writes the rows as coalesced 64-byte global stores.
       const int de = FA_HEAD_DIM - dc;
       const int de_ld = p.de_ld[g];
+      const int e_pitch = p.e_pitch[g];    // elements between consecutive rows
       const int ngrp = (de_ld + 31) >> 5;  // 32-dim groups per row
       __nv_bfloat16* const E0 = p.E[0] + (long long)b * p.e_batch + p.e_off[g];
       __nv_bfloat16* const E1 = p.E[1] + (long long)b * p.e_batch + p.e_off[g];
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
                 const int tau = pw + j * CK_PACK_WARPS;
                 if (tau < ntok)
                   reinterpret_cast<unsigned short*>((x ? E1 : E0) +
-                                                    (long long)(it * CK_BK + tau) * de_ld)[i] =
+                                                    (long long)(it * CK_BK + tau) * e_pitch)[i] =
                       v[x][j];
               }
           }
@@ -478,6 +479,7 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
     cp.dc[g] = plan->dc[g];
     cp.dc_ld[g] = plan->dc_ld[g];
     cp.de_ld[g] = plan->de_ld[g];
+    cp.e_pitch[g] = plan->e_pitch[g];
     memcpy(cp.perm[g], plan->perm[g], FA_HEAD_DIM);
   }
   cp.C[0] = static_cast<float*>(cache->C_K);
@@ -494,11 +496,11 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   const int smem = KT == 2 ? CkCfg<2>::BASE_SMEM : CkCfg<1>::BASE_SMEM;
   cudaError_t e;
   if (KT == 2) {
-    e = cudaFuncSetAttribute(compress_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = raise_smem_limit(reinterpret_cast<const void*>(compress_kernel<2>), smem);
     if (e != cudaSuccess) return e;
     compress_kernel<2><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
   } else {
-    e = cudaFuncSetAttribute(compress_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = raise_smem_limit(reinterpret_cast<const void*>(compress_kernel<1>), smem);
     if (e != cudaSuccess) return e;
     compress_kernel<1><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
   }

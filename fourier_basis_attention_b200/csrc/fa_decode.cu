@@ -451,125 +451,6 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   }
 }
 
-// ------------------------------------------------------------------------- main: sink/recent
-__device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float* sm, int fid) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int kvh = fid / p.n_fsplits, fs = fid - (fid / p.n_fsplits) * p.n_fsplits;
-  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
-  const int r0 = fs * FT, nr = min(FT, p.nF - r0);
-  const int G = p.G;
-  float* qs = sm;                       // [HL][128]
-  float* sc = qs + HL * FA_HEAD_DIM;    // [FT][HL]
-  float* mxs = sc + FT * HL;            // [8][HL]
-  float* mh = mxs + 8 * HL;             // [HL]
-  float* red = mh + HL;                 // [DNT][8]
-
-  for (int idx = tid; idx < HL * FA_HEAD_DIM; idx += DNT) {
-    const int h = idx >> 7, d = idx & 127;
-    qs[idx] = (h < G) ? __bfloat162float(p.q[((long long)b * p.Hq + g * G + h) * FA_HEAD_DIM + d]) *
-                            p.qscale
-                      : 0.0f;
-  }
-  __syncthreads();
-  const __nv_bfloat16* FKh = p.FK + (long long)kvh * p.nF * FA_HEAD_DIM;
-  const __nv_bfloat16* FVh = p.FV + (long long)kvh * p.nF * FA_HEAD_DIM;
-  float s[HL];
-#pragma unroll
-  for (int h = 0; h < HL; ++h) s[h] = 0.0f;
-  if (tid < nr) {
-    const __nv_bfloat16* row = FKh + (long long)(r0 + tid) * FA_HEAD_DIM;
-    for (int c = 0; c < FA_HEAD_DIM; c += 8) {
-      float x[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c), x);
-#pragma unroll
-      for (int h = 0; h < HL; ++h) {
-        if (h < G) {
-          const float4 qa = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c);
-          const float4 qb = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c + 4);
-          s[h] += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
-                  qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
-        }
-      }
-    }
-  }
-#pragma unroll
-  for (int h = 0; h < HL; ++h)
-    if (tid >= nr || h >= G) s[h] = -INFINITY;
-#pragma unroll
-  for (int h = 0; h < HL; ++h) {
-    float m = s[h];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) mxs[warp * HL + h] = m;
-  }
-  __syncthreads();
-  if (tid < HL) {
-    float m = mxs[tid];
-#pragma unroll
-    for (int w = 1; w < 8; ++w) m = fmaxf(m, mxs[w * HL + tid]);
-    mh[tid] = m;
-  }
-  __syncthreads();
-  float l[HL];
-#pragma unroll
-  for (int h = 0; h < HL; ++h) {
-    const float pv = (h < G && tid < nr) ? exp2f(s[h] - mh[h]) : 0.0f;
-    sc[tid * HL + h] = pv;
-    l[h] = pv;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < HL; ++h) {
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
-    if (lane == 0) mxs[warp * HL + h] = l[h];
-  }
-  // values: item (head h, 8-dim chunk c), token group grp
-  const int items = G * 16;
-  const int it = tid % items, grp = tid / items, ngrp = DNT / items;
-  const int h = it >> 4, c = it & 15;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-  for (int rr = grp; rr < nr; rr += ngrp) {
-    const float pv = sc[rr * HL + h];
-    float x[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += pv * x[e];
-  }
-  {
-    float4* dst = reinterpret_cast<float4*>(red + tid * 8);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  }
-  __syncthreads();
-  const long long bhq = (long long)p.B * p.Hq;
-  const int rix = p.n_splits + fs;
-  if (tid < G) {
-    float ls = 0.0f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) ls += mxs[w * HL + tid];
-    float* rec = p.rec + ((long long)rix * bhq + (long long)b * p.Hq + g * G + tid) * p.rec_stride;
-    rec[0] = mh[tid];
-    rec[1] = ls;
-  }
-  if (grp == 0) {
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-    for (int q2 = 0; q2 < ngrp; ++q2) {
-      const float* src = red + (q2 * items + it) * 8;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] += src[e];
-    }
-    float* rec = p.rec + ((long long)rix * bhq + (long long)b * p.Hq + g * G + h) * p.rec_stride +
-                 4 + c * 8;
-    reinterpret_cast<float4*>(rec)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(rec)[1] = make_float4(v[4], v[5], v[6], v[7]);
-  }
-}
-
 template <int SPT>
 __global__ void __launch_bounds__(DNT, SPT == 1 ? 2 : 1)
     decode_main_kernel(const __grid_constant__ DecodeParams p) {
@@ -670,18 +551,13 @@ static size_t main_smem_bytes(int F_pad) {
   const size_t mid = (size_t)(F_pad * HL * 2 + HL * FA_HEAD_DIM + DT * HL + 4 * DT * HL + 8 * HL +
                               2 * HL + DNT * 16) * 4 +
                      HL * 8 + 2 * HL * 4;
-  const size_t fpart = (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + DNT * 8) * 4;
+  const size_t fpart = sink_recent_smem_bytes();
   return mid > fpart ? mid : fpart;
 }
 
 template <int SPT>
 static cudaError_t occupancy(int* blocks, size_t smem) {
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaFuncSetAttribute(decode_main_kernel<SPT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, decode_main_kernel<SPT>, DNT, smem);
+  return cached_occupancy(reinterpret_cast<const void*>(decode_main_kernel<SPT>), DNT, smem, blocks);
 }
 
 // Derive the launch configuration. `requested` <= 0 selects the split count from a
@@ -705,10 +581,11 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   const int n_heads = sh.B * sh.Hkv;
   c->smem_main = main_smem_bytes(c->F_pad);
   c->de_ld_max = de_ld_max;
-  // The tensor-core split kernel holds W and U for 128 heads x 2F slots on chip: it takes
-  // k <= 255 (2F <= 256 slots, in 64-slot swizzle atoms) and up to 64 exact dims per head.
+  // The tensor-core split kernel runs exactly when the plan laid E out token-major (k <=
+  // 255, so W and U of 128 heads x 2F <= 256 slots fit on chip; G in {1, 2, 4}; at most
+  // 32 retained dims per KV head).
   c->tc_F2 = ((2 * c->F + 63) / 64) * 64;
-  c->tc = (M > 0 && c->tc_F2 <= 256 && de_ld_max <= 64) ? 1 : 0;
+  c->tc = (M > 0 && plan->e_token_major) ? 1 : 0;
   int cols = 32;
   while (cols < c->tc_F2 + 64) cols <<= 1;
   c->tc_tmem_cols = cols;
@@ -723,10 +600,8 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
     if (requested > 0) {
       ns = requested < ntiles ? requested : ntiles;
     } else {
-      int dev = 0, sms = 148, occ = 1;
-      cudaError_t e = cudaGetDevice(&dev);
-      if (e != cudaSuccess) return e;
-      e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+      int sms = 148, occ = 1;
+      cudaError_t e = device_sm_count(&sms);
       if (e != cudaSuccess) return e;
       if (c->tc) {
         occ = 1;  // one CTA per SM (shared memory)
@@ -836,13 +711,14 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     decode_prologue_kernel<<<n_heads, DNT, plan->G * FA_HEAD_DIM * 4, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (c.tc && p.n_splits > 0) {
-    // middle span on the tensor cores; the CUDA-core kernel below then only runs the
-    // sink / recent CTAs
-    if ((e = launch_decode_tc(p, c.de_ld_max, stream)) != cudaSuccess) return e;
-    p.n_mid = 0;
+  if (c.tc) {
+    // middle span on the tensor cores, sink / recent rows as extra CTAs of the same grid
+    p.e_row = plan->e_pitch[0];
+    if ((e = launch_decode_tc(p, plan->de_ld[0], stream)) != cudaSuccess) return e;
+  } else if (plan->e_token_major && plan->M > 0) {
+    return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only
   }
-  const int grid = p.n_mid + n_heads * c.n_fsplits;
+  const int grid = c.tc ? 0 : p.n_mid + n_heads * c.n_fsplits;
   if (grid > 0) {
     int occ = 0;
     if (c.SPT == 1) {
@@ -857,11 +733,8 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if (c.smem_combine > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)c.smem_combine);
-    if (e != cudaSuccess) return e;
-  }
+  e = raise_smem_limit(reinterpret_cast<const void*>(decode_combine_kernel), (int)c.smem_combine);
+  if (e != cudaSuccess) return e;
   decode_combine_kernel<<<n_heads, 128, c.smem_combine, stream>>>(p);
   return cudaGetLastError();
 }

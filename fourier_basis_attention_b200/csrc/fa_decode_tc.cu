@@ -8,20 +8,31 @@
 //     U^T[heads x slots]  += P^T[heads x tokens] . Phi_t        (MMA 2, accumulates over tiles)
 // where W holds sigma log2(e) s_f (C_K^T q_c) per slot and Phi_t the unit-amplitude
 // cos / sin of the tile's tokens. Operands are fp16: Phi_t lies in [-1, 1]; P is stored as
-// 2^12 p, so probabilities down to 2^-26 stay normal (U carries the 2^12 until the record
-// is written); W is scaled per head by a power of two to at most 1 in magnitude and split
-// into hi + lo (lo = W - hi), so S takes two MMAs (W_hi . Phi^T + W_lo . Phi^T). The score
-// error is then ~2^-22 relative and the value error ~2^-12 per term, far inside the 3e-3
-// output bar (one plain fp16 or tf32 pass for S would leave only a 5x margin). One buffer per
-// tile holds Phi_t as [token][slot] with 128-byte swizzle: MMA 1 reads it as its K-major B
-// operand, MMA 2 as its MN-major B operand (the layout compress uses for the cache rows).
+// 2^7 p with p <= 2^8 (lazy max below), so it stays normal down to p = 2^-21 (U carries
+// the 2^7 until the record is written); W is scaled per head by a power of two to at most
+// 1 in magnitude and split into hi + lo (lo = W - hi), so S takes two MMAs
+// (W_hi . Phi^T + W_lo . Phi^T). The score error is then ~2^-22 relative and the value
+// error ~2^-12 per term, far inside the 3e-3 output bar (one plain fp16 or tf32 pass for S
+// would leave only a 5x margin). One buffer per tile holds Phi_t as [token][slot] with
+// 128-byte swizzle: MMA 1 reads it as its K-major B operand, MMA 2 as its MN-major B
+// operand (the layout compress uses for the cache rows).
 //
-// Warp roles: warp 0 = TMEM owner and MMA issuer (one thread); warps 1-4 = head threads
-// (thread = TMEM lane = query head): exact-dim dot products, online softmax, P rows,
-// U rescaling, the split record; warps 5-7 = basis generators (thread = token and a third
-// of the frequencies; rotation recurrence over the frequencies, re-seeded every 32 of them
-// from the exactly reduced phase). Tiles are double-buffered (Phi, P, S); every wait is
-// bounded.
+// Warp roles: warp 0 = TMEM owner and MMA issuer (one thread); warps 1-4 = head warps,
+// each owning the 32 query heads of its TMEM lane quadrant; warps 5-7 = basis generators
+// (thread = frequency; rotation recurrence along the tile's tokens, started each tile from
+// the exactly reduced phase). Tiles are double-buffered (Phi, P, S); every wait is bounded.
+//
+// Exact dims: this kernel runs on token-major E (the plan lays E out so that token t of a
+// batch is one row holding every KV head's retained dims, w = 8, 16 or 32 per head). Per
+// token a head warp reads the w-element slices of its 32 / G KV heads as one coalesced row
+// segment, lane = (KV head, 16-byte chunk); the G query heads of a KV head share the load.
+// Dot products are reduced over a KV head's chunk lanes with shuffles and handed to the
+// head lanes through a per-warp [head][token] buffer, which then carries p back; the value
+// accumulator stays distributed (lane = KV head, chunk, query head) until the record is
+// written. Softmax, P rows, U rescaling and (m, l) are per head lane.
+//
+// CTAs [0, B Hkv n_fsplits) of the grid run the sink / recent rows on the CUDA cores
+// (decode_sink_recent), so one launch covers every split record.
 #include "fa_decode_common.cuh"
 
 namespace fa {
@@ -31,39 +42,72 @@ constexpr int TC_T = 32;        // tokens per tile
 constexpr int TC_THREADS = 256; // 8 warps
 constexpr int TC_GEN = 96;      // generator threads (warps 5-7)
 
+// The reference max is raised lazily: only when a tile's max exceeds it by more than
+// TC_LAZY (log2 units) are U, the value accumulator and the sum rescaled, so the head
+// warps rarely wait for the previous tile's MMA 2. p = 2^(s - m_ref) <= 2^8, stored as
+// 2^7 p <= 2^15 in fp16.
+constexpr float TC_LAZY = 8.0f;
+constexpr float TC_P_SCALE = 128.0f;
+constexpr float TC_P_UNSCALE = 1.0f / 128.0f;
+
+constexpr int TC_XS_LD = 33;    // row pitch (floats) of the per-warp [head][token] buffer
+
 struct TcLayout {
-  int w, phi, p, misc, total;  // byte offsets from the 1024-aligned base
+  int w, phi, p, xs, misc, total;  // byte offsets from the 1024-aligned base
 };
 
 // W: hi then lo, each [F2/64 atoms][128 heads][64 fp16] (K-major, 128-byte swizzle)
 // Phi: 2 buffers of [F2/64 atoms][32 tokens][64 fp16] (128-byte swizzle)
 // P: 2 buffers of [128 heads][32 fp16] (K-major, 64-byte swizzle)
+// xs: per head warp [32 heads][TC_XS_LD] fp32: exact-dim scores, then p, of the tile
 __host__ __device__ inline TcLayout tc_layout(int F2) {
   TcLayout L;
   L.w = 0;
   L.phi = L.w + 2 * TC_NH * F2 * 2;
   L.p = L.phi + 2 * TC_T * F2 * 2;
-  L.misc = L.p + 2 * TC_NH * TC_T * 2;
+  L.xs = L.p + 2 * TC_NH * TC_T * 2;
+  L.misc = L.xs + 4 * 32 * TC_XS_LD * 4;
   L.total = L.misc + 256 + 1024;  // + alignment slack
   return L;
 }
 
-constexpr float TC_P_SCALE = 4096.0f;          // P is stored as 2^12 p
-constexpr float TC_P_UNSCALE = 1.0f / 4096.0f;
+size_t decode_tc_smem_bytes(int F2) {
+  const size_t b = (size_t)tc_layout(F2).total;
+  return b > sink_recent_smem_bytes() ? b : sink_recent_smem_bytes();
+}
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-size_t decode_tc_smem_bytes(int F2) { return (size_t)tc_layout(F2).total; }
+// Lane layout of a head warp's exact-dim work. CPS = 16-byte chunks per KV-head slice of
+// a token row (w / 8), G = query heads per KV head. Per step the warp covers TT tokens;
+// lane l, load r handles chunk (32 r + l) % CH: KV head / CPS, chunk % CPS, and token
+// l / CH of the step (all warp-local).
+template <int CPS, int G>
+struct EMap {
+  static constexpr int NK = 32 / G;                                  // KV heads per warp
+  static constexpr int CH = CPS > 0 ? NK * CPS : 32;                 // chunks per token
+  static constexpr int TT = CH >= 32 ? 1 : 32 / CH;                  // tokens per step
+  static constexpr int NI = CH >= 32 ? CH / 32 : 1;                  // loads per lane per step
+  static constexpr int NS = TC_T / TT;                               // steps per tile
+  static constexpr int U = 8 / NI;                                   // steps per load batch
+  static constexpr int CPS1 = CPS > 0 ? CPS : 1;
+};
 
-template <int DE>
+template <int CPS, int G>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     decode_tc_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int n_f = p.B * p.Hkv * p.n_fsplits;  // sink / recent CTAs come first
+  if ((int)blockIdx.x < n_f) {
+    decode_sink_recent(p, reinterpret_cast<float*>(smem), blockIdx.x);
+    return;
+  }
+  const int cta = blockIdx.x - n_f;
   const int F2 = p.tc_F2;
   const TcLayout Ly = tc_layout(F2);
   uint8_t* Ws = smem + Ly.w;      // hi at Ws, lo at Ws + w_half
@@ -76,14 +120,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint64_t* phi_full = bars;      // [2] generators -> MMA (count 3)
   uint64_t* phi_free = bars + 2;  // [2] MMA 2 done: Phi and P buffers reusable (commit)
   uint64_t* s_full = bars + 4;    // [2] MMA 1 done (commit)
-  uint64_t* p_full = bars + 6;    // [2] head threads -> MMA (count 4)
+  uint64_t* p_full = bars + 6;    // [2] head warps -> MMA (count 4)
   uint64_t* u_done = bars + 8;    // last MMA 2 done (commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hg = blockIdx.x / p.n_splits;
-  const int sp = blockIdx.x - hg * p.n_splits;
+  const int hg = cta / p.n_splits;
+  const int sp = cta - hg * p.n_splits;
   const int lo = sp * p.split_len;
   const int hi = min(p.M, lo + p.split_len);
   const int ntiles = (hi - lo + TC_T - 1) / TC_T;
@@ -105,7 +149,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tmem_alloc(tmem_slot, p.tc_tmem_cols);
     tmem_relinquish();
   }
-  // head threads: W rows, scaled by 2^-e to at most 1 in magnitude, split into fp16 hi / lo
+  // head warps: W rows, scaled by 2^-e to at most 1 in magnitude, split into fp16 hi / lo
   // and written into the K-major swizzled operand; S is scaled back by 2^e on readout
   const int h = (warp & 3) * 32 + lane;  // TMEM lane of a head thread
   const long long gh = (long long)hg * TC_NH + h;
@@ -151,7 +195,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (lane == 0) {
       const uint32_t idesc1 = idesc_f16_f32(TC_NH, TC_T, /*b_mn_major=*/false);
       const uint32_t idesc2 = idesc_f16_f32(TC_NH, F2, /*b_mn_major=*/true);
-      const uint32_t w_addr = smem_u32(Ws);
+      // descriptors of buffer 0; a byte offset x inside the (< 256 KB) shared window adds
+      // x >> 4 to the start-address field
+      const uint64_t d_w = smem_desc_sw128(smem_u32(Ws), 16, 1024);
+      // Phi as K-major B of MMA 1: 8-token groups 1024 bytes apart, 64-slot atoms
+      const uint64_t d_phik = smem_desc_sw128(smem_u32(PHI), 16, 1024);
+      // Phi as MN-major B of MMA 2: 64-slot atoms TC_T * 128 bytes apart (leading), 8-token
+      // groups 1024 bytes apart
+      const uint64_t d_phin = smem_desc_sw128(smem_u32(PHI), TC_T * 128, 1024);
+      // P: 64-byte rows (32 tokens), 8-row groups 512 bytes apart
+      const uint64_t d_p = smem_desc_sw64(smem_u32(PS), 16, 512);
+      const int nks = F2 / 16;
       bool ok = true;
       auto mma1 = [&](int i) {
         const int b = i & 1;
@@ -160,15 +214,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           return;
         }
         tc_fence_after();
-        const uint32_t phi_addr = smem_u32(PHI + b * phi_bytes);
-        for (int ks = 0; ks < F2 / 16; ++ks) {
+        const uint64_t dphi = d_phik + (uint64_t)((b * phi_bytes) >> 4);
+        const uint32_t ts = tmem_s + 32 * b;
+#pragma unroll 4
+        for (int ks = 0; ks < nks; ++ks) {
           // 16 slots = 32 bytes further along a swizzled 128-byte row; 64-slot atoms
-          const uint32_t koff = (uint32_t)((ks & 3) * 32);
-          const uint32_t wa = w_addr + (ks >> 2) * (TC_NH * 128) + koff;
-          const uint32_t pa = phi_addr + (ks >> 2) * (TC_T * 128) + koff;
-          const uint64_t bd = smem_desc_sw128(pa, 16, 1024);
-          mma_f16(tmem_s + 32 * b, smem_desc_sw128(wa, 16, 1024), bd, idesc1, ks > 0 ? 1u : 0u);
-          mma_f16(tmem_s + 32 * b, smem_desc_sw128(wa + w_half, 16, 1024), bd, idesc1, 1u);
+          const uint32_t ow = (uint32_t)(((ks >> 2) * (TC_NH * 128) + (ks & 3) * 32) >> 4);
+          const uint32_t op = (uint32_t)(((ks >> 2) * (TC_T * 128) + (ks & 3) * 32) >> 4);
+          mma_f16(ts, d_w + ow, dphi + op, idesc1, ks > 0 ? 1u : 0u);
+          mma_f16(ts, d_w + ow + (uint32_t)(w_half >> 4), dphi + op, idesc1, 1u);
         }
         mma_commit(&s_full[b]);
       };
@@ -184,17 +238,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(PS + b * p_bytes);
-        const uint32_t phi_addr = smem_u32(PHI + b * phi_bytes);
-        for (int ks = 0; ks < TC_T / 16; ++ks) {
-          // P: 64-byte rows (32 tokens), 8-row groups 512 bytes apart; 16 tokens = 32 bytes
-          const uint32_t pa = p_addr + ks * 32;
-          // Phi as MN-major B: 64-slot atoms TC_T * 128 bytes apart (leading), 8-token
-          // groups 1024 bytes apart; 16 tokens = two groups
-          mma_f16(tmem_u, smem_desc_sw64(pa, 16, 512),
-                   smem_desc_sw128(phi_addr + ks * 2048, TC_T * 128, 1024), idesc2,
-                   (i > 0 || ks > 0) ? 1u : 0u);
-        }
+        // 16 tokens per MMA: 32 bytes along the P rows, two 8-token groups of Phi
+#pragma unroll
+        for (int ks = 0; ks < TC_T / 16; ++ks)
+          mma_f16(tmem_u, d_p + (uint64_t)((b * p_bytes + ks * 32) >> 4),
+                  d_phin + (uint64_t)((b * phi_bytes + ks * 2048) >> 4), idesc2,
+                  (i > 0 || ks > 0) ? 1u : 0u);
         mma_commit(&phi_free[b]);
       }
       // TMEM is released only after every MMA of this CTA has completed
@@ -205,39 +254,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else if (warp >= 5) {
     // -------------------------------------------------------------------- basis generators
-    // thread: token tau of the tile and one third of the frequencies, two per 16-byte store
+    // thread gt: frequencies gt and gt + 96; per tile the unit phasor of f (t0 + tau) / M
+    // for tau = 0 .. 31 by rotation, started from the exactly reduced phase f t0 mod M.
+    // Slots 2f (cos) and 2f + 1 (sin) are one fp16 pair: atom f / 32, byte 4 (f % 32) of
+    // the token's 128-byte row, 16-byte chunk swizzled by the token.
     const int gt = threadIdx.x - 160;
-    const int tau = gt & 31, part = gt >> 5;  // part 0..2
-    const int npair = F2 / 4;                 // frequency pairs (f, f+1), f even
-    const int per = (npair + 2) / 3;
-    const int pa = part * per, pb = min(npair, pa + per);
+    const int nf = F2 / 2;
+    float ra[2], rb[2];  // cos, sin of 2 pi f / M
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int f = gt + TC_GEN * u;
+      ra[u] = 1.0f;
+      rb[u] = 0.0f;
+      if (f < nf) phase_sincos(f % M, M, p.two_over_M, &rb[u], &ra[u]);
+    }
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
       if (i >= 2 &&
           !mbar_wait(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag, WD_DECODE | 4u))
         break;
-      const long long tm = (long long)lo + i * TC_T + tau;  // middle-relative token
-      uint8_t* base = PHI + b * phi_bytes + tau * 128;
-      if (pa < pb) {
-        float sa, ca;  // rotation by 2 pi tm / M per frequency step
-        phase_sincos(tm % M, M, p.two_over_M, &sa, &ca);
-        for (int q0 = pa; q0 < pb; q0 += 16) {
+      const long long tm0 = (long long)lo + i * TC_T;  // middle-relative first token
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int f = gt + TC_GEN * u;
+        if (f < nf) {
           float s, c;
-          phase_sincos(((long long)(2 * q0) * tm) % M, M, p.two_over_M, &s, &c);
-          const int q1 = min(pb, q0 + 16);
-          for (int q = q0; q < q1; ++q) {
-            const float c0 = c, s0 = s;
-            float cn = c * ca - s * sa;
-            s = s * ca + c * sa;
+          phase_sincos(((long long)f * tm0) % M, M, p.two_over_M, &s, &c);
+          uint8_t* base = PHI + b * phi_bytes + (f >> 5) * (TC_T * 128) + 4 * (f & 3);
+          const int chunk = (f & 31) >> 2;
+#pragma unroll 8
+          for (int tau = 0; tau < TC_T; ++tau) {
+            *reinterpret_cast<uint32_t*>(base + tau * 128 + ((chunk ^ (tau & 7)) << 4)) =
+                pack_half2(c, s);
+            const float cn = c * ra[u] - s * rb[u];
+            s = s * ra[u] + c * rb[u];
             c = cn;
-            const float c1 = c, s1 = s;
-            cn = c * ca - s * sa;
-            s = s * ca + c * sa;
-            c = cn;
-            // slots 4q .. 4q+3: atom 4q / 64, 16-byte chunk (4q % 64) / 8 swizzled by token
-            const int atom = q >> 4, chunk = (q & 15) >> 1;
-            const int off = atom * (TC_T * 128) + ((chunk ^ (tau & 7)) << 4) + (q & 1) * 8;
-            *reinterpret_cast<uint2*>(base + off) = make_uint2(pack_half2(c0, s0), pack_half2(c1, s1));
           }
         }
       }
@@ -246,74 +297,143 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (lane == 0) mbar_arrive(&phi_full[b]);
     }
   } else {
-    // -------------------------------------------------------------------- head threads
+    // -------------------------------------------------------------------- head warps
+    using EM = EMap<CPS, G>;
+    constexpr int NI = EM::NI;
     const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
-    const int bi = hvalid ? (int)(gh / p.Hq) : 0;
-    const int hq = hvalid ? (int)(gh - (long long)bi * p.Hq) : 0;
-    const int g = hq / p.G;
-    const long long ebase = (long long)bi * p.e_batch + p.e_off[g];
-    const int dle = hvalid ? p.de_ld[g] : 0;
-    const bool leader = hvalid && (hq % p.G) == 0;  // prefetches the group's rows
-    float qe[DE], acc[DE];
+    const long long gbase = (long long)hg * TC_NH + (warp & 3) * 32;  // head of lane 0
+    const int nvalid = (int)max(0LL, min(32LL, bhq - gbase));
+    const int tau_l = EM::TT > 1 ? lane / EM::CH : 0;  // token of this lane within a step
+    // per load r: the lane's KV head (warp-local), its element offset, q_e, accumulator
+    int kap[NI], c8r[NI], de_r[NI];
+    bool ev[NI];
+    long long eoff[NI];
+    uint32_t qv[NI][G][4];  // q_e as bf16 pairs (exact: the query is bf16), unscaled
+    float accv[NI][G][8];
 #pragma unroll
-    for (int d = 0; d < DE; ++d) {
-      qe[d] = (d < dle) ? p.qw[gh * p.qw_stride + d] : 0.0f;
-      acc[d] = 0.0f;
+    for (int r = 0; r < NI; ++r) {
+      const int q = (32 * r + lane) % EM::CH;
+      const int k_ = q / EM::CPS1;
+      const int c_ = q % EM::CPS1;
+      kap[r] = k_;
+      c8r[r] = c_ * 8;
+      ev[r] = CPS > 0 && k_ * G < nvalid;
+      const long long gh0 = gbase + (long long)k_ * G;
+      const int bb = ev[r] ? (int)(gh0 / p.Hq) : 0;
+      const int gg = ev[r] ? (int)(gh0 - (long long)bb * p.Hq) / G : 0;
+      eoff[r] = (long long)bb * p.e_batch + p.e_off[gg] + c_ * 8;
+      de_r[r] = ev[r] ? p.de[gg] - c_ * 8 : 0;  // valid dims of this chunk (may be <= 0)
+#pragma unroll
+      for (int hq = 0; hq < G; ++hq) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          uint32_t pr = 0;
+          for (int u = 0; u < 2; ++u) {
+            const int d = c_ * 8 + 2 * e + u;  // retained-dim index
+            if (ev[r] && d < p.de[gg]) {
+              const int dim = p.perm[gg][p.dc[gg] + d];
+              pr |= (uint32_t)__bfloat16_as_ushort(p.q[(gh0 + hq) * FA_HEAD_DIM + dim]) << (16 * u);
+            }
+          }
+          qv[r][hq][e] = pr;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) accv[r][hq][e] = 0.0f;
+      }
     }
     float m = -INFINITY, l = 0.0f;
-    constexpr int UT = DE <= 32 ? 2 : 1;  // tokens whose rows are in flight together
     bool ok = true;
+    float* xs = reinterpret_cast<float*>(smem + Ly.xs) + (warp - 1) * 32 * TC_XS_LD;
+    const int c_first = ((lane % EM::CH) % EM::CPS1) == 0;  // first chunk lane of its KV head
+
+    // chunks of step s (tokens s * TT + tau_l of the tile) of tensor E
+    auto load_step = [&](const __nv_bfloat16* E, int t0, int nt, int s, uint4 (&x)[NI]) {
+      const int tok = s * EM::TT + tau_l;
+      const long long trow = (long long)(t0 + tok) * p.e_row;
+#pragma unroll
+      for (int r = 0; r < NI; ++r)
+        x[r] = (ev[r] && tok < nt) ? __ldg(reinterpret_cast<const uint4*>(E + eoff[r] + trow))
+                                   : make_uint4(0, 0, 0, 0);
+    };
+
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
       const int t0 = lo + i * TC_T;
       const int nt = min(TC_T, hi - t0);
-      if (leader && i + 1 < ntiles && dle > 0) {
-        const int tn = t0 + TC_T;
-        const int nb = min(TC_T, hi - tn);
-        prefetch_l2_bulk(p.EK + ebase + (long long)tn * dle, (uint32_t)(nb * dle * 2));
-        prefetch_l2_bulk(p.EV + ebase + (long long)tn * dle, (uint32_t)(nb * dle * 2));
+      if constexpr (CPS > 0) {
+        if (i + 1 < ntiles && nvalid > 0) {  // next tile's rows of this warp's batches -> L2
+          const int tn = t0 + TC_T;
+          const int nb = min(TC_T, hi - tn);
+          const int b0 = (int)(gbase / p.Hq), b1 = (int)((gbase + nvalid - 1) / p.Hq);
+          for (int bb = b0 + lane; bb <= b1; bb += 32) {
+            const long long o = (long long)bb * p.e_batch + (long long)tn * p.e_row;
+            prefetch_l2_bulk(p.EK + o, (uint32_t)(nb * p.e_row * 2));
+            prefetch_l2_bulk(p.EV + o, (uint32_t)(nb * p.e_row * 2));
+          }
+        }
+        // exact-dim scores: per step, dot products of the lane's chunks with q_e, summed
+        // over the KV head's CPS chunk lanes, into xs[query head][token]
+#pragma unroll 1
+        for (int s0 = 0; s0 < EM::NS; s0 += EM::U) {
+          uint4 x[EM::U][NI];
+#pragma unroll
+          for (int u = 0; u < EM::U; ++u) load_step(p.EK, t0, nt, s0 + u, x[u]);
+#pragma unroll
+          for (int u = 0; u < EM::U; ++u) {
+            float part[NI][G];
+#pragma unroll
+            for (int r = 0; r < NI; ++r) {
+              float xf[8];
+              bf16x8_to_f32(x[u][r], xf);
+#pragma unroll
+              for (int hq = 0; hq < G; ++hq) {
+                float a = 0.0f;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  a += __uint_as_float(qv[r][hq][e] << 16) * xf[2 * e];
+                  a += __uint_as_float(qv[r][hq][e] & 0xFFFF0000u) * xf[2 * e + 1];
+                }
+                part[r][hq] = a;
+              }
+            }
+#pragma unroll
+            for (int o = 1; o < CPS; o <<= 1)
+#pragma unroll
+              for (int r = 0; r < NI; ++r)
+#pragma unroll
+                for (int hq = 0; hq < G; ++hq)
+                  part[r][hq] += __shfl_xor_sync(0xffffffffu, part[r][hq], o);
+            if (c_first) {
+              const int tok = (s0 + u) * EM::TT + tau_l;
+#pragma unroll
+              for (int r = 0; r < NI; ++r)
+#pragma unroll
+                for (int hq = 0; hq < G; ++hq)
+                  xs[(kap[r] * G + hq) * TC_XS_LD + tok] = part[r][hq] * p.qscale;
+            }
+          }
+        }
+        __syncwarp();
       }
+      float sc[TC_T];
+#pragma unroll
+      for (int t = 0; t < TC_T; ++t) sc[t] = CPS > 0 ? xs[lane * TC_XS_LD + t] : 0.0f;
       ok = mbar_wait(&s_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, WD_DECODE | 5u) && ok;
       __syncwarp();  // tcgen05.ld is warp-collective
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld_32x32b_x32(tmem_s + lanebase + 32 * b, sr);
       tmem_ld_wait();
-      float sc[TC_T];
 #pragma unroll
-      for (int t = 0; t < TC_T; ++t) sc[t] = __uint_as_float(sr[t]) * w_unscale;
-      // exact dims of the middle tokens
-      const __nv_bfloat16* ek = p.EK + ebase + (long long)t0 * dle;
-#pragma unroll 1  // bounded loads in flight (register budget)
-      for (int t8 = 0; t8 < TC_T; t8 += UT) {
-        uint4 rows[UT][DE / 8];
-#pragma unroll
-        for (int u = 0; u < UT; ++u)
-#pragma unroll
-          for (int c8 = 0; c8 < DE / 8; ++c8)
-            rows[u][c8] = (t8 + u < nt && c8 * 8 < dle)
-                              ? *reinterpret_cast<const uint4*>(ek + (long long)(t8 + u) * dle + c8 * 8)
-                              : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < UT; ++u) {
-          float e = 0.0f;
-#pragma unroll
-          for (int c8 = 0; c8 < DE / 8; ++c8) {
-            float x[8];
-            bf16x8_to_f32(rows[u][c8], x);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) e += qe[c8 * 8 + j] * x[j];
-          }
-          sc[t8 + u] += e;
-        }
-      }
+      for (int t = 0; t < TC_T; ++t)
+        sc[t] = hvalid ? __uint_as_float(sr[t]) * w_unscale + sc[t] : 0.0f;
       float tmax = -INFINITY;
 #pragma unroll
       for (int t = 0; t < TC_T; ++t) {
         if (t >= nt) sc[t] = -INFINITY;
         tmax = fmaxf(tmax, sc[t]);
       }
-      const float m_new = fmaxf(m, tmax);
+      const float m_new = (tmax > m + TC_LAZY) ? tmax : m;  // m = -inf: the first tile's max
       const float alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
       float psum = 0.0f;
 #pragma unroll
@@ -323,7 +443,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       l = l * alpha + psum;
       m = m_new;
-      // U^T rows of heads whose running max rose are rescaled before MMA 2 of this tile
+      // a head whose reference max rose rescales its U^T row (after the previous tile's
+      // MMA 2) and its value accumulators
       const bool need = i > 0 && alpha < 1.0f;
       if (__any_sync(0xffffffffu, need)) {
         const bool w_ok = mbar_wait(&phi_free[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u,
@@ -342,34 +463,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           tmem_st_32x32b_x32(tmem_u + lanebase + c * 32, r);
         }
         tmem_st_wait();
-      }
-      // exact-dim values
-      const __nv_bfloat16* ev = p.EV + ebase + (long long)t0 * dle;
 #pragma unroll
-      for (int d = 0; d < DE; ++d) acc[d] *= alpha;
-#pragma unroll 1  // bounded loads in flight (register budget)
-      for (int t8 = 0; t8 < TC_T; t8 += UT) {
-        uint4 rows[UT][DE / 8];
+        for (int r = 0; r < NI; ++r)
 #pragma unroll
-        for (int u = 0; u < UT; ++u)
+          for (int hq = 0; hq < G; ++hq) {
+            const float ah = __shfl_sync(0xffffffffu, a, kap[r] * G + hq);
 #pragma unroll
-          for (int c8 = 0; c8 < DE / 8; ++c8)
-            rows[u][c8] = (t8 + u < nt && c8 * 8 < dle)
-                              ? *reinterpret_cast<const uint4*>(ev + (long long)(t8 + u) * dle + c8 * 8)
-                              : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int u = 0; u < UT; ++u) {
-          const float pv = sc[t8 + u];
-#pragma unroll
-          for (int c8 = 0; c8 < DE / 8; ++c8) {
-            float x[8];
-            bf16x8_to_f32(rows[u][c8], x);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) acc[c8 * 8 + j] += pv * x[j];
+            for (int e = 0; e < 8; ++e) accv[r][hq][e] *= ah;
           }
-        }
       }
-      // P^T row of this head (fp16, 2^12 p) into buffer b, once MMA 2 of tile i-2 released it
+      // P^T row of this head (fp16, 2^7 p) into buffer b, once MMA 2 of tile i-2 released it
       if (i >= 2) {
         const bool w_ok = mbar_wait(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag,
                                     WD_DECODE | 7u);
@@ -390,18 +493,69 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
+      if constexpr (CPS > 0) {
+        // p of this head for the exact-dim values
+#pragma unroll
+        for (int t = 0; t < TC_T; ++t) xs[lane * TC_XS_LD + t] = sc[t];
+        __syncwarp();
+        // exact-dim values: accv[r][hq] += p(head kap G + hq, token) E_V chunk
+#pragma unroll 1
+        for (int s0 = 0; s0 < EM::NS; s0 += EM::U) {
+          uint4 x[EM::U][NI];
+#pragma unroll
+          for (int u = 0; u < EM::U; ++u) load_step(p.EV, t0, nt, s0 + u, x[u]);
+#pragma unroll
+          for (int u = 0; u < EM::U; ++u) {
+            const int tok = (s0 + u) * EM::TT + tau_l;
+#pragma unroll
+            for (int r = 0; r < NI; ++r) {
+              float xf[8];
+              bf16x8_to_f32(x[u][r], xf);
+#pragma unroll
+              for (int hq = 0; hq < G; ++hq) {
+                const float pv = xs[(kap[r] * G + hq) * TC_XS_LD + tok];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) accv[r][hq][e] += pv * xf[e];
+              }
+            }
+          }
+        }
+        __syncwarp();  // xs is rewritten by the next tile's scores
+      }
     }
     // split record: running max, sum, exact-dim values, U
     const bool done = ntiles == 0 || mbar_wait(u_done, 0, abort_flag, WD_DECODE | 8u);
+    const bool all_ok = __all_sync(0xffffffffu, ok && done);
     __syncwarp();
     tc_fence_after();
-    float* rec = p.rec + ((long long)sp * bhq + gh) * p.rec_stride;
-    if (hvalid && ok && done) {
+    if (hvalid && all_ok) {
+      float* rec = p.rec + ((long long)sp * bhq + gh) * p.rec_stride;
       rec[0] = m;
       rec[1] = l;
+    }
+    if constexpr (CPS > 0) {
 #pragma unroll
-      for (int d = 0; d < DE; ++d)
-        if (d < dle) rec[4 + d] = acc[d];
+      for (int o = EM::CH; o < 32; o <<= 1)  // sum over the step's token lanes
+#pragma unroll
+        for (int r = 0; r < NI; ++r)
+#pragma unroll
+          for (int hq = 0; hq < G; ++hq)
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              accv[r][hq][e] += __shfl_xor_sync(0xffffffffu, accv[r][hq][e], o);
+      if (tau_l == 0 && all_ok) {
+#pragma unroll
+        for (int r = 0; r < NI; ++r) {
+          if (!ev[r]) continue;
+#pragma unroll
+          for (int hq = 0; hq < G; ++hq) {
+            float* rec = p.rec + ((long long)sp * bhq + gbase + kap[r] * G + hq) * p.rec_stride;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              if (e < de_r[r]) rec[4 + c8r[r] + e] = accv[r][hq][e];
+          }
+        }
+      }
     }
     const int nslot = 2 * p.F_pad;
 #pragma unroll 1
@@ -409,7 +563,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t r[32];
       tmem_ld_32x32b_x32(tmem_u + lanebase + c * 32, r);
       tmem_ld_wait();
-      if (hvalid && ok && done) {
+      if (hvalid && all_ok) {
+        float* rec = p.rec + ((long long)sp * bhq + gh) * p.rec_stride;
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
           const int slot = c * 32 + j;
@@ -432,21 +587,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 }
 
-cudaError_t launch_decode_tc(const DecodeParams& p, int de_max, cudaStream_t stream) {
+template <int CPS, int G>
+static cudaError_t launch_tc(const DecodeParams& p, int grid, int smem, cudaStream_t stream) {
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(decode_tc_kernel<CPS, G>), smem);
+  if (e != cudaSuccess) return e;
+  decode_tc_kernel<CPS, G><<<grid, TC_THREADS, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+template <int CPS>
+static cudaError_t launch_tc_g(const DecodeParams& p, int grid, int smem, cudaStream_t stream) {
+  switch (p.G) {
+    case 1: return launch_tc<CPS, 1>(p, grid, smem, stream);
+    case 2: return launch_tc<CPS, 2>(p, grid, smem, stream);
+    case 4: return launch_tc<CPS, 4>(p, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream) {
   const int smem = (int)decode_tc_smem_bytes(p.tc_F2);
   const int heads = p.B * p.Hq;
-  const int grid = ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
-  cudaError_t e;
-  if (de_max <= 32) {
-    e = cudaFuncSetAttribute(decode_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_tc_kernel<32><<<grid, TC_THREADS, smem, stream>>>(p);
-  } else {
-    e = cudaFuncSetAttribute(decode_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e != cudaSuccess) return e;
-    decode_tc_kernel<64><<<grid, TC_THREADS, smem, stream>>>(p);
+  const int grid = p.B * p.Hkv * p.n_fsplits + ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
+  switch (de_slot) {
+    case 0: return launch_tc_g<0>(p, grid, smem, stream);
+    case 8: return launch_tc_g<1>(p, grid, smem, stream);
+    case 16: return launch_tc_g<2>(p, grid, smem, stream);
+    case 32: return launch_tc_g<4>(p, grid, smem, stream);
+    default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 }  // namespace fa

@@ -28,6 +28,13 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
 cudaError_t read_and_clear_watchdog(unsigned int* word);
 cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream);
 
+// Per-device launch facts, queried once and cached (fa_runtime.cu).
+cudaError_t device_sm_count(int* sms);
+// Raises `func`'s dynamic shared-memory limit to at least `bytes` on the current device.
+cudaError_t raise_smem_limit(const void* func, int bytes);
+// Resident blocks per SM of `func` at `threads` threads and `smem` dynamic shared bytes.
+cudaError_t cached_occupancy(const void* func, int threads, size_t smem, int* blocks);
+
 // Records `msg` as the calling thread's fa_last_error() text and returns `code`.
 int set_last_error(int code, const char* msg);
 

@@ -74,16 +74,26 @@ typedef struct fa_shape {
  * Hybrid cache layout (element offsets; F and E bf16, C fp32):
  *   F (sink + recent rows, all dims): [B][Hkv][S + R][128]; row i < S is token i, row
  *     S + i is token L - R + i.
- *   E (middle rows, retained dims): block of KV head (b, g) starts at
- *     b * e_batch + e_off[g] and is [M][de_ld[g]] row-major; columns [de[g], de_ld[g])
- *     are zero.
+ *   E (middle rows, retained dims): element (b, g, t, i) of middle token t and retained
+ *     dim i < de_ld[g] sits at b * e_batch + e_off[g] + t * e_pitch[g] + i; columns
+ *     [de[g], de_ld[g]) are zero. Two arrangements:
+ *     e_token_major = 0: one dense [M][de_ld[g]] block per KV head (e_pitch[g] = de_ld[g],
+ *       de_ld[g] = de[g] rounded up to a multiple of 8, blocks in KV-head order);
+ *     e_token_major = 1: the rows of all KV heads of a batch interleaved per token, so
+ *       that token t of batch b is one contiguous row of Hkv * w elements (de_ld[g] = w
+ *       for every g, e_off[g] = g * w, e_pitch[g] = Hkv * w, w = 8, 16 or 32, the
+ *       smallest that holds every de[g]; w = 0 when every dim is compressed).
+ *     fa_plan_init chooses token-major exactly when fa_decode will run the middle span on
+ *     the tensor cores: middle span present, k <= 255, G in {1, 2, 4}, every de[g] <= 32,
+ *     k * G >= 500 and B * Hq >= 128 (a warp then reads one token's retained dims of 32
+ *     query heads as one coalesced row).
  *   C (Fourier coefficients of the middle rows, compressed dims, fp32): block of (b, g)
  *     starts at b * c_batch + c_off[g] and is [kk][dc_ld[g]] row-major,
  *     kk = (M > 0 ? k : 0); columns [dc[g], dc_ld[g]) are zero. Row j is basis function j.
  *     C is kept in fp32: it holds k * dc values per head against M * de for E (about 2%
  *     of the cache at k = M / 128), and a bf16 C would add a second rounding of up to
  *     2^-8 relative to every reconstructed value.
- * de_ld / dc_ld are de / dc rounded up to a multiple of 8 (rows of 16 / 32 bytes).
+ * dc_ld is dc rounded up to a multiple of 8 (rows of 32 bytes).
  *
  * Basis table (fa_build_basis) row stride: phi_ld = M rounded up to a multiple of 8.
  */
@@ -91,8 +101,10 @@ typedef struct fa_plan {
   fa_shape shape;
   int32_t S, R, M, kk, G;
   int32_t phi_ld;
+  int32_t e_token_major;
   int32_t dc[FA_MAX_KV_HEADS], de[FA_MAX_KV_HEADS];
   int32_t dc_ld[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS];
+  int32_t e_pitch[FA_MAX_KV_HEADS];
   int64_t c_off[FA_MAX_KV_HEADS], e_off[FA_MAX_KV_HEADS];
   int64_t c_batch, e_batch;
   int64_t f_elems, e_elems, c_elems; /* elements of each of F_K/F_V, E_K/E_V, C_K/C_V */

@@ -36,11 +36,32 @@ def test_library_exports_every_declared_function():
         assert hasattr(fa.LIB, n)
 
 
-def test_plan_struct_matches_header_size():
-    # fa_plan is plain data; the ctypes mirror must have the C layout the header implies
-    assert ctypes.sizeof(fa.fa_shape) == 32
-    expected = 32 + 6 * 4 + 4 * 4 * 64 + 2 * 8 * 64 + 5 * 8 + 64 * 128
-    assert ctypes.sizeof(fa.fa_plan) == expected
+def test_plan_struct_matches_header_layout(tmp_path):
+    """The ctypes mirrors have the C layout of the header: gcc compiles the header and
+    prints sizeof and every field's offsetof, which must equal the ctypes ones."""
+    structs = {"fa_shape": fa.fa_shape, "fa_plan": fa.fa_plan, "fa_cache": fa.fa_cache}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fourier_attention.h"',
+             "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append(f'  printf("{name} sizeof %zu\\n", sizeof({name}));')
+        for field, _ in cls._fields_:
+            lines.append(f'  printf("{name} {field} %zu\\n", offsetof({name}, {field}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines) + "\n")
+    exe = tmp_path / "layout"
+    include = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c11", "-I", include, str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {}
+    for line in out:
+        if line.strip():
+            name, field, value = line.split()
+            got[(name, field)] = int(value)
+    for name, cls in structs.items():
+        assert got[(name, "sizeof")] == ctypes.sizeof(cls), name
+        for field, _ in cls._fields_:
+            assert got[(name, field)] == getattr(cls, field).offset, (name, field)
 
 
 @pytest.mark.parametrize("w", wl.CONFIGS + [wl.llama3_8b_layer(64, 131072, 5)], ids=lambda w: w.name)
@@ -155,5 +176,77 @@ def test_gpu_test_shapes_have_valid_plans():
     import test_gpu_parity as tg
     shapes = list(tg.SMALL) + list(tg.FULL)
     shapes.append(wl.shrink(wl.LLAMA3_8B_GQA_32K, B=1, Hq=8, Hkv=2, L=2000))
+    shapes.append(tg.TC_BASE)
+    shapes.append(tg.TC_WIDE)
+    for _, k in tg.TC_RAGGED:
+        shapes.append(tg._ragged_shape(k))
     for w in shapes:
         fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+
+
+# ----------------------------------------------------------------------------- E layout
+
+@pytest.mark.parametrize("w,token_major", [
+    (wl.SINGLE_HEAD_2K, False),                   # k = 63, G = 4: k G < 500
+    (wl.LLAMA2_7B_MHA_32K, False),                # k = 255, G = 1: k G < 500
+    (wl.LLAMA3_8B_GQA_32K, False),                # k = 511
+    (wl.LLAMA3_8B_GQA_128K, False),               # k = 1023
+    (wl.llama3_8b_layer(8, 8192, 2), False),      # k = 63
+    (wl.llama3_8b_layer(8, 32768, 2), True),      # k = 255, G = 4, 256 query heads
+    (wl.llama3_8b_layer(2, 32768, 2), False),     # 64 query heads
+    (wl.llama3_8b_layer(8, 131072, 2), False),    # k = 1023
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_token_major_choice(w, token_major):
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    assert bool(p.e_token_major) == token_major
+    if token_major:
+        width = p.de_ld[0]
+        assert width == 32 and all(p.de_ld[g] == width for g in range(w.Hkv))
+        for g in range(w.Hkv):
+            assert p.e_off[g] == g * width and p.e_pitch[g] == w.Hkv * width
+        assert p.e_batch == p.M * w.Hkv * width
+    else:
+        off = 0
+        for g in range(w.Hkv):
+            assert p.de_ld[g] == (p.de[g] + 7) // 8 * 8 and p.e_pitch[g] == p.de_ld[g]
+            assert p.e_off[g] == off
+            off += p.M * p.de_ld[g]
+        assert p.e_batch == off
+    assert p.e_elems == w.B * p.e_batch
+
+
+@pytest.mark.parametrize("retained,G,k,B,expect", [
+    ([5, 1, 3, 8], 4, 127, 8, 8), ([12, 9, 16, 0], 4, 255, 8, 16),
+    ([31, 17, 2, 20], 2, 255, 16, 32), ([0, 0, 0, 0], 4, 127, 8, 0),
+    ([33, 1, 1, 1], 4, 255, 8, None), ([8, 8, 8, 8], 8, 63, 8, None),
+    ([8, 8, 8, 8], 4, 257, 8, None), ([8, 8, 8, 8], 4, 123, 8, None),
+    ([8, 8, 8, 8], 4, 127, 7, None), ([8, 8, 8, 8], 1, 255, 32, None)])
+def test_token_major_width(retained, G, k, B, expect):
+    """Width = the smallest of 8, 16, 32 holding every KV head's retained dims; blocked
+    (None) past 32 dims, for G = 8, for k > 255, for k G < 500 or fewer than 128 query
+    heads."""
+    Hkv = 4
+    mask = np.ones((Hkv, 128), dtype=np.uint8)
+    for g, r in enumerate(retained):
+        mask[g, :r] = 0
+    p = fa.fa_plan_init(B, Hkv * G, Hkv, 1000, 32, 64, k, mask)
+    if expect is None:
+        assert p.e_token_major == 0
+    else:
+        assert p.e_token_major == 1 and all(p.de_ld[g] == expect for g in range(Hkv))
+        assert [p.de[g] for g in range(Hkv)] == retained
+
+
+def test_hand_edited_layout_is_rejected():
+    w = wl.llama3_8b_layer(8, 32768, 2)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    for field, value in (("e_token_major", 0), ("e_pitch", None), ("e_off", None)):
+        q = fa.fa_plan.from_buffer_copy(p)
+        if value is None:
+            getattr(q, field)[1] += 8
+        else:
+            setattr(q, field, value)
+        assert fa.LIB.fa_decode_workspace_size(ctypes.byref(q), 1) == 0, field
+        cache = fa.fa_cache(*([0x1000] * 6))
+        rc = fa.LIB.fa_compress(ctypes.byref(q), 0x1000, 0x1000, 0x1000, ctypes.byref(cache), None)
+        assert rc == fa.FA_ERR_INVALID and "layout" in fa.fa_last_error(), field

@@ -189,6 +189,58 @@ def test_ragged_mask_padding():
     run_small(w, mask=mask)
 
 
+# The plan puts E token-major and fa_decode runs the middle span on the tensor-core split
+# kernel when k <= 255, G in {1, 2, 4}, k G >= 500, at least 128 query heads and at most 32
+# exact dims per KV head; these cases cover its split counts, chunk layouts and head sets.
+TC_BASE = wl.shrink(wl.llama3_8b_layer(1, 8192, 0), B=16, Hq=8, Hkv=2, L=1400, k=127)
+TC_HEADS = [(0, 0), (0, 1), (7, 1), (15, 0), (15, 1)]
+
+
+def test_tensor_core_shapes_are_token_major():
+    masks = [wl.dim_mask(TC_BASE)] + [_ragged(dcs) for dcs, _ in TC_RAGGED]
+    shapes = [TC_BASE] + [_ragged_shape(k) for _, k in TC_RAGGED] + [TC_WIDE]
+    for w, m in zip(shapes, masks + [wl.dim_mask(TC_WIDE)]):
+        assert fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, m).e_token_major == 1
+
+
+@pytest.mark.parametrize("ns", [0, 1, 3, 7, 1000])
+def test_split_counts_tensor_core(ns):
+    run_small(TC_BASE, num_splits=ns, heads=TC_HEADS)
+
+
+TC_RAGGED = [([97, 100, 123, 127], 255),   # 31, 28, 5, 1 exact dims: 32-element rows
+             ([114, 120, 126, 124], 255),  # 14, 8, 2, 4: 16-element rows
+             ([120, 124, 128, 127], 255),  # 8, 4, 0, 1: 8-element rows
+             ([128, 96, 120, 112], 255)]   # 0, 32, 8, 16
+
+
+def _ragged_shape(k):
+    return wl.shrink(wl.LLAMA2_7B_MHA_32K, B=16, Hq=8, Hkv=4, L=1400, k=k)
+
+
+def _ragged(dcs):
+    rng = np.random.default_rng(5)
+    mask = np.zeros((4, D), dtype=np.uint8)
+    for g, dc in enumerate(dcs):
+        mask[g, rng.permutation(D)[:dc]] = 1
+    return mask
+
+
+@pytest.mark.parametrize("dcs,k", TC_RAGGED, ids=lambda x: str(x))
+def test_ragged_mask_tensor_core(dcs, k):
+    """Exact-dim rows of 1, 2 or 4 sixteen-byte chunks, KV heads with 0 to 32 exact dims."""
+    run_small(_ragged_shape(k), mask=_ragged(dcs),
+              heads=[(0, g) for g in range(4)] + [(15, g) for g in range(4)])
+
+
+TC_WIDE = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=40, Hq=8, Hkv=2, L=500, k=127, mask="rand96")
+
+
+def test_more_than_128_query_heads_tensor_core():
+    """Three head sets of 128 query heads; the last holds 64 valid heads."""
+    run_small(TC_WIDE, heads=[(0, 0), (15, 1), (16, 0), (31, 1), (32, 0), (39, 1)])
+
+
 def test_k_equals_M_matches_plain_attention():
     """With k = M nothing is lost: decode is plain attention over the original cache."""
     w = wl.shrink(wl.SINGLE_HEAD_2K, L=96 + 127, k=127)
