@@ -54,11 +54,18 @@ def parse():
 
 
 def workload_by_name(name):
+    """One of the named single-layer workloads, or one layer of the 32-layer LLaMA-3-8B
+    cache as llama3_8b_layer<layer>_b<B>_L<L>[_k<k>] (k is always L / 128 - 1)."""
+    import re
     import workloads as wl
     for w in wl.CONFIGS:
         if w.name == name:
             return w
-    raise SystemExit(f"unknown workload {name}; known: {[w.name for w in wl.CONFIGS]}")
+    m = re.fullmatch(r"llama3_8b_layer(\d+)_b(\d+)_L(\d+)(_k\d+)?", name)
+    if m:
+        return wl.llama3_8b_layer(int(m.group(2)), int(m.group(3)), int(m.group(1)))
+    raise SystemExit(f"unknown workload {name}; known: {[w.name for w in wl.CONFIGS]} or "
+                     "llama3_8b_layer<layer>_b<B>_L<L>")
 
 
 # ----------------------------------------------------------------------------- algorithmic work

@@ -463,80 +463,158 @@ __global__ void __launch_bounds__(DNT, SPT == 1 ? 2 : 1)
 }
 
 // ------------------------------------------------------------------------- combine
-__global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
-  extern __shared__ __align__(16) float cs[];
-  const int kvh = blockIdx.x, tid = threadIdx.x;
-  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
-  const int G = p.G, dc = p.dc[g], dc_ld = p.dc_ld[g], nrec = p.n_rec;
-  const int k_pad = (p.k + 3) & ~3;
-  float* wts = cs;                        // [G][nrec]
-  float* u = wts + G * nrec;              // [G][k_pad]
-  float* oacc = u + G * k_pad;            // [G][128]
-  float* lsum = oacc + G * FA_HEAD_DIM;   // [G] (padded to 8)
-  int* inv = reinterpret_cast<int*>(lsum + 8);  // [128]
-  const long long bhq = (long long)p.B * p.Hq;
+// One CTA per KV head (its G query heads share C_V), CB_THREADS threads = 8 warps.
+//  1. warp h: record weights w_r = 2^(m_r - m*) and the sum l of query head h;
+//  2. the weighted sum over split records of their payload (retained-dim values, then u
+//     slots), 128 columns at a time: warp w takes records w, w + 8, ... and reads each
+//     record's 128 columns as one float4 per lane, so many loads are in flight; the eight
+//     partial rows are then added in a fixed order (deterministic);
+//  3. out_c = u C_V with u_j = basis scale of function j x its slot sum, C_V staged
+//     through shared memory in CB_KC-row chunks;
+//  4. sink / recent records (all 128 dims in natural order) are added per dim, the dims
+//     scattered back, normalised and stored.
+constexpr int CB_THREADS = 256;
+constexpr int CB_KC = 64;
 
-  inv[p.perm[g][tid]] = tid;
-  for (int h = 0; h < G; ++h) {
-    const long long gh = (long long)b * p.Hq + g * G + h;
-    float mstar = -INFINITY;
-    for (int r = 0; r < nrec; ++r) mstar = fmaxf(mstar, p.rec[((long long)r * bhq + gh) * p.rec_stride]);
-    for (int r = tid; r < nrec; r += 128)
-      wts[h * nrec + r] = exp2f(p.rec[((long long)r * bhq + gh) * p.rec_stride] - mstar);
+// Float offsets of the combine's shared arrays; every one a multiple of 4 (16 bytes), so
+// the float4 accesses stay aligned.
+__host__ __device__ inline int combine_wts_floats(int G, int nrec) { return (G * nrec + 3) & ~3; }
+
+__host__ __device__ inline size_t combine_smem_floats(int G, int nrec, int payload) {
+  return (size_t)combine_wts_floats(G, nrec) + 16 + (size_t)G * payload + (size_t)8 * G * 128 +
+         (size_t)CB_KC * FA_HEAD_DIM + 2 * (size_t)G * FA_HEAD_DIM + FA_HEAD_DIM;
+}
+
+__global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  extern __shared__ __align__(16) float cs[];
+  const int kvh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
+  const int G = p.G, dc = p.dc[g], dc_ld = p.dc_ld[g], nrec = p.n_rec, ns = p.n_splits;
+  const int k = p.k;
+  const int payload = p.rec_stride - 4;     // retained-dim values (128) + u slots (2 F_pad)
+  float* wts = cs;                          // [G][nrec]
+  float* mst = wts + combine_wts_floats(G, nrec);  // [8]
+  float* lsum = mst + 8;                    // [8]
+  float* sum = lsum + 8;                    // [G][payload] weighted sum of split payloads
+  float* red = sum + G * payload;           // [8 warps][G][128] partial column sums
+  float* cvs = red + 8 * G * 128;           // [CB_KC][128] chunk of C_V
+  float* cpart = cvs + CB_KC * FA_HEAD_DIM; // [2][G][128] halves of u C_V
+  int* inv = reinterpret_cast<int*>(cpart + 2 * G * FA_HEAD_DIM);  // [128]
+  const long long bhq = (long long)p.B * p.Hq;
+  const long long gh0 = (long long)b * p.Hq + (long long)g * G;
+  auto rec = [&](int r, int h) -> const float* {
+    return p.rec + ((long long)r * bhq + gh0 + h) * p.rec_stride;
+  };
+
+  if (tid < FA_HEAD_DIM) inv[p.perm[g][tid]] = tid;
+  if (warp < G) {
+    const int h = warp;
+    float mx = -INFINITY;
+    for (int r = lane; r < nrec; r += 32) mx = fmaxf(mx, rec(r, h)[0]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float ls = 0.0f;
+    for (int r = lane; r < nrec; r += 32) {
+      const float* rr = rec(r, h);
+      const float w = exp2f(rr[0] - mx);
+      wts[h * nrec + r] = w;
+      ls += w * rr[1];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ls += __shfl_xor_sync(0xffffffffu, ls, o);
+    if (lane == 0) {
+      mst[h] = mx;
+      lsum[h] = ls;
+    }
   }
   __syncthreads();
-  for (int h = 0; h < G; ++h) {
-    const long long gh = (long long)b * p.Hq + g * G + h;
-    if (tid == 0) {
-      float l = 0.0f;
-      for (int r = 0; r < nrec; ++r) l += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 1];
-      lsum[h] = l;
-    }
-    const int d = tid;
-    const int i = inv[d];
-    float v = 0.0f;
-    if (i >= dc)
-      for (int r = 0; r < p.n_splits; ++r)
-        v += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + (i - dc)];
-    for (int r = p.n_splits; r < nrec; ++r)
-      v += wts[h * nrec + r] * p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + d];
-    oacc[h * FA_HEAD_DIM + d] = v;
-    for (int j = tid; j < p.k; j += 128) {
-      const int f = (j + 1) >> 1;
-      const int comp = (j > 0 && (j & 1) == 0) ? 1 : 0;
-      const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
-      float acc = 0.0f;
-      for (int r = 0; r < p.n_splits; ++r)
-        acc += wts[h * nrec + r] *
-               p.rec[((long long)r * bhq + gh) * p.rec_stride + 4 + FA_HEAD_DIM + 2 * f + comp];
-      u[h * k_pad + j] = acc * nrm;
-    }
-  }
-  __syncthreads();
-  if (tid < dc && p.n_splits > 0) {
-    const float* CV = p.CV + (long long)b * p.c_batch + p.c_off[g] + tid;
-    float acc[HL];
+  // weighted sum of the split records' payloads, 128 columns per pass
+  for (int c0 = 0; c0 < payload && ns > 0; c0 += 128) {
+    const int col = c0 + lane * 4;
+    float4 a[HL];
 #pragma unroll
-    for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
-    for (int j = 0; j < p.k; ++j) {
-      const float cv = CV[(long long)j * dc_ld];
+    for (int h = 0; h < HL; ++h) a[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (col < payload) {
+      for (int r = warp; r < ns; r += 8) {
 #pragma unroll
-      for (int h = 0; h < HL; ++h)
-        if (h < G) acc[h] += u[h * k_pad + j] * cv;
+        for (int h = 0; h < HL; ++h) {
+          if (h < G) {
+            const float w = wts[h * nrec + r];
+            const float4 v = *reinterpret_cast<const float4*>(rec(r, h) + 4 + col);
+            a[h].x += w * v.x;
+            a[h].y += w * v.y;
+            a[h].z += w * v.z;
+            a[h].w += w * v.w;
+          }
+        }
+      }
     }
-    const int d = p.perm[g][tid];
 #pragma unroll
     for (int h = 0; h < HL; ++h)
-      if (h < G) oacc[h * FA_HEAD_DIM + d] += acc[h];
+      if (h < G) reinterpret_cast<float4*>(red + (warp * G + h) * 128)[lane] = a[h];
+    __syncthreads();
+    for (int idx = tid; idx < G * 128; idx += CB_THREADS) {
+      const int h = idx >> 7, cc = idx & 127;
+      if (c0 + cc < payload) {
+        float v = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v += red[(w * G + h) * 128 + cc];
+        sum[h * payload + c0 + cc] = v;
+      }
+    }
+    __syncthreads();
+  }
+  // out_c = u C_V: C_V rows in chunks through shared memory; thread (half, column i) sums
+  // the rows of its parity
+  const float* CV = p.CV + (long long)b * p.c_batch + p.c_off[g];
+  const int colc = tid & (FA_HEAD_DIM - 1), half = tid >> 7;
+  float acc[HL];
+#pragma unroll
+  for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
+  for (int j0 = 0; j0 < k && dc > 0 && ns > 0; j0 += CB_KC) {
+    const int nj = min(CB_KC, k - j0);
+    __syncthreads();  // previous chunk consumed (first pass: sum written)
+    for (int e = tid; e < nj * (dc_ld / 4); e += CB_THREADS) {
+      const int jj = e / (dc_ld / 4), c4 = e - jj * (dc_ld / 4);
+      reinterpret_cast<float4*>(cvs + jj * FA_HEAD_DIM)[c4] =
+          reinterpret_cast<const float4*>(CV + (long long)(j0 + jj) * dc_ld)[c4];
+    }
+    __syncthreads();
+    if (colc < dc) {
+      for (int jj = half; jj < nj; jj += 2) {
+        const int j = j0 + jj, f = (j + 1) >> 1;
+        const int slot = FA_HEAD_DIM + 2 * f + ((j > 0 && (j & 1) == 0) ? 1 : 0);
+        const float cv = cvs[jj * FA_HEAD_DIM + colc] *
+                         ((f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair);
+#pragma unroll
+        for (int h = 0; h < HL; ++h)
+          if (h < G) acc[h] += sum[h * payload + slot] * cv;
+      }
+    }
   }
   __syncthreads();
-  for (int h = 0; h < G; ++h) {
-    const long long gh = (long long)b * p.Hq + g * G + h;
-    const float o = oacc[h * FA_HEAD_DIM + tid] / lsum[h];
+#pragma unroll
+  for (int h = 0; h < HL; ++h)
+    if (h < G) cpart[(half * G + h) * FA_HEAD_DIM + colc] = acc[h];
+  __syncthreads();
+  for (int idx = tid; idx < G * FA_HEAD_DIM; idx += CB_THREADS) {
+    const int h = idx / FA_HEAD_DIM, d = idx - h * FA_HEAD_DIM;
+    const int i = inv[d];
+    float o = 0.0f;
+    if (ns > 0) {
+      if (i >= dc)
+        o = sum[h * payload + (i - dc)];
+      else
+        o = cpart[h * FA_HEAD_DIM + i] + cpart[(G + h) * FA_HEAD_DIM + i];
+    }
+    const float* wh = wts + h * nrec;
+    for (int r = ns; r < nrec; ++r) o += wh[r] * rec(r, h)[4 + d];
+    o /= lsum[h];
+    const long long gh = gh0 + h;
     if (p.out_f32)
-      static_cast<float*>(p.out)[gh * FA_HEAD_DIM + tid] = o;
+      static_cast<float*>(p.out)[gh * FA_HEAD_DIM + d] = o;
     else
-      static_cast<__nv_bfloat16*>(p.out)[gh * FA_HEAD_DIM + tid] = __float2bfloat16_rn(o);
+      static_cast<__nv_bfloat16*>(p.out)[gh * FA_HEAD_DIM + d] = __float2bfloat16_rn(o);
   }
 }
 
@@ -629,6 +707,12 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
         }
       }
     }
+    // the combine keeps the G x n_rec record weights in shared memory: at most as many
+    // splits as fit (thousands; only an explicit request can reach the bound)
+    const long long nfs = (plan->S + plan->R + FT - 1) / FT;
+    const long long fixed = (long long)combine_smem_floats(plan->G, 0, FA_HEAD_DIM + 2 * c->F_pad) + 4;
+    const long long ns_max = ((227 * 1024) / 4 - fixed) / plan->G - nfs;
+    if (ns > ns_max) ns = (int)ns_max;
     const int per = (ntiles + ns - 1) / ns;
     c->n_splits = (ntiles + per - 1) / per;
     c->split_len = per * unit_tokens;
@@ -641,10 +725,8 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   const long long bhq = (long long)sh.B * sh.Hq;
   c->qw_bytes = (size_t)(bhq * c->qw_stride * 4);
   c->rec_bytes = (size_t)((long long)c->n_rec * bhq * c->rec_stride * 4);
-  const int k_pad = (sh.k + 3) & ~3;
-  c->smem_combine = (size_t)(plan->G * c->n_rec + plan->G * k_pad + plan->G * FA_HEAD_DIM + 8) * 4 +
-                    FA_HEAD_DIM * 4;
-  return cudaSuccess;
+  c->smem_combine = combine_smem_floats(plan->G, c->n_rec, c->rec_stride - 4) * 4;
+  return c->smem_combine <= 227 * 1024 ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
@@ -735,7 +817,7 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   }
   e = raise_smem_limit(reinterpret_cast<const void*>(decode_combine_kernel), (int)c.smem_combine);
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<n_heads, 128, c.smem_combine, stream>>>(p);
+  decode_combine_kernel<<<n_heads, CB_THREADS, c.smem_combine, stream>>>(p);
   return cudaGetLastError();
 }
 

@@ -177,7 +177,15 @@ __host__ __device__ constexpr size_t sink_recent_smem_bytes() {
 
 // Tensor-core split kernel over token-major E with de_slot = 0, 8, 16 or 32 retained
 // elements per KV head and token (the grid also holds the sink / recent CTAs).
+// bf16 x 8 -> 4 fp32 pairs (element 2i in .x, 2i + 1 in .y) for paired FMAs.
+__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream);
-size_t decode_tc_smem_bytes(int F2);
+size_t decode_tc_smem_bytes(int F2, int de_slot, int G);
 
 }  // namespace fa

@@ -24,8 +24,11 @@
 //
 // Exact dims: this kernel runs on token-major E (the plan lays E out so that token t of a
 // batch is one row holding every KV head's retained dims, w = 8, 16 or 32 per head). Per
-// token a head warp reads the w-element slices of its 32 / G KV heads as one coalesced row
-// segment, lane = (KV head, 16-byte chunk); the G query heads of a KV head share the load.
+// token a head warp needs the w-element slices of its 32 / G KV heads, lane = (KV head,
+// 16-byte chunk): coalesced row segments. Each lane streams its chunks, step after step
+// (K phase, V phase, next tile), into its own slots of a per-warp shared-memory ring with
+// 16-byte asynchronous copies, TC_RING steps ahead of use (one commit group per step), and
+// reads them back; the G query heads of a KV head share each chunk.
 // Dot products are reduced over a KV head's chunk lanes with shuffles and handed to the
 // head lanes through a per-warp [head][token] buffer, which then carries p back; the value
 // accumulator stays distributed (lane = KV head, chunk, query head) until the record is
@@ -51,27 +54,34 @@ constexpr float TC_P_SCALE = 128.0f;
 constexpr float TC_P_UNSCALE = 1.0f / 128.0f;
 
 constexpr int TC_XS_LD = 33;    // row pitch (floats) of the per-warp [head][token] buffer
+constexpr int TC_RING_BYTES = 8192;  // exact-dim ring per head warp
 
 struct TcLayout {
-  int w, phi, p, xs, misc, total;  // byte offsets from the 1024-aligned base
+  int w, phi, p, xs, ring, misc, total;  // byte offsets from the 1024-aligned base
 };
 
 // W: hi then lo, each [F2/64 atoms][128 heads][64 fp16] (K-major, 128-byte swizzle)
 // Phi: 2 buffers of [F2/64 atoms][32 tokens][64 fp16] (128-byte swizzle)
 // P: 2 buffers of [128 heads][32 fp16] (K-major, 64-byte swizzle)
 // xs: per head warp [32 heads][TC_XS_LD] fp32: exact-dim scores, then p, of the tile
+// ring: per head warp TC_RING_BYTES: TC_RING steps of 512 NI bytes (one 16-byte chunk per
+//   lane and load)
+// misc: pipeline mbarriers, TMEM slot, abort flag
 __host__ __device__ inline TcLayout tc_layout(int F2) {
   TcLayout L;
   L.w = 0;
   L.phi = L.w + 2 * TC_NH * F2 * 2;
   L.p = L.phi + 2 * TC_T * F2 * 2;
   L.xs = L.p + 2 * TC_NH * TC_T * 2;
-  L.misc = L.xs + 4 * 32 * TC_XS_LD * 4;
+  L.ring = L.xs + 4 * 32 * TC_XS_LD * 4;
+  L.misc = L.ring + 4 * TC_RING_BYTES;
   L.total = L.misc + 256 + 1024;  // + alignment slack
   return L;
 }
 
-size_t decode_tc_smem_bytes(int F2) {
+size_t decode_tc_smem_bytes(int F2, int de_slot, int G) {
+  (void)de_slot;
+  (void)G;
   const size_t b = (size_t)tc_layout(F2).total;
   return b > sink_recent_smem_bytes() ? b : sink_recent_smem_bytes();
 }
@@ -92,8 +102,8 @@ struct EMap {
   static constexpr int TT = CH >= 32 ? 1 : 32 / CH;                  // tokens per step
   static constexpr int NI = CH >= 32 ? CH / 32 : 1;                  // loads per lane per step
   static constexpr int NS = TC_T / TT;                               // steps per tile
-  static constexpr int U = 8 / NI;                                   // steps per load batch
   static constexpr int CPS1 = CPS > 0 ? CPS : 1;
+  static constexpr int RING = TC_RING_BYTES / (512 * NI);           // steps in flight
 };
 
 template <int CPS, int G>
@@ -308,8 +318,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int kap[NI], c8r[NI], de_r[NI];
     bool ev[NI];
     long long eoff[NI];
-    uint32_t qv[NI][G][4];  // q_e as bf16 pairs (exact: the query is bf16), unscaled
-    float accv[NI][G][8];
+    float2 qv[NI][G][4];    // q_e (scaled by sigma log2 e) of the lane's chunk, in pairs
+    float2 accv[NI][G][4];  // value accumulator of the lane's chunk, in pairs
 #pragma unroll
     for (int r = 0; r < NI; ++r) {
       const int q = (32 * r + lane) % EM::CH;
@@ -324,37 +334,57 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       eoff[r] = (long long)bb * p.e_batch + p.e_off[gg] + c_ * 8;
       de_r[r] = ev[r] ? p.de[gg] - c_ * 8 : 0;  // valid dims of this chunk (may be <= 0)
 #pragma unroll
-      for (int hq = 0; hq < G; ++hq) {
+      for (int hq = 0; hq < G; ++hq)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          uint32_t pr = 0;
-          for (int u = 0; u < 2; ++u) {
-            const int d = c_ * 8 + 2 * e + u;  // retained-dim index
-            if (ev[r] && d < p.de[gg]) {
-              const int dim = p.perm[gg][p.dc[gg] + d];
-              pr |= (uint32_t)__bfloat16_as_ushort(p.q[(gh0 + hq) * FA_HEAD_DIM + dim]) << (16 * u);
-            }
-          }
-          qv[r][hq][e] = pr;
+          const float* qe = p.qw + (gh0 + hq) * p.qw_stride + c_ * 8 + 2 * e;  // zero past de
+          qv[r][hq][e] = ev[r] ? make_float2(qe[0], qe[1]) : make_float2(0.0f, 0.0f);
+          accv[r][hq][e] = make_float2(0.0f, 0.0f);
         }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) accv[r][hq][e] = 0.0f;
-      }
     }
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
     float* xs = reinterpret_cast<float*>(smem + Ly.xs) + (warp - 1) * 32 * TC_XS_LD;
     const int c_first = ((lane % EM::CH) % EM::CPS1) == 0;  // first chunk lane of its KV head
 
-    // chunks of step s (tokens s * TT + tau_l of the tile) of tensor E
-    auto load_step = [&](const __nv_bfloat16* E, int t0, int nt, int s, uint4 (&x)[NI]) {
+    // exact-dim ring: global step gs = (tile, phase K / V, step) uses slot gs % RING; lane
+    // l's chunk of load r sits at byte (32 r + l) * 16 of the slot
+    constexpr int RING = EM::RING;
+    constexpr int STEP = 512 * NI;
+    uint8_t* ring = smem + Ly.ring + (warp - 1) * TC_RING_BYTES;
+    const int nkv = nvalid / G;
+    // this lane's chunks of global step gs, then one commit group (empty past the end)
+    auto issue = [&](int gs) {
+      const int ti = gs / (2 * EM::NS);
+      if (CPS > 0 && ti < ntiles) {
+        const int ph = (gs / EM::NS) & 1;
+        const int st = gs % EM::NS;
+        const int t0 = lo + ti * TC_T;
+        const int tok = st * EM::TT + tau_l;
+        if (tok < min(TC_T, hi - t0)) {
+          const __nv_bfloat16* E = ph ? p.EV : p.EK;
+          const unsigned trow = (unsigned)(t0 + tok) * (unsigned)p.e_row;  // < M e_row < 2^32
+#pragma unroll
+          for (int r = 0; r < NI; ++r)
+            if (ev[r]) cp_async16(ring + (gs % RING) * STEP + (32 * r + lane) * 16, E + eoff[r] + trow);
+        }
+      }
+      cp_async_commit();
+    };
+    // chunks of global step gs (tile-relative token s * TT + tau_l) once this lane's copies
+    // landed; every later step's group may still be in flight
+    auto take = [&](int gs, int s, int nt, uint4 (&x)[NI]) {
+      cp_async_wait<RING - 1>();
       const int tok = s * EM::TT + tau_l;
-      const long long trow = (long long)(t0 + tok) * p.e_row;
 #pragma unroll
       for (int r = 0; r < NI; ++r)
-        x[r] = (ev[r] && tok < nt) ? __ldg(reinterpret_cast<const uint4*>(E + eoff[r] + trow))
-                                   : make_uint4(0, 0, 0, 0);
+        x[r] = (ev[r] && tok < nt)
+                   ? *reinterpret_cast<const uint4*>(ring + (gs % RING) * STEP + (32 * r + lane) * 16)
+                   : make_uint4(0, 0, 0, 0);
     };
+    if constexpr (CPS > 0)
+      if (nkv > 0)
+        for (int gs = 0; gs < RING; ++gs) issue(gs);
 
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
@@ -373,27 +403,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         // exact-dim scores: per step, dot products of the lane's chunks with q_e, summed
         // over the KV head's CPS chunk lanes, into xs[query head][token]
-#pragma unroll 1
-        for (int s0 = 0; s0 < EM::NS; s0 += EM::U) {
-          uint4 x[EM::U][NI];
-#pragma unroll
-          for (int u = 0; u < EM::U; ++u) load_step(p.EK, t0, nt, s0 + u, x[u]);
-#pragma unroll
-          for (int u = 0; u < EM::U; ++u) {
+        if (nkv > 0) {
+#pragma unroll 2
+          for (int s1 = 0; s1 < EM::NS; ++s1) {
+            uint4 x[NI];
+            const int gs = i * 2 * EM::NS + s1;
+            take(gs, s1, nt, x);
             float part[NI][G];
 #pragma unroll
             for (int r = 0; r < NI; ++r) {
-              float xf[8];
-              bf16x8_to_f32(x[u][r], xf);
+              float2 x2[4];
+              bf16x8_to_f32x2(x[r], x2);
 #pragma unroll
               for (int hq = 0; hq < G; ++hq) {
-                float a = 0.0f;
+                float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  a += __uint_as_float(qv[r][hq][e] << 16) * xf[2 * e];
-                  a += __uint_as_float(qv[r][hq][e] & 0xFFFF0000u) * xf[2 * e + 1];
-                }
-                part[r][hq] = a;
+                for (int e = 0; e < 4; ++e) a = __ffma2_rn(qv[r][hq][e], x2[e], a);
+                part[r][hq] = a.x + a.y;
               }
             }
 #pragma unroll
@@ -404,14 +430,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 for (int hq = 0; hq < G; ++hq)
                   part[r][hq] += __shfl_xor_sync(0xffffffffu, part[r][hq], o);
             if (c_first) {
-              const int tok = (s0 + u) * EM::TT + tau_l;
+              const int tok = s1 * EM::TT + tau_l;
 #pragma unroll
               for (int r = 0; r < NI; ++r)
 #pragma unroll
                 for (int hq = 0; hq < G; ++hq)
-                  xs[(kap[r] * G + hq) * TC_XS_LD + tok] = part[r][hq] * p.qscale;
+                  xs[(kap[r] * G + hq) * TC_XS_LD + tok] = part[r][hq];
             }
+            issue(gs + RING);  // into the slot just read (its values are consumed above)
           }
+        } else {
+          for (int t = lane; t < 32 * TC_XS_LD; t += 32) xs[t] = 0.0f;
         }
         __syncwarp();
       }
@@ -469,7 +498,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           for (int hq = 0; hq < G; ++hq) {
             const float ah = __shfl_sync(0xffffffffu, a, kap[r] * G + hq);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) accv[r][hq][e] *= ah;
+            for (int e = 0; e < 4; ++e) accv[r][hq][e] = __fmul2_rn(accv[r][hq][e], make_float2(ah, ah));
           }
       }
       // P^T row of this head (fp16, 2^7 p) into buffer b, once MMA 2 of tile i-2 released it
@@ -499,30 +528,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         for (int t = 0; t < TC_T; ++t) xs[lane * TC_XS_LD + t] = sc[t];
         __syncwarp();
         // exact-dim values: accv[r][hq] += p(head kap G + hq, token) E_V chunk
-#pragma unroll 1
-        for (int s0 = 0; s0 < EM::NS; s0 += EM::U) {
-          uint4 x[EM::U][NI];
-#pragma unroll
-          for (int u = 0; u < EM::U; ++u) load_step(p.EV, t0, nt, s0 + u, x[u]);
-#pragma unroll
-          for (int u = 0; u < EM::U; ++u) {
-            const int tok = (s0 + u) * EM::TT + tau_l;
+        if (nkv > 0) {
+#pragma unroll 2
+          for (int s1 = 0; s1 < EM::NS; ++s1) {
+            uint4 x[NI];
+            const int gs = i * 2 * EM::NS + EM::NS + s1;
+            take(gs, s1, nt, x);
+            const int tok = s1 * EM::TT + tau_l;
 #pragma unroll
             for (int r = 0; r < NI; ++r) {
-              float xf[8];
-              bf16x8_to_f32(x[u][r], xf);
+              float2 x2[4];
+              bf16x8_to_f32x2(x[r], x2);
 #pragma unroll
               for (int hq = 0; hq < G; ++hq) {
                 const float pv = xs[(kap[r] * G + hq) * TC_XS_LD + tok];
+                const float2 pv2 = make_float2(pv, pv);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) accv[r][hq][e] += pv * xf[e];
+                for (int e = 0; e < 4; ++e) accv[r][hq][e] = __ffma2_rn(pv2, x2[e], accv[r][hq][e]);
               }
             }
+            issue(gs + RING);
           }
         }
         __syncwarp();  // xs is rewritten by the next tile's scores
       }
     }
+    cp_async_wait<0>();  // no copy of this thread is left in flight
     // split record: running max, sum, exact-dim values, U
     const bool done = ntiles == 0 || mbar_wait(u_done, 0, abort_flag, WD_DECODE | 8u);
     const bool all_ok = __all_sync(0xffffffffu, ok && done);
@@ -541,8 +572,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
           for (int hq = 0; hq < G; ++hq)
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              accv[r][hq][e] += __shfl_xor_sync(0xffffffffu, accv[r][hq][e], o);
+            for (int e = 0; e < 4; ++e) {
+              accv[r][hq][e].x += __shfl_xor_sync(0xffffffffu, accv[r][hq][e].x, o);
+              accv[r][hq][e].y += __shfl_xor_sync(0xffffffffu, accv[r][hq][e].y, o);
+            }
       if (tau_l == 0 && all_ok) {
 #pragma unroll
         for (int r = 0; r < NI; ++r) {
@@ -552,7 +585,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             float* rec = p.rec + ((long long)sp * bhq + gbase + kap[r] * G + hq) * p.rec_stride;
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-              if (e < de_r[r]) rec[4 + c8r[r] + e] = accv[r][hq][e];
+              if (e < de_r[r]) rec[4 + c8r[r] + e] = (e & 1) ? accv[r][hq][e >> 1].y : accv[r][hq][e >> 1].x;
           }
         }
       }
@@ -606,7 +639,7 @@ static cudaError_t launch_tc_g(const DecodeParams& p, int grid, int smem, cudaSt
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream) {
-  const int smem = (int)decode_tc_smem_bytes(p.tc_F2);
+  const int smem = (int)decode_tc_smem_bytes(p.tc_F2, de_slot, p.G);
   const int heads = p.B * p.Hq;
   const int grid = p.B * p.Hkv * p.n_fsplits + ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
   switch (de_slot) {
