@@ -104,6 +104,10 @@ struct EMap {
   static constexpr int NS = TC_T / TT;                               // steps per tile
   static constexpr int CPS1 = CPS > 0 ? CPS : 1;
   static constexpr int RING = TC_RING_BYTES / (512 * NI);           // steps in flight
+  // exact-dim scores on the warp-level bf16 MMA: one load per lane and step, 8 tokens per MMA
+  static constexpr bool KMMA = CPS > 0 && NI == 1 && RING >= 2 * (8 / TT);
+  static constexpr int SPG = 8 / TT;                                 // steps per 8 tokens
+  static constexpr int KS = CPS >= 2 ? CPS / 2 : 1;                  // 16-dim k-steps
 };
 
 template <int CPS, int G>
@@ -342,6 +346,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           accv[r][hq][e] = make_float2(0.0f, 0.0f);
         }
     }
+    // bf16 query rows for the MMA scores: A[row][k] = q (unscaled, exact in bf16) of query
+    // head `row` of KV head kv at retained dim k (rows >= G zero); this lane holds row
+    // lane / 4, dims 2 (lane % 4) + {0, 1} and + {8, 9} of each 16-dim k-step
+    uint32_t aq[EM::KMMA ? EM::NK : 1][EM::KS][2];
+    if constexpr (EM::KMMA) {
+      const int ar = lane >> 2, ac = (lane & 3) * 2;
+#pragma unroll
+      for (int kv = 0; kv < EM::NK; ++kv) {
+        const long long gh0 = gbase + (long long)kv * G;
+        const bool av = kv * G < nvalid && ar < G;
+        const int bb = av ? (int)(gh0 / p.Hq) : 0;
+        const int gg = av ? (int)(gh0 - (long long)bb * p.Hq) / G : 0;
+#pragma unroll
+        for (int ks = 0; ks < EM::KS; ++ks)
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pr = 0;
+#pragma unroll
+            for (int u2 = 0; u2 < 2; ++u2) {
+              const int d = ks * 16 + hh * 8 + ac + u2;  // retained-dim index
+              if (av && d < p.de[gg])
+                pr |= (uint32_t)__bfloat16_as_ushort(
+                          p.q[(gh0 + ar) * FA_HEAD_DIM + p.perm[gg][p.dc[gg] + d]])
+                      << (16 * u2);
+            }
+            aq[kv][ks][hh] = pr;
+          }
+      }
+    }
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
     float* xs = reinterpret_cast<float*>(smem + Ly.xs) + (warp - 1) * 32 * TC_XS_LD;
@@ -382,9 +415,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                    ? *reinterpret_cast<const uint4*>(ring + (gs % RING) * STEP + (32 * r + lane) * 16)
                    : make_uint4(0, 0, 0, 0);
     };
-    if constexpr (CPS > 0)
+    if constexpr (CPS > 0) {
+      // rows that are never copied (tokens past the split) are read by the MMA path: they
+      // must hold finite values
+      for (int o = lane * 16; o < TC_RING_BYTES; o += 32 * 16)
+        *reinterpret_cast<uint4*>(ring + o) = make_uint4(0, 0, 0, 0);
+      __syncwarp();
       if (nkv > 0)
         for (int gs = 0; gs < RING; ++gs) issue(gs);
+    }
 
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
@@ -401,9 +440,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             prefetch_l2_bulk(p.EV + o, (uint32_t)(nb * p.e_row * 2));
           }
         }
-        // exact-dim scores: per step, dot products of the lane's chunks with q_e, summed
-        // over the KV head's CPS chunk lanes, into xs[query head][token]
-        if (nkv > 0) {
+        if (EM::KMMA && nkv > 0) {
+          // exact-dim scores on the warp-level MMA: per 8 tokens and KV head, B = the 8
+          // token rows of the KV head's slice (ldmatrix from the ring), A = its query rows
+          const int gs0 = i * 2 * EM::NS;
+#pragma unroll 1
+          for (int tg = 0; tg < TC_T / 8; ++tg) {
+            cp_async_wait<RING - EM::SPG>();  // this lane's copies of the 8 tokens landed
+            __syncwarp();                     // and every other lane's
+            const int tok = tg * 8 + (lane & 7);  // ldmatrix row supplied by this lane
+            const int st = tok / EM::TT, tt = tok - (tok / EM::TT) * EM::TT;
+            const uint8_t* rowp =
+                ring + ((gs0 + st) % RING) * STEP + tt * EM::CH * 16 + (lane >> 3) * 16;
+#pragma unroll
+            for (int kv = 0; kv < (EM::KMMA ? EM::NK : 1); ++kv) {
+              if (kv < nkv) {
+                uint32_t bq[4];
+                if constexpr (CPS >= 4)
+                  ldmatrix_x4(bq, rowp + kv * (EM::CPS1 * 16));
+                else if constexpr (CPS == 2)
+                  ldmatrix_x2(bq, rowp + kv * (EM::CPS1 * 16));
+                else
+                  ldmatrix_x1(bq, rowp + kv * (EM::CPS1 * 16));
+                float dq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                mma_bf16_16816_rows8(dq, aq[kv][0][0], aq[kv][0][1], bq[0], bq[1]);
+                if constexpr (EM::KS == 2)
+                  mma_bf16_16816_rows8(dq, aq[kv][EM::KS - 1][0], aq[kv][EM::KS - 1][1], bq[2], bq[3]);
+                if ((lane >> 2) < G) {
+                  float* xr = xs + (kv * G + (lane >> 2)) * TC_XS_LD + tg * 8 + 2 * (lane & 3);
+                  xr[0] = dq[0] * p.qscale;
+                  xr[1] = dq[1] * p.qscale;
+                }
+              }
+            }
+            __syncwarp();  // every lane has read the slots of these 8 tokens
+#pragma unroll
+            for (int u2 = 0; u2 < EM::SPG; ++u2) issue(gs0 + tg * EM::SPG + u2 + RING);
+          }
+        } else if (nkv > 0) {
+          // exact-dim scores: per step, dot products of the lane's chunks with q_e, summed
+          // over the KV head's CPS chunk lanes, into xs[query head][token]
 #pragma unroll 2
           for (int s1 = 0; s1 < EM::NS; ++s1) {
             uint4 x[NI];

@@ -233,6 +233,19 @@ def test_ragged_mask_tensor_core(dcs, k):
               heads=[(0, g) for g in range(4)] + [(15, g) for g in range(4)])
 
 
+@pytest.mark.parametrize("retained", [[14, 9], [5, 3], [16, 0]], ids=str)
+def test_narrow_rows_gqa4_tensor_core(retained):
+    """G = 4 with 16- and 8-element KV slices: two or four tokens per exact-dim step."""
+    w = wl.shrink(wl.llama3_8b_layer(1, 8192, 0), B=16, Hq=8, Hkv=2, L=1400, k=127)
+    mask = np.ones((2, D), dtype=np.uint8)
+    rng = np.random.default_rng(9)
+    for g, r in enumerate(retained):
+        mask[g, rng.permutation(D)[:r]] = 0
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    assert p.e_token_major == 1 and p.de_ld[0] == (16 if max(retained) > 8 else 8)
+    run_small(w, mask=mask, heads=[(0, 0), (0, 1), (15, 0), (15, 1)])
+
+
 TC_WIDE = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=40, Hq=8, Hkv=2, L=500, k=127, mask="rand96")
 
 
