@@ -40,16 +40,16 @@ int check_ptr(const void* p, const char* name, bool required) {
 // Fills the layout fields of a plan (everything below the dim split) from shape, S, R, M,
 // kk, G, dc and de. E is token-major exactly when the tensor-core decode is used: it can
 // run when k <= 255, G is 1, 2 or 4 and every KV head keeps at most 32 dims, and it is
-// chosen when the k-length work per token and KV head (k G) is at least 500 and there are
-// at least 128 query heads (one full tensor-core head set); below that the CUDA-core
-// decode, whose time is then mostly the exact-dim rows, is the faster of the two.
+// chosen when the k-length work per token and KV head (k G) is at least 255 and there are
+// at least 128 query heads (one full tensor-core head set); below that (k = 63 with
+// G = 4, or small batches) the CUDA-core decode measured faster.
 void derive_layout(fa_plan* plan) {
   const fa_shape& s = plan->shape;
   int max_de = 0;
   for (int g = 0; g < s.Hkv; ++g) max_de = plan->de[g] > max_de ? plan->de[g] : max_de;
   const int G = plan->G;
   const bool tm = plan->M > 0 && s.k <= 255 && (G == 1 || G == 2 || G == 4) && max_de <= 32 &&
-                  s.k * G >= 500 && (long long)s.B * s.Hq >= 128;
+                  s.k * G >= 255 && (long long)s.B * s.Hq >= 128;
   const int w = max_de == 0 ? 0 : (max_de <= 8 ? 8 : (max_de <= 16 ? 16 : 32));
   plan->e_token_major = tm ? 1 : 0;
   long long ce = 0, ee = 0;

@@ -65,6 +65,12 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   float* mh = mxs + 8 * HL;             // [HL]
   float* red = mh + HL;                 // [DNT][8]
 
+  const __nv_bfloat16* FKh = p.FK + (long long)kvh * p.nF * FA_HEAD_DIM;
+  const __nv_bfloat16* FVh = p.FV + (long long)kvh * p.nF * FA_HEAD_DIM;
+  if (tid == 0) {  // this CTA's rows of both tensors into L2 while q is staged
+    prefetch_l2_bulk(FKh + (long long)r0 * FA_HEAD_DIM, (uint32_t)(nr * FA_HEAD_DIM * 2));
+    prefetch_l2_bulk(FVh + (long long)r0 * FA_HEAD_DIM, (uint32_t)(nr * FA_HEAD_DIM * 2));
+  }
   for (int idx = tid; idx < HL * FA_HEAD_DIM; idx += DNT) {
     const int h = idx >> 7, d = idx & 127;
     qs[idx] = (h < G) ? __bfloat162float(p.q[((long long)b * p.Hq + g * G + h) * FA_HEAD_DIM + d]) *
@@ -72,8 +78,6 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
                       : 0.0f;
   }
   __syncthreads();
-  const __nv_bfloat16* FKh = p.FK + (long long)kvh * p.nF * FA_HEAD_DIM;
-  const __nv_bfloat16* FVh = p.FV + (long long)kvh * p.nF * FA_HEAD_DIM;
   float s[HL];
 #pragma unroll
   for (int h = 0; h < HL; ++h) s[h] = 0.0f;
@@ -132,6 +136,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+#pragma unroll 8  // independent row loads in flight
   for (int rr = grp; rr < nr; rr += ngrp) {
     const float pv = sc[rr * HL + h];
     float x[8];

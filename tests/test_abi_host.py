@@ -187,8 +187,8 @@ def test_gpu_test_shapes_have_valid_plans():
 # ----------------------------------------------------------------------------- E layout
 
 @pytest.mark.parametrize("w,token_major", [
-    (wl.SINGLE_HEAD_2K, False),                   # k = 63, G = 4: k G < 500
-    (wl.LLAMA2_7B_MHA_32K, False),                # k = 255, G = 1: k G < 500
+    (wl.SINGLE_HEAD_2K, False),                   # k = 63, G = 4: k G < 255
+    (wl.LLAMA2_7B_MHA_32K, True),                 # k = 255, G = 1, 256 query heads
     (wl.LLAMA3_8B_GQA_32K, False),                # k = 511
     (wl.LLAMA3_8B_GQA_128K, False),               # k = 1023
     (wl.llama3_8b_layer(8, 8192, 2), False),      # k = 63
@@ -219,11 +219,12 @@ def test_token_major_choice(w, token_major):
     ([5, 1, 3, 8], 4, 127, 8, 8), ([12, 9, 16, 0], 4, 255, 8, 16),
     ([31, 17, 2, 20], 2, 255, 16, 32), ([0, 0, 0, 0], 4, 127, 8, 0),
     ([33, 1, 1, 1], 4, 255, 8, None), ([8, 8, 8, 8], 8, 63, 8, None),
-    ([8, 8, 8, 8], 4, 257, 8, None), ([8, 8, 8, 8], 4, 123, 8, None),
-    ([8, 8, 8, 8], 4, 127, 7, None), ([8, 8, 8, 8], 1, 255, 32, None)])
+    ([8, 8, 8, 8], 4, 257, 8, None), ([8, 8, 8, 8], 4, 63, 8, None),
+    ([8, 8, 8, 8], 4, 127, 7, None), ([8, 8, 8, 8], 1, 255, 32, 8),
+    ([8, 8, 8, 8], 2, 127, 16, None)])
 def test_token_major_width(retained, G, k, B, expect):
     """Width = the smallest of 8, 16, 32 holding every KV head's retained dims; blocked
-    (None) past 32 dims, for G = 8, for k > 255, for k G < 500 or fewer than 128 query
+    (None) past 32 dims, for G = 8, for k > 255, for k G < 255 or fewer than 128 query
     heads."""
     Hkv = 4
     mask = np.ones((Hkv, 128), dtype=np.uint8)

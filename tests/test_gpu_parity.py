@@ -190,7 +190,7 @@ def test_ragged_mask_padding():
 
 
 # The plan puts E token-major and fa_decode runs the middle span on the tensor-core split
-# kernel when k <= 255, G in {1, 2, 4}, k G >= 500, at least 128 query heads and at most 32
+# kernel when k <= 255, G in {1, 2, 4}, k G >= 255, at least 128 query heads and at most 32
 # exact dims per KV head; these cases cover its split counts, chunk layouts and head sets.
 TC_BASE = wl.shrink(wl.llama3_8b_layer(1, 8192, 0), B=16, Hq=8, Hkv=2, L=1400, k=127)
 TC_HEADS = [(0, 0), (0, 1), (7, 1), (15, 0), (15, 1)]
@@ -244,6 +244,15 @@ def test_narrow_rows_gqa4_tensor_core(retained):
     p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
     assert p.e_token_major == 1 and p.de_ld[0] == (16 if max(retained) > 8 else 8)
     run_small(w, mask=mask, heads=[(0, 0), (0, 1), (15, 0), (15, 1)])
+
+
+@pytest.mark.parametrize("dcs", [[97, 123, 127, 108], [120, 124, 128, 127]], ids=str)
+def test_mha_tensor_core(dcs):
+    """G = 1 (each KV head its own query head) at k = 255: 32- and 8-element KV slices."""
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=32, Hq=4, Hkv=4, L=1400, k=255)
+    mask = _ragged(dcs)
+    assert fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask).e_token_major == 1
+    run_small(w, mask=mask, heads=[(0, g) for g in range(4)] + [(31, g) for g in range(4)])
 
 
 TC_WIDE = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=40, Hq=8, Hkv=2, L=500, k=127, mask="rand96")
