@@ -430,16 +430,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const int t0 = lo + i * TC_T;
       const int nt = min(TC_T, hi - t0);
       if constexpr (CPS > 0) {
-        if (i + 1 < ntiles && nvalid > 0) {  // next tile's rows of this warp's batches -> L2
-          const int tn = t0 + TC_T;
-          const int nb = min(TC_T, hi - tn);
-          const int b0 = (int)(gbase / p.Hq), b1 = (int)((gbase + nvalid - 1) / p.Hq);
-          for (int bb = b0 + lane; bb <= b1; bb += 32) {
-            const long long o = (long long)bb * p.e_batch + (long long)tn * p.e_row;
-            prefetch_l2_bulk(p.EK + o, (uint32_t)(nb * p.e_row * 2));
-            prefetch_l2_bulk(p.EV + o, (uint32_t)(nb * p.e_row * 2));
-          }
-        }
+        // (no separate L2 prefetch: the ring's own copies run far enough ahead, and an
+        // extra bulk prefetch of the next tile measured slower)
         if (EM::KMMA && nkv > 0) {
           // exact-dim scores on the warp-level MMA: per 8 tokens and KV head, B = the 8
           // token rows of the KV head's slice (ldmatrix from the ring), A = its query rows
