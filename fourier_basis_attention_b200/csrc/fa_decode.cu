@@ -664,8 +664,8 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   // 32 retained dims per KV head).
   c->tc_F2 = ((2 * c->F + 63) / 64) * 64;
   c->tc = (M > 0 && plan->e_token_major) ? 1 : 0;
-  int cols = 32;
-  while (cols < c->tc_F2 + 64) cols <<= 1;
+  int cols = 32;  // U (2F slots), S (2 x 32 tokens), W_lo (2F / 2 columns of slot pairs)
+  while (cols < c->tc_F2 + 64 + c->tc_F2 / 2) cols <<= 1;
   c->tc_tmem_cols = cols;
   const int unit_tokens = c->tc ? 32 : DT;  // tokens per tile
   const int n_headsets = c->tc ? (sh.B * sh.Hq + 127) / 128 : (n_heads + c->NKV - 1) / c->NKV;

@@ -11,7 +11,7 @@
 // 2^7 p with p <= 2^8 (lazy max below), so it stays normal down to p = 2^-21 (U carries
 // the 2^7 until the record is written); W is scaled per head by a power of two to at most
 // 1 in magnitude and split into hi + lo (lo = W - hi), so S takes two MMAs
-// (W_hi . Phi^T + W_lo . Phi^T). The score error is then ~2^-22 relative and the value
+// (W_hi . Phi^T with W_hi in shared memory + W_lo . Phi^T with W_lo in tensor memory). The score error is then ~2^-22 relative and the value
 // error ~2^-12 per term, far inside the 3e-3 output bar (one plain fp16 or tf32 pass for S
 // would leave only a 5x margin). One buffer per tile holds Phi_t as [token][slot] with
 // 128-byte swizzle: MMA 1 reads it as its K-major B operand, MMA 2 as its MN-major B
@@ -54,13 +54,13 @@ constexpr float TC_P_SCALE = 128.0f;
 constexpr float TC_P_UNSCALE = 1.0f / 128.0f;
 
 constexpr int TC_XS_LD = 33;    // row pitch (floats) of the per-warp [head][token] buffer
-constexpr int TC_RING_BYTES = 8192;  // exact-dim ring per head warp
+constexpr int TC_RING_BYTES = 24576;  // exact-dim ring per head warp
 
 struct TcLayout {
   int w, phi, p, xs, ring, misc, total;  // byte offsets from the 1024-aligned base
 };
 
-// W: hi then lo, each [F2/64 atoms][128 heads][64 fp16] (K-major, 128-byte swizzle)
+// W_hi: [F2/64 atoms][128 heads][64 fp16] (K-major, 128-byte swizzle); W_lo lives in TMEM
 // Phi: 2 buffers of [F2/64 atoms][32 tokens][64 fp16] (128-byte swizzle)
 // P: 2 buffers of [128 heads][32 fp16] (K-major, 64-byte swizzle)
 // xs: per head warp [32 heads][TC_XS_LD] fp32: exact-dim scores, then p, of the tile
@@ -70,7 +70,7 @@ struct TcLayout {
 __host__ __device__ inline TcLayout tc_layout(int F2) {
   TcLayout L;
   L.w = 0;
-  L.phi = L.w + 2 * TC_NH * F2 * 2;
+  L.phi = L.w + TC_NH * F2 * 2;
   L.p = L.phi + 2 * TC_T * F2 * 2;
   L.xs = L.p + 2 * TC_NH * TC_T * 2;
   L.ring = L.xs + 4 * 32 * TC_XS_LD * 4;
@@ -124,10 +124,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int cta = blockIdx.x - n_f;
   const int F2 = p.tc_F2;
   const TcLayout Ly = tc_layout(F2);
-  uint8_t* Ws = smem + Ly.w;      // hi at Ws, lo at Ws + w_half
+  uint8_t* Ws = smem + Ly.w;      // W_hi
   uint8_t* PHI = smem + Ly.phi;   // buffer b at PHI + b * phi_bytes
   uint8_t* PS = smem + Ly.p;      // buffer b at PS + b * p_bytes
-  const int w_half = TC_NH * F2 * 2;
   const int phi_bytes = TC_T * F2 * 2;
   const int p_bytes = TC_NH * TC_T * 2;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.misc);
@@ -163,8 +162,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     tmem_alloc(tmem_slot, p.tc_tmem_cols);
     tmem_relinquish();
   }
-  // head warps: W rows, scaled by 2^-e to at most 1 in magnitude, split into fp16 hi / lo
-  // and written into the K-major swizzled operand; S is scaled back by 2^e on readout
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem_u = tmem;              // U^T: columns [0, F2)
+  const uint32_t tmem_s = tmem + F2;         // S^T buffer b: columns F2 + 32 b
+  const uint32_t tmem_wlo = tmem + F2 + 64;  // W_lo: columns [F2 + 64, F2 + 64 + F2 / 2)
+  // head warps: W rows, scaled by 2^-e to at most 1 in magnitude, split into fp16 hi (the
+  // K-major swizzled shared operand) and lo (TMEM row = this head's lane, two slots per
+  // column); S is scaled back by 2^e on readout
   const int h = (warp & 3) * 32 + lane;  // TMEM lane of a head thread
   const long long gh = (long long)hg * TC_NH + h;
   const bool is_head = warp >= 1 && warp <= 4;
@@ -179,30 +186,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if (wmax > 0.0f) frexpf(wmax, &ex);  // wmax < 2^ex
     const float w_scale = ldexpf(1.0f, -ex);
     w_unscale = ldexpf(1.0f, ex);
-    for (int c8 = 0; c8 < F2 / 8; ++c8) {
-      uint32_t hv[4], lv[4];
+    const uint32_t lanebase_w = (uint32_t)((warp & 3) * 32) << 16;
+    for (int c64 = 0; c64 < F2 / 64; ++c64) {  // 64 slots: one swizzle atom, 32 TMEM columns
+      uint32_t lo32[32];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int slot = c8 * 8 + 2 * e;
-        const float a = slot < nslot ? wsrc[slot] * w_scale : 0.0f;
-        const float b = slot + 1 < nslot ? wsrc[slot + 1] * w_scale : 0.0f;
-        hv[e] = pack_half2(a, b);
-        const __half2 hh = *reinterpret_cast<const __half2*>(&hv[e]);
-        lv[e] = pack_half2(a - __low2float(hh), b - __high2float(hh));
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t hv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int slot = c64 * 64 + c8 * 8 + 2 * e;
+          const float a = slot < nslot ? wsrc[slot] * w_scale : 0.0f;
+          const float b = slot + 1 < nslot ? wsrc[slot + 1] * w_scale : 0.0f;
+          hv[e] = pack_half2(a, b);
+          const __half2 hh = *reinterpret_cast<const __half2*>(&hv[e]);
+          lo32[c8 * 4 + e] = pack_half2(a - __low2float(hh), b - __high2float(hh));
+        }
+        const int off = c64 * (TC_NH * 128) + h * 128 + ((c8 ^ (h & 7)) << 4);
+        *reinterpret_cast<uint4*>(Ws + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
       }
-      const int atom = c8 >> 3, chunk = c8 & 7;
-      const int off = atom * (TC_NH * 128) + h * 128 + ((chunk ^ (h & 7)) << 4);
-      *reinterpret_cast<uint4*>(Ws + off) = make_uint4(hv[0], hv[1], hv[2], hv[3]);
-      *reinterpret_cast<uint4*>(Ws + w_half + off) = make_uint4(lv[0], lv[1], lv[2], lv[3]);
+      tmem_st_32x32b_x32(tmem_wlo + lanebase_w + c64 * 32, lo32);
     }
+    tmem_st_wait();
     fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_u = tmem;              // U^T: columns [0, F2)
-  const uint32_t tmem_s = tmem + F2;         // S^T buffer b: columns F2 + 32 b
 
   if (warp == 0) {
     // -------------------------------------------------------------------- MMA issuer
@@ -236,7 +245,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t ow = (uint32_t)(((ks >> 2) * (TC_NH * 128) + (ks & 3) * 32) >> 4);
           const uint32_t op = (uint32_t)(((ks >> 2) * (TC_T * 128) + (ks & 3) * 32) >> 4);
           mma_f16(ts, d_w + ow, dphi + op, idesc1, ks > 0 ? 1u : 0u);
-          mma_f16(ts, d_w + ow + (uint32_t)(w_half >> 4), dphi + op, idesc1, 1u);
+          mma_f16_ta(ts, tmem_wlo + 8 * ks, dphi + op, idesc1, 1u);  // 16 slots = 8 columns
         }
         mma_commit(&s_full[b]);
       };

@@ -326,6 +326,18 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t lbo_
   return smem_desc(saddr, lbo_bytes, sbo_bytes, 4u);
 }
 
+// D[tmem] (+)= A[tmem] * B[smem], kind::f16: A (M rows = TMEM lanes, K along the columns,
+// two 16-bit elements per 32-bit column) read from tensor memory.
+__device__ __forceinline__ void mma_f16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Instruction descriptor of kind::f16 with fp16 A/B, fp32 D, A K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, bool b_mn_major) {
   return (1u << 4)                          // D format f32 (A, B format fields 0 = f16)
