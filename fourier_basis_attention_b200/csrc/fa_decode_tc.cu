@@ -389,8 +389,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     float* xs = reinterpret_cast<float*>(smem + Ly.xs) + (warp - 1) * 32 * TC_XS_LD;
     const int c_first = ((lane % EM::CH) % EM::CPS1) == 0;  // first chunk lane of its KV head
 
-    // exact-dim ring: global step gs = (tile, phase K / V, step) uses slot gs % RING; lane
-    // l's chunk of load r sits at byte (32 r + l) * 16 of the slot
+    // exact-dim ring: global step gs = (tile, phase K / V, step) uses slot gs % RING; chunk c
+    // of a slot (lane l's load r: c = 32 r + l) sits at 16-byte position c ^ (token & 7),
+    // so the 8 token rows an ldmatrix reads from 8 slots fall in 8 different banks
     constexpr int RING = EM::RING;
     constexpr int STEP = 512 * NI;
     uint8_t* ring = smem + Ly.ring + (warp - 1) * TC_RING_BYTES;
@@ -408,7 +409,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const unsigned trow = (unsigned)(t0 + tok) * (unsigned)p.e_row;  // < M e_row < 2^32
 #pragma unroll
           for (int r = 0; r < NI; ++r)
-            if (ev[r]) cp_async16(ring + (gs % RING) * STEP + (32 * r + lane) * 16, E + eoff[r] + trow);
+            if (ev[r])
+              cp_async16(ring + (gs % RING) * STEP + (((32 * r + lane) ^ (tok & 7)) * 16),
+                         E + eoff[r] + trow);
         }
       }
       cp_async_commit();
@@ -421,7 +424,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
       for (int r = 0; r < NI; ++r)
         x[r] = (ev[r] && tok < nt)
-                   ? *reinterpret_cast<const uint4*>(ring + (gs % RING) * STEP + (32 * r + lane) * 16)
+                   ? *reinterpret_cast<const uint4*>(ring + (gs % RING) * STEP +
+                                                     (((32 * r + lane) ^ (tok & 7)) * 16))
                    : make_uint4(0, 0, 0, 0);
     };
     if constexpr (CPS > 0) {
@@ -451,18 +455,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             __syncwarp();                     // and every other lane's
             const int tok = tg * 8 + (lane & 7);  // ldmatrix row supplied by this lane
             const int st = tok / EM::TT, tt = tok - (tok / EM::TT) * EM::TT;
-            const uint8_t* rowp =
-                ring + ((gs0 + st) % RING) * STEP + tt * EM::CH * 16 + (lane >> 3) * 16;
+            const uint8_t* slotp = ring + ((gs0 + st) % RING) * STEP;
+            const int cbase = tt * EM::CH + (lane >> 3);  // chunk of matrix lane / 8 of KV 0
 #pragma unroll
             for (int kv = 0; kv < (EM::KMMA ? EM::NK : 1); ++kv) {
               if (kv < nkv) {
                 uint32_t bq[4];
+                const uint8_t* rowp = slotp + (((cbase + kv * EM::CPS1) ^ (lane & 7)) * 16);
                 if constexpr (CPS >= 4)
-                  ldmatrix_x4(bq, rowp + kv * (EM::CPS1 * 16));
+                  ldmatrix_x4(bq, rowp);
                 else if constexpr (CPS == 2)
-                  ldmatrix_x2(bq, rowp + kv * (EM::CPS1 * 16));
+                  ldmatrix_x2(bq, rowp);
                 else
-                  ldmatrix_x1(bq, rowp + kv * (EM::CPS1 * 16));
+                  ldmatrix_x1(bq, rowp);
                 float dq[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 mma_bf16_16816_rows8(dq, aq[kv][0][0], aq[kv][0][1], bq[0], bq[1]);
                 if constexpr (EM::KS == 2)
