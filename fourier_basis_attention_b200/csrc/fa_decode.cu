@@ -535,6 +535,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
 #pragma unroll
     for (int h = 0; h < HL; ++h) a[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (col < payload) {
+#pragma unroll 4  // several records' rows in flight per lane
       for (int r = warp; r < ns; r += 8) {
 #pragma unroll
         for (int h = 0; h < HL; ++h) {
