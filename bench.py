@@ -441,13 +441,16 @@ def run_ours(args):
 
 def launches_per_step(w, plan):
     """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel and
-    compress_kernel; then fa_decode's prologue (middle span present), one split kernel (the
-    tensor-core one when the plan laid E out token-major, else the CUDA-core one; either
-    also covers the sink / recent rows), and the combine."""
+    compress_kernel; then fa_decode's prologue (middle span present), the split kernel (the
+    tensor-core one when the plan laid E out token-major, followed by the CUDA-core kernel
+    for the sink / recent rows; else the CUDA-core one for both), and the combine."""
     n = 1 + 2
     n += 1 if plan.M > 0 else 0          # prologue
-    if plan.M > 0 or plan.S + plan.R > 0:
-        n += 1                           # split kernel
+    if plan.e_token_major and plan.M > 0:
+        n += 1                           # tensor-core split kernel
+        n += 1 if plan.S + plan.R > 0 else 0  # sink / recent rows (CUDA-core kernel)
+    elif plan.M > 0 or plan.S + plan.R > 0:
+        n += 1                           # CUDA-core split kernel (+ sink / recent rows)
     return n + 1                         # combine
 
 

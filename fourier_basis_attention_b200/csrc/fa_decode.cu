@@ -794,14 +794,20 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     decode_prologue_kernel<<<n_heads, DNT, plan->G * FA_HEAD_DIM * 4, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  // The sink / recent rows run either as extra CTAs of the tensor-core grid or, when
+  // kTcSinkRecentSeparate, in a CUDA-core launch of their own after it (small CTAs, two per
+  // SM, instead of holding a whole SM each).
+  constexpr bool kTcSinkRecentSeparate = true;
   if (c.tc) {
-    // middle span on the tensor cores, sink / recent rows as extra CTAs of the same grid
     p.e_row = plan->e_pitch[0];
+    p.tc_nf = kTcSinkRecentSeparate ? 0 : n_heads * c.n_fsplits;
     if ((e = launch_decode_tc(p, plan->de_ld[0], stream)) != cudaSuccess) return e;
+    p.n_mid = 0;
   } else if (plan->e_token_major && plan->M > 0) {
     return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only
   }
-  const int grid = c.tc ? 0 : p.n_mid + n_heads * c.n_fsplits;
+  const int grid = c.tc ? (kTcSinkRecentSeparate ? n_heads * c.n_fsplits : 0)
+                        : p.n_mid + n_heads * c.n_fsplits;
   if (grid > 0) {
     int occ = 0;
     if (c.SPT == 1) {

@@ -34,8 +34,8 @@
 // accumulator stays distributed (lane = KV head, chunk, query head) until the record is
 // written. Softmax, P rows, U rescaling and (m, l) are per head lane.
 //
-// CTAs [0, B Hkv n_fsplits) of the grid run the sink / recent rows on the CUDA cores
-// (decode_sink_recent), so one launch covers every split record.
+// CTAs [0, tc_nf) of the grid may run the sink / recent rows on the CUDA cores
+// (decode_sink_recent); otherwise the CUDA-core kernel runs them in a launch of its own.
 #include "fa_decode_common.cuh"
 
 namespace fa {
@@ -116,7 +116,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int n_f = p.B * p.Hkv * p.n_fsplits;  // sink / recent CTAs come first
+  const int n_f = p.tc_nf;  // sink / recent CTAs come first
   if ((int)blockIdx.x < n_f) {
     decode_sink_recent(p, reinterpret_cast<float*>(smem), blockIdx.x);
     return;
@@ -723,7 +723,7 @@ static cudaError_t launch_tc_g(const DecodeParams& p, int grid, int smem, cudaSt
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream) {
   const int smem = (int)decode_tc_smem_bytes(p.tc_F2, de_slot, p.G);
   const int heads = p.B * p.Hq;
-  const int grid = p.B * p.Hkv * p.n_fsplits + ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
+  const int grid = p.tc_nf + ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
   switch (de_slot) {
     case 0: return launch_tc_g<0>(p, grid, smem, stream);
     case 8: return launch_tc_g<1>(p, grid, smem, stream);
