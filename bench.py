@@ -442,12 +442,14 @@ def run_ours(args):
 def launches_per_step(w, plan):
     """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel and
     compress_kernel; then fa_decode's prologue (middle span present), the split kernel (the
-    tensor-core one when the plan laid E out token-major, followed by the CUDA-core kernel
-    for the sink / recent rows; else the CUDA-core one for both), and the combine."""
+    tensor-core one when the plan laid E out token-major, or the warp-MMA one for other
+    plans with 256 <= k <= 1023, each followed by the CUDA-core kernel for the sink / recent
+    rows; else the CUDA-core one for both), and the combine."""
     n = 1 + 2
     n += 1 if plan.M > 0 else 0          # prologue
-    if plan.e_token_major and plan.M > 0:
-        n += 1                           # tensor-core split kernel
+    hm = plan.M > 0 and not plan.e_token_major and 256 <= w.k <= 1023
+    if (plan.e_token_major or hm) and plan.M > 0:
+        n += 1                           # tensor-core or warp-MMA split kernel
         n += 1 if plan.S + plan.R > 0 else 0  # sink / recent rows (CUDA-core kernel)
     elif plan.M > 0 or plan.S + plan.R > 0:
         n += 1                           # CUDA-core split kernel (+ sink / recent rows)

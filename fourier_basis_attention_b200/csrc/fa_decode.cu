@@ -665,11 +665,16 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   // 32 retained dims per KV head).
   c->tc_F2 = ((2 * c->F + 63) / 64) * 64;
   c->tc = (M > 0 && plan->e_token_major) ? 1 : 0;
+  // The warp-MMA split kernel (16 query heads per CTA, U in registers) takes the other
+  // plans with 256 <= k <= 1023 (2F rounded up to 512 or 1024 slots).
+  c->hm_F2 = 2 * c->F <= 256 ? 256 : (2 * c->F <= 512 ? 512 : 1024);
+  c->hm = (!c->tc && M > 0 && sh.k >= 256 && c->hm_F2 <= 1024) ? 1 : 0;
   int cols = 32;  // U (2F slots), S (2 x 32 tokens), W_lo (2F / 2 columns of slot pairs)
   while (cols < c->tc_F2 + 64 + c->tc_F2 / 2) cols <<= 1;
   c->tc_tmem_cols = cols;
-  const int unit_tokens = c->tc ? 32 : DT;  // tokens per tile
-  const int n_headsets = c->tc ? (sh.B * sh.Hq + 127) / 128 : (n_heads + c->NKV - 1) / c->NKV;
+  const int unit_tokens = c->tc ? 32 : DT;  // tokens per tile (64 for the warp-MMA kernel)
+  const int n_headsets = c->tc ? (sh.B * sh.Hq + 127) / 128
+                               : (c->hm ? (sh.B * sh.Hq + 15) / 16 : (n_heads + c->NKV - 1) / c->NKV);
   const int ntiles = (M + unit_tokens - 1) / unit_tokens;
   if (M == 0) {
     c->n_splits = 0;
@@ -682,7 +687,7 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
       int sms = 148, occ = 1;
       cudaError_t e = device_sm_count(&sms);
       if (e != cudaSuccess) return e;
-      if (c->tc) {
+      if (c->tc || c->hm) {
         occ = 1;  // one CTA per SM (shared memory)
       } else {
         e = c->SPT == 1 ? occupancy<1>(&occ, c->smem_main)
@@ -805,6 +810,10 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     p.n_mid = 0;
   } else if (plan->e_token_major && plan->M > 0) {
     return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only
+  } else if (c.hm) {
+    // middle span on warp-level MMAs; the CUDA-core kernel below runs the sink / recent rows
+    if ((e = launch_decode_hmma(p, c.hm_F2, stream)) != cudaSuccess) return e;
+    p.n_mid = 0;
   }
   const int grid = c.tc ? (kTcSinkRecentSeparate ? n_heads * c.n_fsplits : 0)
                         : p.n_mid + n_heads * c.n_fsplits;

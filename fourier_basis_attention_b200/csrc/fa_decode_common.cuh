@@ -181,6 +181,10 @@ __host__ __device__ constexpr size_t sink_recent_smem_bytes() {
   return (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + DNT * 8) * 4;
 }
 
+// Warp-MMA split kernel over per-KV-head E blocks, F2 = 256, 512 or 1024 slots.
+cudaError_t launch_decode_hmma(const DecodeParams& p, int F2, cudaStream_t stream);
+size_t decode_hmma_smem_bytes(int F2);
+
 // Tensor-core split kernel over token-major E with de_slot = 0, 8, 16 or 32 retained
 // elements per KV head and token (the grid also holds the sink / recent CTAs).
 // bf16 x 8 -> 4 fp32 pairs (element 2i in .x, 2i + 1 in .y) for paired FMAs.

@@ -12,6 +12,7 @@ namespace fa {
 struct DecodeConfig {
   int n_splits, split_len, n_fsplits, n_rec, F, F_pad, SPT, NTU, TG, DEC, TGE, NKV;
   int tc, tc_F2, tc_tmem_cols, de_ld_max;  // tensor-core split kernel chosen, its slots / TMEM
+  int hm, hm_F2;  // warp-MMA split kernel chosen (blocked E, large k), its slots
   size_t qw_bytes, rec_bytes, smem_main, smem_combine;
   int rec_stride, qw_stride;
 };

@@ -255,6 +255,33 @@ def test_mha_tensor_core(dcs):
     run_small(w, mask=mask, heads=[(0, g) for g in range(4)] + [(31, g) for g in range(4)])
 
 
+# Plans that are not token-major with 256 <= k <= 1023 run the middle span on the warp-MMA
+# split kernel (16 query heads per CTA): group sizes, ragged exact dims, both slot counts.
+@pytest.mark.parametrize("G,Hkv,k,dcs", [(8, 2, 511, None), (1, 4, 511, [37, 1, 127, 90]),
+                                         (2, 4, 1023, [100, 64, 17, 128]), (4, 2, 300, [0, 96])],
+                         ids=["G8_k511", "G1_k511_ragged", "G2_k1023_ragged", "G4_k300_none_all"])
+def test_warp_mma_decode(G, Hkv, k, dcs):
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=3, Hq=Hkv * G, Hkv=Hkv, L=k + 96 + 333, k=k)
+    mask = wl.dim_mask(w) if dcs is None else _ragged_hkv(dcs, Hkv)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    assert p.e_token_major == 0
+    run_small(w, mask=mask)
+
+
+def _ragged_hkv(dcs, Hkv):
+    rng = np.random.default_rng(13)
+    mask = np.zeros((Hkv, D), dtype=np.uint8)
+    for g, dc in enumerate(dcs):
+        mask[g, rng.permutation(D)[:dc]] = 1
+    return mask
+
+
+@pytest.mark.parametrize("ns", [1, 5, 1000])
+def test_split_counts_warp_mma(ns):
+    run_small(wl.shrink(wl.LLAMA3_8B_GQA_128K, B=1, Hq=32, Hkv=8, L=3300), num_splits=ns,
+              heads=[(0, 0), (0, 7)])
+
+
 TC_WIDE = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=40, Hq=8, Hkv=2, L=500, k=127, mask="rand96")
 
 
