@@ -16,7 +16,9 @@
 //   D. online softmax per head with a lazily raised reference max (only when a tile exceeds
 //      it by more than 2^8), P = 2^7 p in fp16;
 //   E. U += P . Phi_t: warp w keeps U for its slots in registers (16 heads x F2 / 8 slots);
-//   F. exact-dim values acc += p E_V[t] on the CUDA cores.
+//   F. exact-dim values acc += p E_V[t] on the CUDA cores; when a tile's E_V rows of the
+//      CTA's KV heads fit in HM_EV_BYTES they are staged into shared memory with cp.async
+//      at the start of the tile, so their loads overlap phases A-E.
 // The split record (m, l, exact-dim values, U) has the layout of the other split kernels,
 // so the same combine merges it. Sink / recent rows run in the CUDA-core kernel.
 #include "fa_decode_common.cuh"
@@ -30,9 +32,10 @@ constexpr int HM_LD = HM_T + 4;    // fp32 row pitch of the [head][token] buffer
 constexpr float HM_LAZY = 8.0f;
 constexpr float HM_P_SCALE = 128.0f;
 constexpr float HM_P_UNSCALE = 1.0f / 128.0f;
+constexpr int HM_EV_BYTES = 32768;  // staged E_V rows of one tile
 
 struct HmLayout {
-  int phi, red, esc, ph, qe, misc, total;  // byte offsets
+  int phi, red, esc, ph, qe, ev, misc, total;  // byte offsets
 };
 
 // phi: [64 tokens][F2] fp16; red: [8 warps][16 heads][HM_LD] fp32 partial scores;
@@ -45,8 +48,9 @@ __host__ __device__ inline HmLayout hm_layout(int F2) {
   L.esc = L.red + 8 * HM_NH * HM_LD * 4;
   L.ph = L.esc + HM_NH * HM_LD * 4;
   L.qe = L.ph + HM_NH * HM_T * 2;
-  L.misc = L.qe + HM_NH * FA_HEAD_DIM * 4;
-  L.total = L.misc + 4 * HM_NH * 4;
+  L.ev = L.qe + HM_NH * FA_HEAD_DIM * 4;
+  L.misc = L.ev + HM_EV_BYTES;
+  L.total = L.misc + 4 * HM_NH * 4 + HM_NH * 16;
   return L;
 }
 
@@ -99,6 +103,9 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
   float* wsc = reinterpret_cast<float*>(smem + Ly.misc);  // [16] 2^-e (W scale)
   float* wun = wsc + HM_NH;                               // [16] 2^e
   float* alph = wun + HM_NH;                              // [16] alpha of the tile
+  uint8_t* ev = smem + Ly.ev;                             // [KV head][64 tokens][evld] bf16
+  long long* kvb = reinterpret_cast<long long*>(alph + HM_NH);  // [16 / G] E offsets
+  int* kvd = reinterpret_cast<int*>(kvb + HM_NH);               // [16 / G] de_ld
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int hs = blockIdx.x / p.n_splits, sp = blockIdx.x - (blockIdx.x / p.n_splits) * p.n_splits;
@@ -116,6 +123,28 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
     const int h = idx >> 7, d = idx & 127;
     qe[idx] = h < nvh ? p.qw[(gh0 + h) * p.qw_stride + d] : 0.0f;
   }
+  const int nkv = HM_NH / p.G;  // KV heads of the CTA (G divides 16)
+  if (tid < nkv) {
+    const long long gh = gh0 + (long long)tid * p.G;
+    if (gh < bhq) {
+      const int bb = (int)(gh / p.Hq), gg = (int)(gh - (long long)bb * p.Hq) / p.G;
+      kvb[tid] = (long long)bb * p.e_batch + p.e_off[gg];
+      kvd[tid] = p.de_ld[gg];
+    } else {
+      kvb[tid] = 0;
+      kvd[tid] = 0;
+    }
+  }
+  // E_V rows of a tile staged in shared memory when they fit (row pitch evld elements)
+  int evld = 8;
+  for (int g2 = 0; g2 < nkv; ++g2) {
+    const long long gh = gh0 + (long long)g2 * p.G;
+    if (gh < bhq) {
+      const int bb = (int)(gh / p.Hq), gg = (int)(gh - (long long)bb * p.Hq) / p.G;
+      evld = max(evld, p.de_ld[gg]);
+    }
+  }
+  const bool stage = nkv * HM_T * evld * 2 <= HM_EV_BYTES;
   if (tid < HM_NH) {
     float wmax = 0.0f;
     if (tid < nvh) {
@@ -188,6 +217,18 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
   for (int i = 0; i < ntiles; ++i) {
     const int t0 = lo + i * HM_T;
     const int nt = min(HM_T, hi - t0);
+    if (stage) {  // this tile's E_V rows -> shared memory, landing while A-E run
+      const int cpr = evld / 8;  // 16-byte chunks per staged row
+      for (int idx = tid; idx < nkv * HM_T * cpr; idx += HM_THREADS) {
+        const int kv = idx / (HM_T * cpr), rem = idx - kv * (HM_T * cpr);
+        const int t = rem / cpr, c = rem - (rem / cpr) * cpr;
+        const int dle = kvd[kv];
+        if (t < nt && 8 * c < dle)
+          cp_async16(ev + ((kv * HM_T + t) * evld + 8 * c) * 2,
+                     p.EV + kvb[kv] + (long long)(t0 + t) * dle + 8 * c);
+      }
+      cp_async_commit();
+    }
     // ---- A: basis tile
 #pragma unroll
     for (int u = 0; u < NFT; ++u) {
@@ -292,6 +333,7 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
       for (int u = 0; u < 4; ++u) esc[sh * HM_LD + 4 * sq + u] = s4[u];
       if (sq == 0) alph[sh] = alpha;
     }
+    if (stage) cp_async_wait<0>();  // this thread's staged rows landed
     __syncthreads();
     // ---- E: U += P . Phi over this warp's slots
     {
@@ -329,15 +371,27 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) acc8[e] *= a;
       if (vh < nvh && 8 * vc < v_de) {
-        const __nv_bfloat16* col = p.EV + v_base + (long long)t0 * v_ld + 8 * vc;
         const float* pv = esc + vh * HM_LD;
+        if (stage) {
+          const uint8_t* col = ev + ((vh / p.G) * HM_T * evld + 8 * vc) * 2;
 #pragma unroll 8
-        for (int t = 0; t < nt; ++t) {
-          float x[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(col + (long long)t * v_ld), x);
-          const float pt = pv[t];
+          for (int t = 0; t < nt; ++t) {
+            float x[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(col + t * evld * 2), x);
+            const float pt = pv[t];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc8[e] += pt * x[e];
+            for (int e = 0; e < 8; ++e) acc8[e] += pt * x[e];
+          }
+        } else {
+          const __nv_bfloat16* col = p.EV + v_base + (long long)t0 * v_ld + 8 * vc;
+#pragma unroll 8
+          for (int t = 0; t < nt; ++t) {
+            float x[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4*>(col + (long long)t * v_ld), x);
+            const float pt = pv[t];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc8[e] += pt * x[e];
+          }
         }
       }
     }
