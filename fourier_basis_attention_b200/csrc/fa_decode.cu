@@ -667,7 +667,7 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   c->tc = (M > 0 && plan->e_token_major) ? 1 : 0;
   // The warp-MMA split kernel (16 query heads per CTA, U in registers) takes the other
   // plans with 256 <= k <= 1023 (2F rounded up to 512 or 1024 slots).
-  c->hm_F2 = 2 * c->F <= 256 ? 256 : (2 * c->F <= 512 ? 512 : 1024);
+  c->hm_F2 = 2 * c->F <= 512 ? 512 : 1024;
   c->hm = (!c->tc && M > 0 && sh.k >= 256 && c->hm_F2 <= 1024) ? 1 : 0;
   int cols = 32;  // U (2F slots), S (2 x 32 tokens), W_lo (2F / 2 columns of slot pairs)
   while (cols < c->tc_F2 + 64 + c->tc_F2 / 2) cols <<= 1;

@@ -181,7 +181,7 @@ __host__ __device__ constexpr size_t sink_recent_smem_bytes() {
   return (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + DNT * 8) * 4;
 }
 
-// Warp-MMA split kernel over per-KV-head E blocks, F2 = 256, 512 or 1024 slots.
+// Warp-MMA split kernel over per-KV-head E blocks, F2 = 512 or 1024 slots.
 cudaError_t launch_decode_hmma(const DecodeParams& p, int F2, cudaStream_t stream);
 size_t decode_hmma_smem_bytes(int F2);
 

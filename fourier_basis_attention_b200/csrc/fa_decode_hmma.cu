@@ -436,8 +436,7 @@ static cudaError_t launch_hm(const DecodeParams& p, int grid, cudaStream_t strea
 cudaError_t launch_decode_hmma(const DecodeParams& p, int F2, cudaStream_t stream) {
   const int heads = p.B * p.Hq;
   const int grid = ((heads + HM_NH - 1) / HM_NH) * p.n_splits;
-  switch (F2) {
-    case 256: return launch_hm<2>(p, grid, stream);
+  switch (F2) {  // the plans sent here have 256 <= k <= 1023
     case 512: return launch_hm<4>(p, grid, stream);
     case 1024: return launch_hm<8>(p, grid, stream);
     default: return cudaErrorInvalidValue;
