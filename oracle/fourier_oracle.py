@@ -30,6 +30,13 @@ Readings of points the pages leave open (each is listed in the design notes):
   window keeps the remaining min(R, L - S) tokens, and every token is stored once.
 * Decode: one query per sequence attends to all L cached tokens with softmax scale
   1/sqrt(D); query head h reads KV head h // (Hq / Hkv).
+* Basis period. By default the basis period P equals the middle length M. A cache that
+  takes appended tokens during decoding keeps a fixed period P >= M (its capacity):
+  the middle tokens t < M are projected onto the period-P functions, which is the same
+  as projecting the middle zero-padded to P tokens (pinned against a library FFT), and
+  a token that leaves the recent window joins the middle at t = M. The pages say only
+  that the spectral coefficients have a fixed length; they do not say how the cache is
+  maintained while decoding.
 
 Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
 (closed forms, library FFT equality, orthonormality, Parseval, brute force).
@@ -83,29 +90,31 @@ def split_dims(mask_row) -> tuple[np.ndarray, np.ndarray]:
 
 
 def _norm(f: np.ndarray, M: int) -> np.ndarray:
-    """Orthonormal scale of frequency f: 1/sqrt(M) for DC and Nyquist, else sqrt(2/M)."""
+    """Orthonormal scale of frequency f over period M: 1/sqrt(M) for DC and Nyquist,
+    else sqrt(2/M)."""
     single = (f == 0) | (2 * f == M)
     return np.where(single, 1.0 / np.sqrt(M), np.sqrt(2.0 / M))
 
 
 @lru_cache(maxsize=2)
-def _basis_full(M: int, k: int) -> np.ndarray:
-    """The whole table, cached (read-only) so that one head's K, V and reconstruction
-    share it; the values are those of ``basis``."""
-    phi = basis(M, k, 0, M)
+def _basis_full(P: int, k: int, M: int) -> np.ndarray:
+    """Rows 0..M-1 of the period-P table, cached (read-only) so that one head's K, V and
+    reconstruction share it; the values are those of ``basis``."""
+    phi = basis(P, k, 0, M)
     phi.setflags(write=False)
     return phi
 
 
 def basis(M: int, k: int, t0: int = 0, t1: int | None = None) -> np.ndarray:
-    """Rows t0..t1-1 of Phi (M x k), Phi[t, j] = phi_j(t), in fp64.
+    """Rows t0..t1-1 of Phi (M x k), Phi[t, j] = phi_j(t), in fp64; M is the period.
 
     [abstract]: "orthogonal Fourier bases"; [skill] "Architecture overview": a
     translation (shift) Fourier transform turns the span into k << L fixed-length
     spectral coefficients. Function j: j = 0 is the constant; for j >= 1 the frequency
     is f = (j + 1) // 2, odd j is the cosine and even j the sine of 2*pi*f*t/M.
     The phase f*t is reduced modulo M in exact integer arithmetic before the fp64
-    cos/sin, so large M loses no accuracy.
+    cos/sin, so large M loses no accuracy. Rows past the period (t1 > M) are allowed;
+    a cache with reserved room evaluates rows t < (its middle length) <= M.
     """
     if not (1 <= k <= M):
         raise ValueError(f"need 1 <= k <= M, got k={k}, M={M}")
@@ -129,6 +138,7 @@ class Hybrid:
     recent: [R_eff, D]  tokens [L - R_eff, L), all dims, exact
     E:      [M, De]     middle tokens, retained dims ``ed`` (ascending), exact
     C:      [k, Dc]     Fourier coefficients of the middle tokens' compressed dims ``cd``
+    P:      basis period (P >= M; P == M unless room for appended tokens was reserved)
     """
 
     L: int
@@ -143,28 +153,35 @@ class Hybrid:
     recent: np.ndarray
     E: np.ndarray
     C: np.ndarray
+    P: int = 0
 
 
-def compress(X, mask_row, S: int, R: int, k: int) -> Hybrid:
+def compress(X, mask_row, S: int, R: int, k: int, period: int | None = None) -> Hybrid:
     """Compress one KV head's cache X [L, D] into its hybrid form.
 
     [skill] Step 3 splits the tokens, Step 2 projects the middle span onto the basis
     (``fourier_compress_kv_cache``); [abstract] restricts the projection to the
-    long-context-insensitive dims. C = Phi^T X[S:L-R, cd] (fp64 BLAS).
+    long-context-insensitive dims. C = Phi^T X[S:L-R, cd] (fp64 BLAS), with Phi the
+    first M rows of the period-P basis (``period``; default P = M, and P >= M).
+    A cache that had tokens appended while decoding is, by this reading, the cache of
+    the longer sequence with the period it was created with.
     """
     X = np.asarray(X, dtype=np.float64)
     L, D = X.shape
     s_eff, r_eff, M = partition(L, S, R)
+    P = M if period is None else int(period)
+    if M > 0 and P < M:
+        raise ValueError(f"period P={P} is shorter than the middle span M={M}")
     cd, ed = split_dims(mask_row)
     mid = X[s_eff:L - r_eff]
     if M > 0 and cd.size > 0:
-        phi = _basis_full(M, k)
+        phi = _basis_full(P, k, M)
         C = phi.T @ mid[:, cd]
     else:
         C = np.zeros((k if M > 0 else 0, cd.size))
     return Hybrid(L=L, D=D, S=s_eff, R=r_eff, M=M, k=k, cd=cd, ed=ed,
                   sink=X[:s_eff].copy(), recent=X[L - r_eff:].copy(),
-                  E=mid[:, ed].copy(), C=C)
+                  E=mid[:, ed].copy(), C=C, P=P)
 
 
 def reconstruct(h: Hybrid) -> np.ndarray:
@@ -172,7 +189,8 @@ def reconstruct(h: Hybrid) -> np.ndarray:
 
     [skill] Step 4 (``reconstruct_from_fourier``): zero-filled spectrum, inverse
     transform to the original length. Here written as the basis expansion Phi @ C,
-    which equals that truncated inverse real FFT (pinned in the tests).
+    which equals that truncated inverse real FFT (pinned in the tests). With a period
+    P > M the expansion is evaluated on the first M rows of the period-P basis.
     """
     Xt = np.zeros((h.L, h.D))
     Xt[:h.S] = h.sink
@@ -181,7 +199,7 @@ def reconstruct(h: Hybrid) -> np.ndarray:
         mid = np.zeros((h.M, h.D))
         mid[:, h.ed] = h.E
         if h.cd.size > 0:
-            mid[:, h.cd] = _basis_full(h.M, h.k) @ h.C
+            mid[:, h.cd] = _basis_full(h.P or h.M, h.k, h.M) @ h.C
         Xt[h.S:h.S + h.M] = mid
     return Xt
 

@@ -56,6 +56,26 @@ def check_truncated_irfft(basis_fn, M, kb, rng):
     return np.abs(phi @ (phi.T @ x) - ref).max()
 
 
+def check_period_rfft(basis_fn, P, M, k, rng):
+    """Rows t < M of the period-P basis against numpy's rfft of the M samples zero-padded
+    to P (n=P): the same bin relations as check_rfft_bins, with P in place of M."""
+    x = rng.standard_normal(M)
+    C = basis_fn(P, k, 0, M).T @ x
+    R = np.fft.rfft(np.concatenate([x, np.zeros(P - M)]), n=P)
+    ref = np.empty(k)
+    for j in range(k):
+        f = (j + 1) // 2
+        if j == 0:
+            ref[j] = R[0].real / np.sqrt(P)
+        elif 2 * f == P:
+            ref[j] = R[f].real / np.sqrt(P)
+        elif j % 2 == 1:
+            ref[j] = np.sqrt(2.0 / P) * R[f].real
+        else:
+            ref[j] = -np.sqrt(2.0 / P) * R[f].imag
+    return np.abs(C - ref).max() / max(1.0, np.abs(ref).max())
+
+
 # ----------------------------------------------------------------------------- partition
 
 def test_partition_brute_force():
@@ -196,6 +216,42 @@ def test_sink_recent_retained_are_exact_copies():
     assert np.abs(Xt[S:L - R][:, cd] - X[S:L - R][:, cd]).max() > 1e-3
 
 
+@pytest.mark.parametrize("P,M,k", [(700, 500, 63), (701, 300, 255), (1024, 1023, 1024),
+                                   (64, 1, 64), (4099, 4000, 255)])
+def test_period_rows_equal_zero_padded_rfft(P, M, k):
+    """A cache with reserved room projects its M middle tokens onto the period-P basis:
+    that is the rfft of the middle zero-padded to P samples."""
+    assert check_period_rfft(fo.basis, P, M, k, np.random.default_rng(P + M)) < TOL
+
+
+@pytest.mark.parametrize("P,M", [(40, 31), (64, 63), (129, 100)])
+def test_period_full_basis_reconstructs_exactly(P, M):
+    """k = P functions of period P are a complete orthonormal basis of P samples, so the
+    zero-padded middle, and with it every middle token, is reconstructed exactly."""
+    rng = np.random.default_rng(P)
+    S, R, D = 4, 3, 128
+    X = rng.standard_normal((S + M + R, D))
+    mask = (rng.random(D) < 0.75).astype(np.uint8)
+    h = fo.compress(X, mask, S, R, P, period=P)
+    assert h.P == P and h.M == M
+    assert np.abs(fo.reconstruct(h) - X).max() < 1e-12
+    q = rng.standard_normal((2, D))
+    hv = fo.compress(X[::-1].copy(), mask, S, R, P, period=P)
+    ref = fo.attention(q, X, X[::-1], 1 / np.sqrt(D))
+    assert np.abs(fo.decode(q, h, hv) - ref).max() < 1e-12
+
+
+def test_period_default_is_the_middle_length():
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((300, 128))
+    mask = (rng.random(128) < 0.75).astype(np.uint8)
+    a = fo.compress(X, mask, 16, 32, 31)
+    b = fo.compress(X, mask, 16, 32, 31, period=a.M)
+    assert a.P == a.M == 252 and np.array_equal(a.C, b.C)
+    with pytest.raises(ValueError):
+        fo.compress(X, mask, 16, 32, 31, period=a.M - 1)
+
+
 # ----------------------------------------------------------------------------- attention
 
 def test_attention_hand_case(hand_cases):
@@ -283,6 +339,23 @@ def _mutant(kind):
             phi = base * np.where((f == 0) | (2 * f == M), 1 / np.sqrt(M), np.sqrt(2.0 / M))
         return phi
     return fn
+
+
+def _period_mutant(kind):
+    """Slips in handling a period P longer than the M rows evaluated."""
+    def fn(P, k, t0=0, t1=None):
+        M = P if t1 is None else t1
+        if kind == "period_is_rows":        # the row count used as the period
+            return fo.basis(M, k, t0, t1)
+        if kind == "norm_over_rows":        # right functions, scale of the M-row span
+            return fo.basis(P, k, t0, t1) * np.sqrt(P / M)
+        raise ValueError(kind)
+    return fn
+
+
+@pytest.mark.parametrize("kind", ["period_is_rows", "norm_over_rows"])
+def test_period_pins_reject_planted_mistakes(kind):
+    assert check_period_rfft(_period_mutant(kind), 700, 500, 63, np.random.default_rng(1)) > TOL
 
 
 @pytest.mark.parametrize("kind", ["sin_sign", "swap_cos_sin", "norm_dc_like", "freq_off_by_one",
