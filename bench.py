@@ -277,7 +277,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
+        fa.fa_build_basis(plan.P, w.k, phiT, plan.phi_ld, False, stream)
         fa.fa_compress(plan, K, V, phiT, cache, stream)
         fa.fa_decode(plan, q, cache, out, ws, 0, stream)
 
@@ -302,7 +302,7 @@ def run_ours(args):
     for i in range(args.steps):
         e = ev[i]
         e[0].record(stream)
-        fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
+        fa.fa_build_basis(plan.P, w.k, phiT, plan.phi_ld, False, stream)
         e[1].record(stream)
         fa.fa_compress(plan, K, V, phiT, cache, stream)
         e[2].record(stream)
@@ -360,7 +360,7 @@ def run_ours(args):
             Kd.copy_(Kh, non_blocking=True)
             Vd.copy_(Vh, non_blocking=True)
             qd.copy_(qh, non_blocking=True)
-            fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
+            fa.fa_build_basis(plan.P, w.k, phiT, plan.phi_ld, False, stream)
             fa.fa_compress(plan, Kd, Vd, phiT, cache, stream)
             fa.fa_decode(plan, qd, cache, out, ws, 0, stream)
             oh.copy_(out, non_blocking=True)
@@ -500,6 +500,43 @@ def _time_graph(fn, n):
     return a.elapsed_time(b) / n
 
 
+APPEND_STEPS = 50
+
+
+def append_bytes(plan):
+    """Algorithmic bytes of one fa_append: per (batch, KV head) and K / V, the k x dc_ld
+    coefficient block read and written, one E row written, the leaving ring row read, the
+    new token read and written to the ring."""
+    s = plan.shape
+    per = sum(2 * plan.kk * plan.dc_ld[g] * 4 + plan.de_ld[g] * 2 + 3 * 128 * 2
+              for g in range(s.Hkv))
+    return 2 * s.B * per
+
+
+def time_append(w, plan, K, V, stream):
+    """Device time of one fa_append (one new token per sequence) on a copy of ``plan`` with
+    room reserved for the warm-up and timed appends; returns (ms, bytes per launch)."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    pa = fa.fa_plan.from_buffer_copy(plan)
+    fa.fa_plan_reserve(pa, w.L + APPEND_STEPS + 3)
+    cache = fa.Cache(pa, device=K.device)
+    phiT = fa.basis_table(pa, device=K.device, stream=stream)
+    fa.fa_compress(pa, K, V, phiT, cache, stream)
+    kn = K[:, :, -1].contiguous()
+    vn = V[:, :, -1].contiguous()
+    app = lambda: fa.fa_append(pa, kn, vn, cache, stream)
+    for _ in range(3):
+        app()
+    nbytes = append_bytes(pa)
+    ms = _time(app, APPEND_STEPS, stream)
+    fa.fa_device_status(stream)
+    del cache, phiT
+    torch.cuda.empty_cache()
+    return ms, nbytes
+
+
 def run_sweep(args):
     """Per-workload timings (1 GPU): the four single-layer workloads, then the 32-layer
     LLaMA-3-8B-shaped cache: compress every layer (distinct seeded masks), and time one
@@ -525,7 +562,7 @@ def run_sweep(args):
         phiT = torch.empty(w.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
         ws = torch.empty(fa.fa_decode_workspace_size(plan), dtype=torch.uint8, device=dev)
         out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
-        basis = lambda: fa.fa_build_basis(plan.M, w.k, phiT, plan.phi_ld, False, stream)
+        basis = lambda: fa.fa_build_basis(plan.P, w.k, phiT, plan.phi_ld, False, stream)
         comp = lambda: fa.fa_compress(plan, K, V, phiT, cache, stream)
         dec = lambda: fa.fa_decode(plan, q, cache, out, ws, 0, stream)
         for f in (basis, comp, dec):
@@ -535,6 +572,8 @@ def run_sweep(args):
         td_eager = _time(dec, 20, stream)
         td = _time_graph(lambda s: fa.fa_decode(plan, q, cache, out, ws, 0, s), 20)
         fa.fa_device_status(stream)
+        del cache, ws
+        ta, a_bytes = time_append(w, plan, K, V, stream)
         wm = work_model(w, plan)
         print(json.dumps({"sweep": "single_layer", "workload": w.name, "basis_us": tb * 1e3,
                           "compress_us": tcmp * 1e3,
@@ -546,8 +585,10 @@ def run_sweep(args):
                           "decode_timing": "CUDA graph replay (eager launches in decode_us_eager)",
                           "decode_hbm_gbs": wm["decode_bytes"] / td / 1e6,
                           "decode_frac_hbm": wm["decode_bytes"] / td / 1e6 / hbm,
-                          "decode_fp32_tflops": wm["decode_flops"] / td / 1e9}), flush=True)
-        del K, V, cache, ws, out, phiT
+                          "decode_fp32_tflops": wm["decode_flops"] / td / 1e9,
+                          "append_us": ta * 1e3, "append_hbm_gbs": a_bytes / ta / 1e6,
+                          "append_frac_hbm": a_bytes / ta / 1e6 / hbm}), flush=True)
+        del K, V, out, phiT
         torch.cuda.empty_cache()
 
     points = [(B, L) for L in wl.SWEEP_L for B in wl.SWEEP_BATCH]
@@ -577,7 +618,7 @@ def run_sweep(args):
                 resident += 1
             if phiT is None:
                 phiT = torch.empty(wlay.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
-                fa.fa_build_basis(plan.M, wlay.k, phiT, plan.phi_ld, False, stream)
+                fa.fa_build_basis(plan.P, wlay.k, phiT, plan.phi_ld, False, stream)
             # the K / V of every layer are the same synthetic draw (its mask differs); the
             # compress cost does not depend on the values
             fa.fa_compress(plan, K, V, phiT, caches[-1], stream)

@@ -4,8 +4,8 @@ Argument marshalling only: every step of the hot path runs in the CUDA kernels o
 ``libfourier_attention.so`` behind the C ABI declared in ``include/fourier_attention.h``.
 PyTorch is used for device memory and streams. The functions keep the C names:
 
-    fa_plan_init, fa_build_basis, fa_compress, fa_decode_workspace_size, fa_decode,
-    fa_device_status, fa_last_error
+    fa_plan_init, fa_plan_reserve, fa_build_basis, fa_compress, fa_decode_workspace_size,
+    fa_decode, fa_decode_noalloc, fa_append, fa_device_status, fa_last_error
 
 There is no CPU fallback: if the shared library is missing or fails to load, importing
 this package raises.
@@ -25,9 +25,9 @@ MAX_K_DECODE = 2047
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE = range(5)
 FA_BF16, FA_F32 = 0, 1
 
-EXPORTED = ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode_workspace_size",
-            "fa_decode", "fa_decode_noalloc", "fa_device_status", "fa_watchdog_selftest",
-            "fa_last_error")
+EXPORTED = ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress",
+            "fa_decode_workspace_size", "fa_decode", "fa_decode_noalloc", "fa_append",
+            "fa_device_status", "fa_watchdog_selftest", "fa_last_error")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -49,7 +49,7 @@ class fa_plan(ctypes.Structure):
         ("shape", fa_shape),
         ("S", ctypes.c_int32), ("R", ctypes.c_int32), ("M", ctypes.c_int32),
         ("kk", ctypes.c_int32), ("G", ctypes.c_int32), ("phi_ld", ctypes.c_int32),
-        ("e_token_major", ctypes.c_int32),
+        ("e_token_major", ctypes.c_int32), ("P", ctypes.c_int32), ("recent_head", ctypes.c_int32),
         ("dc", ctypes.c_int32 * _H), ("de", ctypes.c_int32 * _H),
         ("dc_ld", ctypes.c_int32 * _H), ("de_ld", ctypes.c_int32 * _H),
         ("e_pitch", ctypes.c_int32 * _H),
@@ -77,7 +77,9 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     """Declare the C signatures on a loaded copy of the library."""
     P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
     lib.fa_plan_init.argtypes = [ctypes.POINTER(fa_shape), P, ctypes.POINTER(fa_plan)]
+    lib.fa_plan_reserve.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_build_basis.argtypes = [I32, I32, I32, I32, P, I64, P]
+    lib.fa_append.argtypes = [ctypes.POINTER(fa_plan), P, P, ctypes.POINTER(fa_cache), P]
     lib.fa_compress.argtypes = [ctypes.POINTER(fa_plan), P, P, P, ctypes.POINTER(fa_cache), P]
     lib.fa_decode_workspace_size.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_decode_workspace_size.restype = SZ
@@ -89,8 +91,8 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_watchdog_selftest.argtypes = [ctypes.c_uint32, P]
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
-    for name in ("fa_plan_init", "fa_build_basis", "fa_compress", "fa_decode", "fa_decode_noalloc",
-                 "fa_device_status", "fa_watchdog_selftest"):
+    for name in ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress", "fa_decode",
+                 "fa_decode_noalloc", "fa_append", "fa_device_status", "fa_watchdog_selftest"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -131,6 +133,12 @@ def fa_plan_init(B, Hq, Hkv, L, S, R, k, mask, D=HEAD_DIM) -> fa_plan:
     shape = fa_shape(B, Hq, Hkv, D, L, S, R, k)
     plan = fa_plan()
     _check(LIB.fa_plan_init(ctypes.byref(shape), m.ctypes.data, ctypes.byref(plan)))
+    return plan
+
+
+def fa_plan_reserve(plan: fa_plan, L_max: int) -> fa_plan:
+    """Room for tokens appended while decoding: basis period P = L_max - S - R (in place)."""
+    _check(LIB.fa_plan_reserve(ctypes.byref(plan), int(L_max)))
     return plan
 
 
@@ -175,6 +183,12 @@ def fa_decode_noalloc(plan: fa_plan, q, cache: "Cache", out, num_splits: int = 0
                                  out_dtype, num_splits, _stream(stream)))
 
 
+def fa_append(plan: fa_plan, k_new, v_new, cache: "Cache", stream=None) -> None:
+    """Append one token per sequence (k_new, v_new: bf16 [B, Hkv, 128]); advances ``plan``."""
+    _check(LIB.fa_append(ctypes.byref(plan), _ptr(k_new), _ptr(v_new), ctypes.byref(cache.c),
+                         _stream(stream)))
+
+
 def fa_device_status(stream=None) -> None:
     _check(LIB.fa_device_status(_stream(stream)))
 
@@ -205,6 +219,7 @@ class Cache:
 
     # views in the documented layouts (for tests and callers that inspect the cache)
     def F(self, which: str):
+        """[B, Hkv, S + R, 128]: sink rows, then the recent ring (oldest at S + recent_head)."""
         p = self.plan
         t = self.F_K if which == "K" else self.F_V
         return t[:p.f_elems].view(p.shape.B, p.shape.Hkv, p.S + p.R, HEAD_DIM)
@@ -219,7 +234,7 @@ class Cache:
         return t[off:off + p.kk * p.dc_ld[g]].view(p.kk, p.dc_ld[g])[:, :p.dc[g]]
 
     def E_raw(self, which: str, b: int, g: int):
-        """[M, de_ld] view of KV head (b, g)'s rows (strided when E is token-major)."""
+        """[M, de_ld] view of KV head (b, g)'s middle rows (strided when E is token-major)."""
         p = self.plan
         t = self.E_K if which == "K" else self.E_V
         off = b * p.e_batch + p.e_off[g]
@@ -233,12 +248,12 @@ class Cache:
 
 
 def basis_table(plan: fa_plan, device="cuda", stream=None):
-    """Allocate and fill the bf16 basis table fa_compress reads (None if M == 0)."""
+    """Allocate and fill the bf16 basis table (period P) fa_compress reads (None if M == 0)."""
     import torch
     if plan.M == 0:
         return None
     phiT = torch.empty(plan.shape.k, plan.phi_ld, dtype=torch.bfloat16, device=device)
-    fa_build_basis(plan.M, plan.shape.k, phiT, plan.phi_ld, normalized=False, stream=stream)
+    fa_build_basis(plan.P, plan.shape.k, phiT, plan.phi_ld, normalized=False, stream=stream)
     return phiT
 
 

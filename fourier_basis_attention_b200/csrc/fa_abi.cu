@@ -38,7 +38,7 @@ int check_ptr(const void* p, const char* name, bool required) {
 }
 
 // Fills the layout fields of a plan (everything below the dim split) from shape, S, R, M,
-// kk, G, dc and de. E is token-major exactly when the tensor-core decode is used: it can
+// P, kk, G, dc and de (E holds P rows per KV head). E is token-major exactly when the tensor-core decode is used: it can
 // run when k <= 255, G is 1, 2 or 4 and every KV head keeps at most 32 dims, and it is
 // chosen when the k-length work per token and KV head (k G) is at least 255 and there are
 // at least 128 query heads (one full tensor-core head set); below that (k = 63 with
@@ -65,10 +65,10 @@ void derive_layout(fa_plan* plan) {
       plan->de_ld[g] = round8(plan->de[g]);
       plan->e_off[g] = ee;
       plan->e_pitch[g] = plan->de_ld[g];
-      ee += (long long)plan->M * plan->de_ld[g];
+      ee += (long long)plan->P * plan->de_ld[g];
     }
   }
-  if (tm) ee = (long long)plan->M * s.Hkv * w;
+  if (tm) ee = (long long)plan->P * s.Hkv * w;
   plan->c_batch = ce;
   plan->e_batch = ee;
   plan->f_elems = (long long)s.B * s.Hkv * (plan->S + plan->R) * FA_HEAD_DIM;
@@ -89,6 +89,12 @@ int check_plan(const fa_plan* plan) {
     return fail(FA_ERR_INVALID, "plan token partition is inconsistent");
   if (plan->G != s.Hq / s.Hkv) return fail(FA_ERR_INVALID, "plan G is inconsistent");
   if (plan->kk != (plan->M > 0 ? s.k : 0)) return fail(FA_ERR_INVALID, "plan kk is inconsistent");
+  if (plan->P < plan->M || (plan->M == 0 && plan->P != 0))
+    return fail(FA_ERR_INVALID, "plan period P=%d is inconsistent with M=%d", plan->P, plan->M);
+  if (plan->phi_ld != round8(plan->P > 8 ? plan->P : 8))
+    return fail(FA_ERR_INVALID, "plan phi_ld is inconsistent");
+  if (plan->recent_head < 0 || plan->recent_head >= (plan->R > 0 ? plan->R : 1))
+    return fail(FA_ERR_INVALID, "plan recent_head is inconsistent");
   for (int g = 0; g < s.Hkv; ++g) {
     if (plan->dc[g] < 0 || plan->dc[g] > FA_HEAD_DIM || plan->de[g] != FA_HEAD_DIM - plan->dc[g])
       return fail(FA_ERR_INVALID, "plan dims of KV head %d are inconsistent", g);
@@ -138,7 +144,9 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) 
   plan->M = s.L - plan->S - plan->R;
   plan->kk = plan->M > 0 ? s.k : 0;
   plan->G = s.Hq / s.Hkv;
-  plan->phi_ld = round8(plan->M > 8 ? plan->M : 8);
+  plan->P = plan->M;
+  plan->recent_head = 0;
+  plan->phi_ld = round8(plan->P > 8 ? plan->P : 8);
   bool any_dc = false;
   for (int g = 0; g < s.Hkv; ++g) {
     int n = 0;
@@ -152,6 +160,21 @@ int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan) 
   }
   if (plan->M > 0 && any_dc && s.k > plan->M)
     return fail(FA_ERR_UNSUPPORTED, "k=%d exceeds the middle span M=%d", s.k, plan->M);
+  derive_layout(plan);
+  return FA_OK;
+}
+
+int fa_plan_reserve(fa_plan* plan, int32_t L_max) {
+  if (int r = check_plan(plan)) return r;
+  if (plan->M < 1) return fail(FA_ERR_UNSUPPORTED, "fa_plan_reserve needs a middle span (M >= 1)");
+  if (plan->P != plan->M || plan->recent_head != 0)
+    return fail(FA_ERR_UNSUPPORTED, "plan already has room reserved or tokens appended");
+  const long long P = (long long)L_max - plan->S - plan->R;
+  if (L_max < plan->shape.L || P >= (1 << 21))
+    return fail(FA_ERR_INVALID, "L_max=%d must satisfy L=%d <= L_max and L_max - S - R < 2^21",
+                L_max, plan->shape.L);
+  plan->P = (int32_t)P;
+  plan->phi_ld = round8(plan->P > 8 ? plan->P : 8);
   derive_layout(plan);
   return FA_OK;
 }
@@ -201,7 +224,7 @@ static int decode_checks(const fa_plan* plan) {
     return fail(FA_ERR_UNSUPPORTED, "fa_decode supports Hq/Hkv in {1, 2, 4, 8}, got %d", G);
   if (plan->M > 0 && plan->shape.k > FA_MAX_K_DECODE)
     return fail(FA_ERR_UNSUPPORTED, "fa_decode supports k <= %d, got %d", FA_MAX_K_DECODE, plan->shape.k);
-  if (plan->M >= (1 << 21)) return fail(FA_ERR_UNSUPPORTED, "fa_decode supports M < 2^21");
+  if (plan->P >= (1 << 21)) return fail(FA_ERR_UNSUPPORTED, "fa_decode supports P < 2^21");
   return FA_OK;
 }
 
@@ -237,6 +260,31 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
   e = fa::launch_decode(plan, c, q, cache, out, out_dtype, workspace,
                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fa_decode: launch");
+  return FA_OK;
+}
+
+int fa_append(fa_plan* plan, const void* k_new, const void* v_new, const fa_cache* cache,
+              void* stream) {
+  if (int r = check_plan(plan)) return r;
+  if (plan->M < 1) return fail(FA_ERR_UNSUPPORTED, "fa_append needs a middle span (M >= 1)");
+  if (plan->M >= plan->P)
+    return fail(FA_ERR_UNSUPPORTED, "no room left: M = P = %d (see fa_plan_reserve)", plan->P);
+  if (plan->kk > FA_MAX_K_DECODE)
+    return fail(FA_ERR_UNSUPPORTED, "fa_append supports k <= %d, got %d", FA_MAX_K_DECODE, plan->kk);
+  if (!cache) return fail(FA_ERR_INVALID, "cache is NULL");
+  if (int r = check_ptr(k_new, "k_new", true)) return r;
+  if (int r = check_ptr(v_new, "v_new", true)) return r;
+  if (int r = check_ptr(cache->F_K, "cache->F_K", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->F_V, "cache->F_V", plan->f_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_K, "cache->E_K", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->E_V, "cache->E_V", plan->e_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_K, "cache->C_K", plan->c_elems > 0)) return r;
+  if (int r = check_ptr(cache->C_V, "cache->C_V", plan->c_elems > 0)) return r;
+  cudaError_t e = fa::launch_append(plan, k_new, v_new, cache, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_append: launch");
+  plan->M += 1;
+  plan->shape.L += 1;
+  if (plan->R > 0) plan->recent_head = (plan->recent_head + 1) % plan->R;
   return FA_OK;
 }
 

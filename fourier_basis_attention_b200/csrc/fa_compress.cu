@@ -53,7 +53,7 @@ struct CkCfg {
 
 
 struct CompressParams {
-  int M, k, S, L, Hkv, n_ktiles, n_pairs;
+  int M, P, k, S, L, Hkv, n_ktiles, n_pairs;
   const void* K;
   const void* V;
   float norm_single, norm_pair;
@@ -321,7 +321,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
           if (r >= rows) continue;
           const int j = jt + r;
           const int f = (j + 1) >> 1;
-          const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+          const float nrm = (f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair;
           float v[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -343,10 +343,11 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   }
 }
 
-// Sink and recent rows, all dims: F[head][i] = X[head][i < S ? i : L - R + (i - S)].
+// Sink and recent rows, all dims: F[head][i] = X[head][i] for i < S; the recent rows form
+// a ring starting at row S + rhead: F[head][S + (rhead + a) % R] = X[head][L - R + a].
 __global__ void __launch_bounds__(256) copy_sink_recent_kernel(
     const uint4* __restrict__ K, const uint4* __restrict__ V, uint4* __restrict__ FK,
-    uint4* __restrict__ FV, int L, int S, int R, long long n_heads) {
+    uint4* __restrict__ FV, int L, int S, int R, int rhead, long long n_heads) {
   const int nrow = S + R;
   const long long total = n_heads * nrow * 16;  // 16 x 16 bytes per 128-dim row
   for (long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x; id < total;
@@ -355,7 +356,8 @@ __global__ void __launch_bounds__(256) copy_sink_recent_kernel(
     const int c = (int)(id & 15);
     const long long head = row / nrow;
     const int i = (int)(row - head * nrow);
-    const long long t = (i < S) ? i : (long long)(L - R) + (i - S);
+    const int a = i - S - rhead < 0 ? i - S - rhead + R : i - S - rhead;  // age in the ring
+    const long long t = (i < S) ? i : (long long)(L - R) + a;
     const long long src = ((head * L + t) << 4) + c;
     FK[id] = K[src];
     FV[id] = V[src];
@@ -421,7 +423,7 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
     copy_sink_recent_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const uint4*>(K), static_cast<const uint4*>(V),
         static_cast<uint4*>(cache->F_K), static_cast<uint4*>(cache->F_V), sh.L, plan->S,
-        plan->R, n_heads);
+        plan->R, plan->recent_head, n_heads);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -464,6 +466,7 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   CompressParams cp;
   memset(&cp, 0, sizeof(cp));
   cp.M = plan->M;
+  cp.P = plan->P;
   cp.k = sh.k;
   cp.S = plan->S;
   cp.L = sh.L;
@@ -484,8 +487,8 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   }
   cp.C[0] = static_cast<float*>(cache->C_K);
   cp.C[1] = static_cast<float*>(cache->C_V);
-  cp.norm_single = (float)(1.0 / sqrt((double)plan->M));
-  cp.norm_pair = (float)sqrt(2.0 / (double)plan->M);
+  cp.norm_single = (float)(1.0 / sqrt((double)plan->P));
+  cp.norm_pair = (float)sqrt(2.0 / (double)plan->P);
   cp.E[0] = static_cast<__nv_bfloat16*>(cache->E_K);
   cp.E[1] = static_cast<__nv_bfloat16*>(cache->E_V);
 

@@ -66,7 +66,7 @@ __global__ void __launch_bounds__(DNT) decode_prologue_kernel(const __grid_const
     }
     const int f = (j + 1) >> 1;
     const int comp = (j > 0 && (j & 1) == 0) ? 1 : 0;
-    const float nrm = (f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair;
+    const float nrm = (f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair;
 #pragma unroll
     for (int h = 0; h < HL; ++h) {
       if (h < p.G) {
@@ -84,7 +84,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   const int hs = cta / p.n_splits, sp = cta - (cta / p.n_splits) * p.n_splits;
   const int lo = sp * p.split_len;
   const int hi = min(p.M, lo + p.split_len);
-  const int M = p.M;
+  const int P = p.P;  // basis period
 
   float* Ws = sm;                           // [F_pad][cos | sin][HL]
   float* qes = Ws + p.F_pad * HL * 2;       // [HL][128]
@@ -149,7 +149,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
   float cb[SPT], sb[SPT];
 #pragma unroll
   for (int j = 0; j < SPT; ++j) {
-    phase_sincos((long long)(ui + j * p.NTU) % M, M, p.two_over_M, &sb[j], &cb[j]);
+    phase_sincos((long long)(ui + j * p.NTU) % P, P, p.two_over_P, &sb[j], &cb[j]);
 #pragma unroll
     for (int pr2 = 0; pr2 < HL / 2; ++pr2) ucs[j][pr2] = uss[j][pr2] = make_float2(0.0f, 0.0f);
   }
@@ -194,10 +194,10 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
       }
       if (fb < fe) {
         float sa, ca;
-        phase_sincos(tm, M, p.two_over_M, &sa, &ca);
+        phase_sincos(tm, P, p.two_over_P, &sa, &ca);
         for (int f0 = fb; f0 < fe; f0 += 32) {
           float s, c;
-          phase_sincos(((long long)f0 * tm) % M, M, p.two_over_M, &s, &c);
+          phase_sincos(((long long)f0 * tm) % P, P, p.two_over_P, &s, &c);
           const int f1 = min(fe, f0 + 32);
           for (int f = f0; f < f1; ++f) {
             const float4* w4 = reinterpret_cast<const float4*>(Ws + f * (HL * 2));
@@ -325,7 +325,7 @@ __device__ __forceinline__ void decode_middle(const DecodeParams& p, float* sm, 
         float c[SPT], s[SPT];
 #pragma unroll
         for (int j = 0; j < SPT; ++j)
-          phase_sincos(((long long)(ui + j * p.NTU) * (t0 + tb)) % M, M, p.two_over_M, &s[j],
+          phase_sincos(((long long)(ui + j * p.NTU) * (t0 + tb)) % P, P, p.two_over_P, &s[j],
                        &c[j]);
         for (int t = tb; t < te; ++t) {
           const float4 pa = *reinterpret_cast<const float4*>(ps + t * HL);
@@ -586,7 +586,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
         const int j = j0 + jj, f = (j + 1) >> 1;
         const int slot = FA_HEAD_DIM + 2 * f + ((j > 0 && (j & 1) == 0) ? 1 : 0);
         const float cv = cvs[jj * FA_HEAD_DIM + colc] *
-                         ((f == 0 || 2 * f == p.M) ? p.norm_single : p.norm_pair);
+                         ((f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair);
 #pragma unroll
         for (int h = 0; h < HL; ++h)
           if (h < G) acc[h] += sum[h * payload + slot] * cv;
@@ -767,10 +767,11 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   p.DEC = c.DEC;
   p.TGE = c.TGE;
   p.qscale = (float)(1.4426950408889634 / sqrt((double)FA_HEAD_DIM));
-  const int Mq = plan->M > 0 ? plan->M : 1;
-  p.norm_single = (float)(1.0 / sqrt((double)Mq));
-  p.norm_pair = (float)sqrt(2.0 / (double)Mq);
-  p.two_over_M = (float)(2.0 / (double)Mq);
+  const int Pq = plan->P > 0 ? plan->P : 1;  // basis period
+  p.P = Pq;
+  p.norm_single = (float)(1.0 / sqrt((double)Pq));
+  p.norm_pair = (float)sqrt(2.0 / (double)Pq);
+  p.two_over_P = (float)(2.0 / (double)Pq);
   p.e_batch = plan->e_batch;
   p.c_batch = plan->c_batch;
   for (int g = 0; g < sh.Hkv; ++g) {

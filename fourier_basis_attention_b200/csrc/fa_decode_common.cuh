@@ -14,14 +14,14 @@ constexpr int HL = 8;     // query heads per CTA (zero-padded)
 constexpr int FT = 256;   // sink/recent rows per CTA
 
 struct DecodeParams {
-  int B, Hq, Hkv, G, M, k, F, F_pad, nF;
+  int B, Hq, Hkv, G, M, P, k, F, F_pad, nF;  // M middle tokens, P basis period
   int n_splits, split_len, n_fsplits, NKV, n_mid, n_rec;
   int rec_stride, qw_stride;
   int NTU, TG, DEC, TGE;
   int tc_F2, tc_tmem_cols;  // tensor-core split kernel: coefficient slots, TMEM columns
   int e_row;                // token-major E: elements per token row of a batch
   int tc_nf;                // sink / recent CTAs at the front of the tensor-core grid
-  float qscale, norm_single, norm_pair, two_over_M;
+  float qscale, norm_single, norm_pair, two_over_P;
   long long e_batch, c_batch;
   long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
   int de[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS], dc[FA_MAX_KV_HEADS], dc_ld[FA_MAX_KV_HEADS];
@@ -34,11 +34,11 @@ struct DecodeParams {
   float* rec;
 };
 
-// cos / sin of 2 pi r / M for an exactly reduced integer phase 0 <= r < M.
-__device__ __forceinline__ void phase_sincos(long long r, int M, float two_over_M, float* s,
+// cos / sin of 2 pi r / P for an exactly reduced integer phase 0 <= r < P.
+__device__ __forceinline__ void phase_sincos(long long r, int P, float two_over_P, float* s,
                                              float* c) {
-  const long long rr = (2 * r > M) ? r - M : r;  // (-M/2, M/2]
-  sincospif((float)rr * two_over_M, s, c);
+  const long long rr = (2 * r > P) ? r - P : r;  // (-P/2, P/2]
+  sincospif((float)rr * two_over_P, s, c);
 }
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&x)[8]) {

@@ -112,7 +112,7 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
   const int lo = sp * p.split_len;
   const int hi = min(p.M, lo + p.split_len);
   const int ntiles = (hi - lo + HM_T - 1) / HM_T;
-  const int M = p.M;
+  const int P = p.P;  // basis period
   const long long bhq = (long long)p.B * p.Hq;
   const long long gh0 = (long long)hs * HM_NH;  // first query head of the CTA
   const int nvh = (int)max(0LL, min((long long)HM_NH, bhq - gh0));
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
     const int f = tid + HM_THREADS * u;
     ra[u] = 1.0f;
     rb[u] = 0.0f;
-    if (f < F2 / 2) phase_sincos(f % M, M, p.two_over_M, &rb[u], &ra[u]);
+    if (f < F2 / 2) phase_sincos(f % P, P, p.two_over_P, &rb[u], &ra[u]);
   }
 
   for (int i = 0; i < ntiles; ++i) {
@@ -235,7 +235,7 @@ __global__ void __launch_bounds__(HM_THREADS, 1)
       const int f = tid + HM_THREADS * u;
       if (f < F2 / 2) {
         float s, c;
-        phase_sincos(((long long)f * t0) % M, M, p.two_over_M, &s, &c);
+        phase_sincos(((long long)f * t0) % P, P, p.two_over_P, &s, &c);
         const int chunk = f >> 2, within = (f & 3) * 4;
 #pragma unroll 8
         for (int tau = 0; tau < HM_T; ++tau) {

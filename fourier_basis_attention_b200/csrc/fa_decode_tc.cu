@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const int lo = sp * p.split_len;
   const int hi = min(p.M, lo + p.split_len);
   const int ntiles = (hi - lo + TC_T - 1) / TC_T;
-  const int M = p.M;
+  const int P = p.P;  // basis period
   const long long bhq = (long long)p.B * p.Hq;
 
   if (threadIdx.x == 0) {
@@ -283,13 +283,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // the token's 128-byte row, 16-byte chunk swizzled by the token.
     const int gt = threadIdx.x - 160;
     const int nf = F2 / 2;
-    float ra[2], rb[2];  // cos, sin of 2 pi f / M
+    float ra[2], rb[2];  // cos, sin of 2 pi f / P
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int f = gt + TC_GEN * u;
       ra[u] = 1.0f;
       rb[u] = 0.0f;
-      if (f < nf) phase_sincos(f % M, M, p.two_over_M, &rb[u], &ra[u]);
+      if (f < nf) phase_sincos(f % P, P, p.two_over_P, &rb[u], &ra[u]);
     }
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
@@ -302,7 +302,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const int f = gt + TC_GEN * u;
         if (f < nf) {
           float s, c;
-          phase_sincos(((long long)f * tm0) % M, M, p.two_over_M, &s, &c);
+          phase_sincos(((long long)f * tm0) % P, P, p.two_over_P, &s, &c);
           uint8_t* base = PHI + b * phi_bytes + (f >> 5) * (TC_T * 128) + 4 * (f & 3);
           const int chunk = (f & 31) >> 2;
 #pragma unroll 8

@@ -26,6 +26,8 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
                           const fa_cache* cache, void* out, int out_dtype, void* workspace,
                           cudaStream_t stream);
+cudaError_t launch_append(const fa_plan* plan, const void* k_new, const void* v_new,
+                          const fa_cache* cache, cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
 cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream);
 

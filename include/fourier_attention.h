@@ -71,13 +71,24 @@ typedef struct fa_shape {
  * head g, perm[g][0 .. dc[g]) lists the compressed dims in ascending order and
  * perm[g][dc[g] .. 128) the retained dims in ascending order.
  *
+ * Basis period P: the middle span is projected onto the first k functions of the
+ *   orthonormal real Fourier basis of period P. fa_plan_init sets P = M. A cache that
+ *   takes appended tokens while decoding (fa_append) is planned with room for them
+ *   (fa_plan_reserve): P = L_max - S - R >= M stays fixed while M grows, and the middle
+ *   tokens t < M are projected onto the period-P functions, which equals projecting the
+ *   middle zero-padded to P tokens. (The pages give fixed-length spectral coefficients
+ *   and a recent window of the current sequence; they do not say how the cache is kept
+ *   while decoding. This is the reading the library takes.)
+ *
  * Hybrid cache layout (element offsets; F and E bf16, C fp32):
- *   F (sink + recent rows, all dims): [B][Hkv][S + R][128]; row i < S is token i, row
- *     S + i is token L - R + i.
- *   E (middle rows, retained dims): element (b, g, t, i) of middle token t and retained
+ *   F (sink + recent rows, all dims): [B][Hkv][S + R][128]; row i < S is token i, and
+ *     the recent rows form a ring: row S + ((recent_head + i) mod R) is token L - R + i
+ *     (recent_head = 0 until fa_append advances it).
+ *   E (middle rows, retained dims), room for P rows: element (b, g, t, i) of middle
+ *     token t < M and retained
  *     dim i < de_ld[g] sits at b * e_batch + e_off[g] + t * e_pitch[g] + i; columns
  *     [de[g], de_ld[g]) are zero. Two arrangements:
- *     e_token_major = 0: one dense [M][de_ld[g]] block per KV head (e_pitch[g] = de_ld[g],
+ *     e_token_major = 0: one dense [P][de_ld[g]] block per KV head (e_pitch[g] = de_ld[g],
  *       de_ld[g] = de[g] rounded up to a multiple of 8, blocks in KV-head order);
  *     e_token_major = 1: the rows of all KV heads of a batch interleaved per token, so
  *       that token t of batch b is one contiguous row of Hkv * w elements (de_ld[g] = w
@@ -95,13 +106,15 @@ typedef struct fa_shape {
  *     2^-8 relative to every reconstructed value.
  * dc_ld is dc rounded up to a multiple of 8 (rows of 32 bytes).
  *
- * Basis table (fa_build_basis) row stride: phi_ld = M rounded up to a multiple of 8.
+ * Basis table (fa_build_basis) row stride: phi_ld = P rounded up to a multiple of 8.
  */
 typedef struct fa_plan {
   fa_shape shape;
   int32_t S, R, M, kk, G;
   int32_t phi_ld;
   int32_t e_token_major;
+  int32_t P;           /* basis period, P >= M (P = M = 0 without a middle span) */
+  int32_t recent_head; /* ring position of the oldest recent row, 0 <= recent_head < max(R, 1) */
   int32_t dc[FA_MAX_KV_HEADS], de[FA_MAX_KV_HEADS];
   int32_t dc_ld[FA_MAX_KV_HEADS], de_ld[FA_MAX_KV_HEADS];
   int32_t e_pitch[FA_MAX_KV_HEADS];
@@ -137,6 +150,19 @@ typedef struct fa_cache {
 int fa_plan_init(const fa_shape* shape, const uint8_t* dim_mask, fa_plan* plan);
 
 /*
+ * fa_plan_reserve -- make room in a plan for tokens appended while decoding (fa_append).
+ *   plan   host, in/out: a plan from fa_plan_init with a middle span (M >= 1) and nothing
+ *          reserved or appended yet (P == M). On success P = L_max - S - R, phi_ld and
+ *          every layout field are re-derived (E holds P rows per KV head), and the plan
+ *          accepts up to L_max - L calls of fa_append. Call it before allocating the
+ *          cache and before fa_build_basis / fa_compress, which then use period P.
+ *   L_max  largest sequence length the cache will hold, L <= L_max, L_max - S - R < 2^21.
+ * Returns FA_ERR_INVALID (bad plan or L_max) or FA_ERR_UNSUPPORTED (no middle span, or a
+ * plan already reserved / appended to). Pure host function.
+ */
+int fa_plan_reserve(fa_plan* plan, int32_t L_max);
+
+/*
  * fa_build_basis -- the orthonormal real Fourier basis over a span of M tokens, transposed.
  * ([abstract] "orthogonal Fourier bases"; [skill] Step 2 keeps the leading spectral
  * terms of a real FFT along the sequence.)
@@ -158,12 +184,14 @@ int fa_build_basis(int32_t M, int32_t k, int32_t dtype, int32_t normalized, void
 /*
  * fa_compress -- prefill compression of one layer ([skill] Steps 2-3; [abstract]).
  *   K, V   device bf16 [B][Hkv][L][128], the full-precision cache (read only).
- *   phiT   device bf16 [k][plan->phi_ld] from fa_build_basis(M, k, FA_BF16, 0, ...) (the
- *          unscaled table); may be NULL only when M == 0.
+ *   phiT   device bf16 [k][plan->phi_ld] from fa_build_basis(P, k, FA_BF16, 0, ...) (the
+ *          unscaled table of period P; columns t < M are read); may be NULL only when
+ *          M == 0.
  *   cache  host struct of device output buffers (see fa_plan for layouts); written:
  *          F = sink/recent rows, E = retained dims of the middle (bit-exact copies),
  *          C = Phi^T X[S:S+M, compressed dims], fp32 (bf16 x bf16 products accumulated in
- *          fp32 on the tensor cores, then scaled by the orthonormal factor of each row).
+ *          fp32 on the tensor cores, then scaled by the orthonormal factor of each row);
+ *          the recent rows go to F in the ring order of plan->recent_head.
  * The projection runs on the tcgen05 tensor cores (TMA-fed, accumulator in TMEM).
  * Requires bf16 values to be finite (a non-finite recent-token value meets a zero basis
  * entry in the ragged last K tile).
@@ -191,7 +219,8 @@ size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits);
  * softmax across split-L partitions merged by a combine pass. The result equals softmax
  * attention over the reconstructed cache (Phi C on the compressed dims of the middle).
  *   workspace  device scratch of at least fa_decode_workspace_size(plan, num_splits) bytes.
- * Requires k <= FA_MAX_K_DECODE and M < 2^21 tokens.
+ * The basis of the middle span has period P (fa_plan_reserve); tokens t < M are read.
+ * Requires k <= FA_MAX_K_DECODE and P < 2^21 tokens.
  */
 int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
               int32_t out_dtype, void* workspace, size_t workspace_bytes, int32_t num_splits,
@@ -223,6 +252,29 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
 #define FA_NOALLOC_SCRATCH_BYTES (16u << 20)
 int fa_decode_noalloc(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
                       int32_t out_dtype, int32_t num_splits, void* stream);
+
+/*
+ * fa_append -- add one token to every sequence of a compressed cache while decoding
+ * (decode-time cache maintenance). The pages keep a recent window of the current
+ * sequence ([skill] Step 3) and fixed-length spectral coefficients for the middle
+ * ([abstract] method details); this entry point keeps both as the sequence grows.
+ *   plan    host, in/out: a plan with room left (M < P, see fa_plan_reserve). On success
+ *           the plan describes the longer sequence: L and M grow by 1 and recent_head
+ *           advances by one ring position (when R > 0).
+ *   k_new, v_new  device bf16 [B][Hkv][128]: the key and value of the new token L.
+ *   cache   the hybrid cache written by fa_compress / fa_append under this plan.
+ * Per (b, g): the oldest recent token x (the new token itself when R == 0) leaves the
+ * recent window and becomes middle token t = M: its retained dims are written to E row t
+ * (padding columns zero) and its compressed dims are folded into the coefficients,
+ * C_j += phi_j(t) x_c for every j < k (the rank-1 update that extends the projection by
+ * one token under the fixed period P, fp32). The new token takes the freed ring row.
+ * The result equals fa_compress of the longer sequence with the same period, up to fp32
+ * rounding of the coefficients (E and F are bit-exact).
+ * Returns FA_ERR_UNSUPPORTED when no room is left (M == P) or the plan has no middle
+ * span; argument errors as for the other entry points. Launches one kernel.
+ */
+int fa_append(fa_plan* plan, const void* k_new, const void* v_new, const fa_cache* cache,
+              void* stream);
 
 /*
  * fa_device_status -- synchronise `stream`, then read and clear the library's kernel

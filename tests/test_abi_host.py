@@ -251,3 +251,63 @@ def test_hand_edited_layout_is_rejected():
         cache = fa.fa_cache(*([0x1000] * 6))
         rc = fa.LIB.fa_compress(ctypes.byref(q), 0x1000, 0x1000, 0x1000, ctypes.byref(cache), None)
         assert rc == fa.FA_ERR_INVALID and "layout" in fa.fa_last_error(), field
+
+
+# ----------------------------------------------------------------------------- append (host side)
+
+def test_reserve_sets_period_and_sizes_e_by_capacity():
+    w = wl.llama3_8b_layer(2, 4096, 3)
+    m = wl.dim_mask(w)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, m)
+    assert p.P == p.M and p.recent_head == 0
+    e0, c0, f0 = p.e_elems, p.c_elems, p.f_elems
+    fa.fa_plan_reserve(p, w.L + 1000)
+    assert p.P == p.M + 1000 and p.phi_ld == (p.P + 7) // 8 * 8
+    assert p.c_elems == c0 and p.f_elems == f0          # k coefficients and S + R rows: fixed
+    assert p.e_elems * p.M == e0 * p.P                  # E holds P rows per KV head
+    # the layout choice does not depend on the period
+    q = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, m)
+    assert p.e_token_major == q.e_token_major and list(p.de_ld) == list(q.de_ld)
+    assert fa.fa_decode_workspace_size(p, 4) > 0
+
+
+def test_reserve_and_append_rejections():
+    m = np.ones((1, 128))
+    p = fa.fa_plan_init(1, 4, 1, 300, 32, 64, 31, m)
+    for L_max in (299, 32 + 64 + (1 << 21)):
+        with pytest.raises(fa.FaError) as e:
+            fa.fa_plan_reserve(fa.fa_plan.from_buffer_copy(p), L_max)
+        assert e.value.code == fa.FA_ERR_INVALID
+    q = fa.fa_plan.from_buffer_copy(p)
+    fa.fa_plan_reserve(q, 400)
+    with pytest.raises(fa.FaError) as e:                 # reserved twice
+        fa.fa_plan_reserve(q, 500)
+    assert e.value.code == fa.FA_ERR_UNSUPPORTED
+    with pytest.raises(fa.FaError) as e:                 # no middle span
+        fa.fa_plan_reserve(fa.fa_plan_init(1, 4, 1, 90, 32, 64, 31, m), 400)
+    assert e.value.code == fa.FA_ERR_UNSUPPORTED
+    cache = fa.fa_cache(*([0x1000] * 6))
+    lib = fa.LIB
+    # no room: P == M (a plan straight from fa_plan_init); nothing is launched
+    r = lib.fa_append(ctypes.byref(p), 0x1000, 0x1000, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_UNSUPPORTED and "room" in fa.fa_last_error()
+    assert p.M == 204 and p.shape.L == 300
+    r = lib.fa_append(ctypes.byref(q), None, 0x1000, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_INVALID and "k_new" in fa.fa_last_error()
+    r = lib.fa_append(ctypes.byref(q), 0x1000, 0x1008, ctypes.byref(cache), None)
+    assert r == fa.FA_ERR_INVALID and "aligned" in fa.fa_last_error()
+    assert q.M == 204 and q.recent_head == 0            # failed calls leave the plan alone
+
+
+def test_hand_edited_period_or_ring_is_rejected():
+    m = np.ones((1, 128))
+    p = fa.fa_plan_init(1, 4, 1, 300, 32, 64, 31, m)
+    fa.fa_plan_reserve(p, 400)
+    cache = fa.fa_cache(*([0x1000] * 6))
+    for field, value, word in (("P", 200, "period"), ("recent_head", 64, "recent_head"),
+                               ("recent_head", -1, "recent_head"), ("phi_ld", 208, "phi_ld")):
+        q = fa.fa_plan.from_buffer_copy(p)
+        setattr(q, field, value)
+        rc = fa.LIB.fa_compress(ctypes.byref(q), 0x1000, 0x1000, 0x1000, ctypes.byref(cache), None)
+        assert rc == fa.FA_ERR_INVALID and word in fa.fa_last_error(), field
+        assert fa.LIB.fa_decode_workspace_size(ctypes.byref(q), 1) == 0
