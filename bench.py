@@ -530,9 +530,20 @@ def time_append(w, plan, K, V, stream):
     for _ in range(3):
         app()
     nbytes = append_bytes(pa)
-    ms = _time(app, APPEND_STEPS, stream)
+    # each append timed alone after a 256 MB read that evicts the 126 MB L2 with clean lines,
+    # as in a decode loop where the attention step streams the cache between two appends
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=K.device)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(APPEND_STEPS)]
+    for a, b in evs:
+        flush.sum()
+        a.record(stream)
+        app()
+        b.record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in evs) / APPEND_STEPS
     fa.fa_device_status(stream)
-    del cache, phiT
+    del cache, phiT, flush
     torch.cuda.empty_cache()
     return ms, nbytes
 

@@ -44,13 +44,15 @@ def decode(p, cache, q, num_splits=0):
     return out
 
 
-def run_append(w, n_app, extra, mask=None, heads=None, num_splits=0):
+def run_append(w, n_app, extra, mask=None, heads=None, num_splits=0, gen_device="cpu"):
     """Compress the first w.L tokens into a cache with room for n_app + extra more, append
-    n_app tokens one by one, then check every part of the cache and a decode step."""
+    n_app tokens one by one, then check every part of the cache (of the sampled heads) and
+    a decode step."""
     mask = wl.dim_mask(w) if mask is None else mask
     L1 = w.L + n_app
     wf = dataclasses.replace(w, L=L1)
-    K, V, q = wl.kv_cache(wf, "K"), wl.kv_cache(wf, "V"), wl.queries(w)
+    K, V = wl.kv_cache(wf, "K", device=gen_device), wl.kv_cache(wf, "V", device=gen_device)
+    q = wl.queries(w)
     Kd, Vd = K.cuda(), V.cuda()
     p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
     M0 = p.M
@@ -71,7 +73,7 @@ def run_append(w, n_app, extra, mask=None, heads=None, num_splits=0):
     for b, g in pairs:
         cd, ed = fa.perm_lists(p, g)
         hyb = {}
-        for which, X in (("K", K[b, g]), ("V", V[b, g])):
+        for which, X in (("K", K[b, g].cpu()), ("V", V[b, g].cpu())):
             ref = fo.compress(X.double().numpy(), mask[g], w.S, w.R, w.k, period=P)
             hyb[which] = ref
             F = ring_in_token_order(cache.F(which)[b, g].cpu(), p)
@@ -159,3 +161,13 @@ def test_append_until_full_then_refused():
         fa.fa_append(p, x, x, cache)
     assert e.value.code == fa.FA_ERR_UNSUPPORTED
     fa.fa_device_status()
+
+
+@pytest.mark.parametrize("w", [wl.LLAMA2_7B_MHA_32K, wl.LLAMA3_8B_GQA_128K], ids=lambda w: w.name)
+def test_append_full_size_sampled_heads(w):
+    """The bench-sized caches (tensor-core and warp-MMA decode paths): 16 appends, then the
+    first and last (batch, KV head) against the oracle of the longer sequence."""
+    p, cache, K, V = run_append(w, 16, 8, heads=[(0, 0), (w.B - 1, w.Hkv - 1)], gen_device="cuda")
+    assert p.M == w.L - w.S - w.R + 16
+    idx = [p.S + (p.recent_head + a) % p.R for a in range(p.R)]
+    assert torch.equal(cache.F("K")[:, :, idx], K[:, :, p.shape.L - p.R:])
