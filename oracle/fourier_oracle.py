@@ -38,6 +38,12 @@ Readings of points the pages leave open (each is listed in the design notes):
   that the spectral coefficients have a fixed length; they do not say how the cache is
   maintained while decoding.
 
+* Dimension analysis ([skill] Step 1, ``analyze_head_dimensions``): each head dim d in
+  turn gets 0.1 * N(0, 1) noise added to the VALUES of every token, and its sensitivity
+  is the Frobenius norm of the change of the attention output. Scores are kept per KV
+  head (the masks are per KV head), over all batch rows and the query heads of the group.
+  The noise draws are an input. The dims with the lowest scores are the ones compressed.
+
 Parity status: every function below is pinned by ``tests/test_oracle_pins.py``
 (closed forms, library FFT equality, orthonormality, Parseval, brute force).
 """
@@ -57,6 +63,9 @@ __all__ = [
     "reconstruct",
     "attention",
     "decode",
+    "NOISE_SCALE",
+    "dim_sensitivity",
+    "select_dims",
 ]
 
 
@@ -224,3 +233,44 @@ def decode(q, hk: Hybrid, hv: Hybrid, scale: float | None = None) -> np.ndarray:
     if scale is None:
         scale = 1.0 / np.sqrt(D)
     return attention(q, reconstruct(hk), reconstruct(hv), scale)
+
+
+NOISE_SCALE = 0.1
+
+
+def dim_sensitivity(q, K, V, noise, scale: float | None = None) -> np.ndarray:
+    """Sensitivity score of every head dim of one KV head ([skill] Step 1).
+
+    q [B, G, D] (the query heads of the group in every batch row), K, V, noise [B, L, D].
+    For each dim d, as the page's loop does: the unperturbed output, the output with
+    V[:, :, d] += NOISE_SCALE * noise[:, :, d], and the norm of their difference over
+    every batch row, query head and dim. Returns [D] (fp64).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    noise = np.asarray(noise, dtype=np.float64)
+    B, _, D = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    base = np.stack([attention(q[b], K[b], V[b], scale) for b in range(B)])
+    out = np.empty(D)
+    for d in range(D):
+        Vn = V.copy()
+        Vn[:, :, d] += NOISE_SCALE * noise[:, :, d]
+        noisy = np.stack([attention(q[b], K[b], Vn[b], scale) for b in range(B)])
+        out[d] = np.linalg.norm(base - noisy)
+    return out
+
+
+def select_dims(scores, n_compressed: int) -> np.ndarray:
+    """Mask row of one KV head: the n_compressed dims with the lowest sensitivity are
+    compressed (1), the rest retained (0) ([skill] Step 1: low-sensitivity dims are the
+    compression candidates). Equal scores are ranked by dim index (stable order)."""
+    scores = np.asarray(scores, dtype=np.float64)
+    if not 0 <= n_compressed <= scores.size:
+        raise ValueError("n_compressed out of range")
+    order = np.argsort(scores, kind="stable")
+    mask = np.zeros(scores.size, dtype=np.uint8)
+    mask[order[:n_compressed]] = 1
+    return mask

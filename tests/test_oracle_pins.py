@@ -367,3 +367,68 @@ def test_pins_reject_planted_mistakes(kind):
               or check_rfft_bins(fn, 4099, 255, rng) > TOL
               or check_truncated_irfft(fn, 4099, 100, rng) > TOL)
     assert caught, kind
+
+
+# ----------------------------------------------------------------------------- dim analysis
+
+def _sens_case(seed, B=2, G=3, L=50, D=128):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((B, G, D)), rng.standard_normal((B, L, D)),
+            rng.standard_normal((B, L, D)), rng.standard_normal((B, L, D)))
+
+
+def test_sensitivity_equals_weighted_noise_closed_form():
+    """Only V changes, so by linearity the output change of dim d is 0.1 * P n_d with P the
+    (unchanged) softmax weights: written here with torch's softmax, not the oracle's."""
+    q, K, V, n = _sens_case(1)
+    s = fo.dim_sensitivity(q, K, V, n)
+    qt, Kt, nt = (torch.from_numpy(x) for x in (q, K, n))
+    P = torch.softmax(qt @ Kt.transpose(1, 2) / np.sqrt(128), dim=-1)     # [B, G, L]
+    ref = 0.1 * torch.linalg.vector_norm(P @ nt, dim=(0, 1)).numpy()      # [D]
+    assert np.abs(s - ref).max() < 1e-12 * ref.max()
+
+
+def test_sensitivity_hand_case():
+    """One token: softmax weight 1, so the change is exactly 0.1 * noise of that token."""
+    q, K, V, n = _sens_case(2, B=1, G=2, L=1)
+    s = fo.dim_sensitivity(q, K, V, n)
+    assert np.abs(s - 0.1 * np.sqrt(2) * np.abs(n[0, 0])).max() < 1e-15
+
+
+def test_sensitivity_ignores_values_and_zero_noise():
+    q, K, V, n = _sens_case(3)
+    a = fo.dim_sensitivity(q, K, V, n)
+    assert np.abs(a - fo.dim_sensitivity(q, K, 5 * V + 3, n)).max() < 1e-12 * a.max()
+    n[:, :, 7] = 0
+    assert fo.dim_sensitivity(q, K, V, n)[7] < 1e-15
+
+
+def test_select_dims_brute_force():
+    rng = np.random.default_rng(4)
+    for _ in range(50):
+        sc = rng.integers(0, 6, size=12).astype(float)       # many ties
+        nc = int(rng.integers(0, 13))
+        m = fo.select_dims(sc, nc)
+        assert m.sum() == nc
+        # every compressed dim ranks below every retained one in (score, index) order
+        key = [(sc[i], i) for i in range(12)]
+        if 0 < nc < 12:
+            assert max(key[i] for i in range(12) if m[i]) < min(key[i] for i in range(12) if not m[i])
+
+
+def test_sensitivity_pin_rejects_planted_mistakes():
+    q, K, V, n = _sens_case(5)
+    qt, Kt, nt = (torch.from_numpy(x) for x in (q, K, n))
+    P = torch.softmax(qt @ Kt.transpose(1, 2) / np.sqrt(128), dim=-1)
+    ref = 0.1 * torch.linalg.vector_norm(P @ nt, dim=(0, 1)).numpy()
+    good = fo.dim_sensitivity(q, K, V, n)
+    # perturbing the keys instead, or dropping the 0.1 scale, is caught by the closed form
+    keys = np.empty(128)
+    base = np.stack([fo.attention(q[b], K[b], V[b], 1 / np.sqrt(128)) for b in range(2)])
+    for d in range(128):
+        Kn = K.copy()
+        Kn[:, :, d] += 0.1 * n[:, :, d]
+        keys[d] = np.linalg.norm(base - np.stack([fo.attention(q[b], Kn[b], V[b], 1 / np.sqrt(128))
+                                                  for b in range(2)]))
+    for wrong in (keys, good / 0.1):
+        assert np.abs(wrong - ref).max() > 1e-6 * ref.max()
