@@ -548,6 +548,27 @@ def time_append(w, plan, K, V, stream):
     return ms, nbytes
 
 
+def time_sensitivity(w, K, q, stream):
+    """Device time of one fa_dim_sensitivity over the workload's keys and a seeded noise
+    tensor of the same shape; returns (ms, algorithmic bytes: K and noise read once)."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+    noise = wl.value_noise(w, device=K.device)
+    ws = torch.empty(fa.fa_dim_sensitivity_workspace_size(w.B, w.Hq, w.Hkv, w.L),
+                     dtype=torch.uint8, device=K.device)
+    scores = torch.empty(w.Hkv, 128, dtype=torch.float32, device=K.device)
+    run = lambda: fa.fa_dim_sensitivity(q, K, noise, scores, ws, stream)
+    for _ in range(2):
+        run()
+    ms = _time(run, 5, stream)
+    fa.fa_device_status(stream)
+    del noise, ws, scores
+    torch.cuda.empty_cache()
+    return ms, 2 * K_bytes(w)
+
+
 def run_sweep(args):
     """Per-workload timings (1 GPU): the four single-layer workloads, then the 32-layer
     LLaMA-3-8B-shaped cache: compress every layer (distinct seeded masks), and time one
@@ -585,6 +606,7 @@ def run_sweep(args):
         fa.fa_device_status(stream)
         del cache, ws
         ta, a_bytes = time_append(w, plan, K, V, stream)
+        tsens, s_bytes = time_sensitivity(w, K, q, stream)
         wm = work_model(w, plan)
         print(json.dumps({"sweep": "single_layer", "workload": w.name, "basis_us": tb * 1e3,
                           "compress_us": tcmp * 1e3,
@@ -598,7 +620,9 @@ def run_sweep(args):
                           "decode_frac_hbm": wm["decode_bytes"] / td / 1e6 / hbm,
                           "decode_fp32_tflops": wm["decode_flops"] / td / 1e9,
                           "append_us": ta * 1e3, "append_hbm_gbs": a_bytes / ta / 1e6,
-                          "append_frac_hbm": a_bytes / ta / 1e6 / hbm}), flush=True)
+                          "append_frac_hbm": a_bytes / ta / 1e6 / hbm,
+                          "sensitivity_us": tsens * 1e3, "sensitivity_hbm_gbs": s_bytes / tsens / 1e6,
+                          "sensitivity_frac_hbm": s_bytes / tsens / 1e6 / hbm}), flush=True)
         del K, V, out, phiT
         torch.cuda.empty_cache()
 

@@ -5,7 +5,8 @@ Argument marshalling only: every step of the hot path runs in the CUDA kernels o
 PyTorch is used for device memory and streams. The functions keep the C names:
 
     fa_plan_init, fa_plan_reserve, fa_build_basis, fa_compress, fa_decode_workspace_size,
-    fa_decode, fa_decode_noalloc, fa_append, fa_device_status, fa_last_error
+    fa_decode, fa_decode_noalloc, fa_append, fa_dim_sensitivity_workspace_size,
+    fa_dim_sensitivity, fa_select_dims, fa_device_status, fa_last_error
 
 There is no CPU fallback: if the shared library is missing or fails to load, importing
 this package raises.
@@ -27,7 +28,9 @@ FA_BF16, FA_F32 = 0, 1
 
 EXPORTED = ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress",
             "fa_decode_workspace_size", "fa_decode", "fa_decode_noalloc", "fa_append",
+            "fa_dim_sensitivity_workspace_size", "fa_dim_sensitivity", "fa_select_dims",
             "fa_device_status", "fa_watchdog_selftest", "fa_last_error")
+NOISE_SCALE = 0.1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -80,6 +83,10 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_plan_reserve.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_build_basis.argtypes = [I32, I32, I32, I32, P, I64, P]
     lib.fa_append.argtypes = [ctypes.POINTER(fa_plan), P, P, ctypes.POINTER(fa_cache), P]
+    lib.fa_dim_sensitivity_workspace_size.argtypes = [ctypes.POINTER(fa_shape)]
+    lib.fa_dim_sensitivity_workspace_size.restype = SZ
+    lib.fa_dim_sensitivity.argtypes = [ctypes.POINTER(fa_shape), P, P, P, P, P, SZ, P]
+    lib.fa_select_dims.argtypes = [P, I32, I32, P]
     lib.fa_compress.argtypes = [ctypes.POINTER(fa_plan), P, P, P, ctypes.POINTER(fa_cache), P]
     lib.fa_decode_workspace_size.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_decode_workspace_size.restype = SZ
@@ -92,7 +99,8 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_last_error.argtypes = []
     lib.fa_last_error.restype = ctypes.c_char_p
     for name in ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress", "fa_decode",
-                 "fa_decode_noalloc", "fa_append", "fa_device_status", "fa_watchdog_selftest"):
+                 "fa_decode_noalloc", "fa_append", "fa_dim_sensitivity", "fa_select_dims",
+                 "fa_device_status", "fa_watchdog_selftest"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -187,6 +195,29 @@ def fa_append(plan: fa_plan, k_new, v_new, cache: "Cache", stream=None) -> None:
     """Append one token per sequence (k_new, v_new: bf16 [B, Hkv, 128]); advances ``plan``."""
     _check(LIB.fa_append(ctypes.byref(plan), _ptr(k_new), _ptr(v_new), ctypes.byref(cache.c),
                          _stream(stream)))
+
+
+def fa_dim_sensitivity_workspace_size(B, Hq, Hkv, L) -> int:
+    return LIB.fa_dim_sensitivity_workspace_size(ctypes.byref(fa_shape(B, Hq, Hkv, HEAD_DIM, L, 0, 0, 1)))
+
+
+def fa_dim_sensitivity(q, K, noise, scores, workspace, stream=None) -> None:
+    """Sensitivity scores [Hkv, 128] (fp32, device) of every head dim under value noise.
+    q: bf16 [B, Hq, 128]; K, noise: bf16 [B, Hkv, L, 128]."""
+    B, Hkv, L, D = K.shape
+    shape = fa_shape(B, q.shape[1], Hkv, D, L, 0, 0, 1)
+    _check(LIB.fa_dim_sensitivity(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(noise), _ptr(scores),
+                                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                  _stream(stream)))
+
+
+def fa_select_dims(scores, n_compressed: int) -> np.ndarray:
+    """Host: uint8 mask [Hkv, 128] compressing the n_compressed lowest-score dims per KV head."""
+    sc = np.ascontiguousarray(np.asarray(scores, dtype=np.float32))
+    Hkv = sc.shape[0]
+    mask = np.zeros((Hkv, HEAD_DIM), dtype=np.uint8)
+    _check(LIB.fa_select_dims(sc.ctypes.data, Hkv, int(n_compressed), mask.ctypes.data))
+    return mask
 
 
 def fa_device_status(stream=None) -> None:

@@ -288,6 +288,66 @@ int fa_append(fa_plan* plan, const void* k_new, const void* v_new, const fa_cach
   return FA_OK;
 }
 
+static int sensitivity_setup(const fa_shape* shape, fa_plan* plan, fa::DecodeConfig* c,
+                             size_t* bytes) {
+  if (!shape) return fail(FA_ERR_INVALID, "shape is NULL");
+  if (int r = fa::sensitivity_plan(shape, plan)) return r;  // fa_plan_init set the message
+  if (int r = decode_checks(plan)) return r;
+  cudaError_t e = fa::decode_configure(plan, 0, c);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_dim_sensitivity: configure");
+  *bytes = fa::sensitivity_out_offset(*c) +
+           (size_t)plan->shape.B * plan->shape.Hq * FA_HEAD_DIM * sizeof(float);
+  return FA_OK;
+}
+
+size_t fa_dim_sensitivity_workspace_size(const fa_shape* shape) {
+  fa_plan plan;
+  fa::DecodeConfig c;
+  size_t bytes = 0;
+  return sensitivity_setup(shape, &plan, &c, &bytes) == FA_OK ? bytes : 0;
+}
+
+int fa_dim_sensitivity(const fa_shape* shape, const void* q, const void* K, const void* noise,
+                       float* scores, void* workspace, size_t workspace_bytes, void* stream) {
+  fa_plan plan;
+  fa::DecodeConfig c;
+  size_t need = 0;
+  if (int r = sensitivity_setup(shape, &plan, &c, &need)) return r;
+  if (int r = check_ptr(q, "q", true)) return r;
+  if (int r = check_ptr(K, "K", true)) return r;
+  if (int r = check_ptr(noise, "noise", true)) return r;
+  if (int r = check_ptr(scores, "scores", true)) return r;
+  if (int r = check_ptr(workspace, "workspace", true)) return r;
+  if (workspace_bytes < need)
+    return fail(FA_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                workspace_bytes, need);
+  cudaError_t e = fa::launch_sensitivity(&plan, c, q, K, noise, scores, workspace,
+                                         static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_dim_sensitivity: launch");
+  return FA_OK;
+}
+
+int fa_select_dims(const float* scores, int32_t Hkv, int32_t n_compressed, uint8_t* mask_out) {
+  if (!scores || !mask_out) return fail(FA_ERR_INVALID, "NULL argument");
+  if (Hkv < 1 || Hkv > FA_MAX_KV_HEADS || n_compressed < 0 || n_compressed > FA_HEAD_DIM)
+    return fail(FA_ERR_INVALID, "Hkv=%d or n_compressed=%d out of range", Hkv, n_compressed);
+  for (int g = 0; g < Hkv; ++g) {
+    const float* sc = scores + g * FA_HEAD_DIM;
+    for (int d = 0; d < FA_HEAD_DIM; ++d) {
+      // rank of d in (score, index) order; NaN scores rank last
+      int rank = 0;
+      const bool dn = sc[d] != sc[d];
+      for (int e = 0; e < FA_HEAD_DIM; ++e) {
+        const bool en = sc[e] != sc[e];
+        const bool before = (en != dn) ? dn : (dn ? e < d : (sc[e] < sc[d] || (sc[e] == sc[d] && e < d)));
+        rank += before ? 1 : 0;
+      }
+      mask_out[g * FA_HEAD_DIM + d] = rank < n_compressed ? 1 : 0;
+    }
+  }
+  return FA_OK;
+}
+
 int fa_watchdog_selftest(uint32_t wait_ns, void* stream) {
   if (wait_ns < 1000u || wait_ns > 1000000000u)
     return fail(FA_ERR_INVALID, "wait_ns=%u outside [1 us, 1 s]", wait_ns);

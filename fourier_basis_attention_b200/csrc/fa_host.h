@@ -28,6 +28,11 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
                           cudaStream_t stream);
 cudaError_t launch_append(const fa_plan* plan, const void* k_new, const void* v_new,
                           const fa_cache* cache, cudaStream_t stream);
+int sensitivity_plan(const fa_shape* shape, fa_plan* plan);  // fa_status code
+size_t sensitivity_out_offset(const DecodeConfig& c);
+cudaError_t launch_sensitivity(const fa_plan* plan, const DecodeConfig& c, const void* q,
+                               const void* K, const void* noise, float* scores, void* workspace,
+                               cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
 cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream);
 

@@ -277,6 +277,40 @@ int fa_append(fa_plan* plan, const void* k_new, const void* v_new, const fa_cach
               void* stream);
 
 /*
+ * fa_dim_sensitivity -- head-dimension sensitivity scores, for choosing the dim mask of
+ * fa_plan_init ([skill] Step 1 and "Architecture overview": a noise-perturbation analysis
+ * finds the dims that must stay exact; the dims least sensitive to noise are compressed).
+ *   shape   host; B, Hq, Hkv, D = 128 and L are used (S, R, k are ignored).
+ *           Hq / Hkv in {1, 2, 4, 8}.
+ *   q       device bf16 [B][Hq][128]: the probe queries.
+ *   K       device bf16 [B][Hkv][L][128]: the keys (full precision, the layout of fa_compress).
+ *   noise   device bf16 [B][Hkv][L][128]: N(0, 1) draws, one per token and dim (the
+ *           caller's random numbers).
+ *   scores  device fp32 [Hkv][128], written: scores[g][d] is the Frobenius norm, over every
+ *           batch row, every query head of KV head g and every output dim, of the change of
+ *           softmax attention (scale 1/sqrt(128)) when value dim d of every token of KV head
+ *           g gets FA_NOISE_SCALE * noise added.
+ * Only the values change, so the output change is FA_NOISE_SCALE * P n_d with P the
+ * attention weights: the library runs one exact attention pass over (K, noise) and takes
+ * per-dim norms. The values themselves are not needed and not read.
+ *   workspace  device scratch of at least fa_dim_sensitivity_workspace_size(shape) bytes.
+ * Returns 0 from the size query for unusable shapes.
+ */
+#define FA_NOISE_SCALE 0.1f
+size_t fa_dim_sensitivity_workspace_size(const fa_shape* shape);
+int fa_dim_sensitivity(const fa_shape* shape, const void* q, const void* K, const void* noise,
+                       float* scores, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_select_dims -- host: the dim mask from sensitivity scores. For each KV head g the
+ * n_compressed dims with the lowest scores[g][*] are marked compressed (1), the others
+ * retained (0); equal scores rank by dim index. scores: host fp32 [Hkv][128]; mask_out:
+ * host uint8 [Hkv][128], the dim_mask argument of fa_plan_init. Requires
+ * 1 <= Hkv <= FA_MAX_KV_HEADS and 0 <= n_compressed <= 128. Pure host function.
+ */
+int fa_select_dims(const float* scores, int32_t Hkv, int32_t n_compressed, uint8_t* mask_out);
+
+/*
  * fa_device_status -- synchronise `stream`, then read and clear the library's kernel
  * watchdog word. Returns FA_OK if no kernel launched since the last call hit a wait
  * limit, FA_ERR_DEVICE (message names the kernel and wait) if one did, FA_ERR_CUDA if

@@ -311,3 +311,30 @@ def test_hand_edited_period_or_ring_is_rejected():
         rc = fa.LIB.fa_compress(ctypes.byref(q), 0x1000, 0x1000, 0x1000, ctypes.byref(cache), None)
         assert rc == fa.FA_ERR_INVALID and word in fa.fa_last_error(), field
         assert fa.LIB.fa_decode_workspace_size(ctypes.byref(q), 1) == 0
+
+
+# ----------------------------------------------------------------------------- dim selection
+
+def test_select_dims_matches_oracle():
+    rng = np.random.default_rng(11)
+    for trial in range(20):
+        Hkv = int(rng.integers(1, 9))
+        sc = rng.integers(0, 40, size=(Hkv, 128)).astype(np.float32)   # ties
+        if trial % 5 == 0:
+            sc[0, rng.integers(0, 128, 3)] = np.nan
+        nc = int(rng.integers(0, 129))
+        got = fa.fa_select_dims(sc, nc)
+        for g in range(Hkv):
+            assert np.array_equal(got[g], fo.select_dims(sc[g].astype(np.float64), nc)), (trial, g)
+
+
+def test_select_dims_rejections():
+    with pytest.raises(fa.FaError):
+        fa.fa_select_dims(np.zeros((2, 128)), 129)
+    with pytest.raises(fa.FaError):
+        fa.fa_select_dims(np.zeros((65, 128)), 3)
+    shape = fa.fa_shape(1, 3, 1, 128, 100, 0, 0, 1)          # G = 3: no decode kernel
+    assert fa.LIB.fa_dim_sensitivity_workspace_size(ctypes.byref(shape)) == 0
+    r = fa.LIB.fa_dim_sensitivity(ctypes.byref(shape), 0x1000, 0x1000, 0x1000, 0x1000, 0x1000,
+                                  1 << 20, None)
+    assert r == fa.FA_ERR_UNSUPPORTED

@@ -169,3 +169,9 @@ def queries(w: Workload, device="cpu") -> torch.Tensor:
     """bf16 [B, Hq, D] decode queries, N(0, 1)."""
     gen = _gen(device, (w.seed * 1_000_003 + 424_242) & 0x7FFFFFFF)
     return torch.randn(w.B, w.Hq, D, generator=gen, device=device).to(torch.bfloat16)
+
+
+def value_noise(w: Workload, device="cpu") -> torch.Tensor:
+    """bf16 [B, Hkv, L, D] N(0, 1) draws: the noise of the head-dimension analysis."""
+    gen = _gen(device, (w.seed * 1_000_003 + 777_767) & 0x7FFFFFFF)
+    return torch.randn(w.B, w.Hkv, w.L, D, generator=gen, device=device).to(torch.bfloat16)
