@@ -341,3 +341,20 @@ def test_bounded_wait_reports_and_context_survives():
     assert e.value.code == fa.FA_ERR_DEVICE and "kernel 15" in str(e.value)
     fa.fa_device_status()  # cleared
     run_small(wl.shrink(wl.SINGLE_HEAD_2K, L=600))
+
+
+# ----------------------------------------------------------------------------- determinism at scale
+
+def test_compress_many_heads_is_deterministic():
+    """160 (KV head, tile pair) units: more CTAs than SMs; repeated calls write identical bits."""
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=40, Hq=4, Hkv=4, L=2000, k=255)
+    mask = wl.dim_mask(w)
+    K, V = wl.kv_cache(w, "K", device="cuda"), wl.kv_cache(w, "V", device="cuda")
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    phiT = fa.basis_table(p)
+    c1, c2 = fa.Cache(p), fa.Cache(p)
+    fa.fa_compress(p, K, V, phiT, c1)
+    fa.fa_compress(p, K, V, phiT, c2)
+    fa.fa_device_status()
+    assert torch.equal(c1.C_K, c2.C_K) and torch.equal(c1.C_V, c2.C_V)
+    assert torch.equal(c1.E_K, c2.E_K) and torch.equal(c1.E_V, c2.E_V)
