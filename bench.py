@@ -441,16 +441,16 @@ def run_ours(args):
 
 def launches_per_step(w, plan):
     """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel and
-    compress_kernel; then fa_decode's prologue (middle span present), the split kernel (the
-    tensor-core one when the plan laid E out token-major, or the warp-MMA one for other
-    plans with 256 <= k <= 1023, each followed by the CUDA-core kernel for the sink / recent
-    rows; else the CUDA-core one for both), and the combine."""
+    compress_kernel; then fa_decode's prologue (middle span present; on the tensor-core and
+    warp-MMA paths its launch also runs the sink / recent rows), the split kernel (the
+    tensor-core one when the plan laid E out token-major, the warp-MMA one for other plans
+    with 256 <= k <= 1023, else the CUDA-core one, which then also runs the sink / recent
+    rows), and the combine."""
     n = 1 + 2
-    n += 1 if plan.M > 0 else 0          # prologue
+    n += 1 if plan.M > 0 else 0          # prologue (+ sink / recent rows)
     hm = plan.M > 0 and not plan.e_token_major and 256 <= w.k <= 1023
     if (plan.e_token_major or hm) and plan.M > 0:
         n += 1                           # tensor-core or warp-MMA split kernel
-        n += 1 if plan.S + plan.R > 0 else 0  # sink / recent rows (CUDA-core kernel)
     elif plan.M > 0 or plan.S + plan.R > 0:
         n += 1                           # CUDA-core split kernel (+ sink / recent rows)
     return n + 1                         # combine

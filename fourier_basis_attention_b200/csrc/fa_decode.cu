@@ -25,8 +25,15 @@
 namespace fa {
 
 // ------------------------------------------------------------------------- prologue
+// CTAs [0, n_pro): the prologue of one KV head each. CTAs past n_pro (tensor-core and
+// warp-MMA paths): the sink / recent rows, which need only q, so they run beside the prologue
+// instead of in a launch of their own.
 __global__ void __launch_bounds__(DNT) decode_prologue_kernel(const __grid_constant__ DecodeParams p) {
-  extern __shared__ float qc_s[];  // [G][128]
+  extern __shared__ __align__(16) float qc_s[];  // [G][128] (sink / recent CTAs: their buffers)
+  if ((int)blockIdx.x >= p.n_pro) {
+    decode_sink_recent(p, qc_s, (int)blockIdx.x - p.n_pro);
+    return;
+  }
   const int kvh = blockIdx.x;
   const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
   const int dc = p.dc[g], de = p.de[g], dc_ld = p.dc_ld[g];
@@ -482,7 +489,7 @@ __host__ __device__ inline int combine_wts_floats(int G, int nrec) { return (G *
 
 __host__ __device__ inline size_t combine_smem_floats(int G, int nrec, int payload) {
   return (size_t)combine_wts_floats(G, nrec) + 16 + (size_t)G * payload + (size_t)8 * G * 128 +
-         (size_t)CB_KC * FA_HEAD_DIM + 2 * (size_t)G * FA_HEAD_DIM + FA_HEAD_DIM;
+         (size_t)2 * CB_KC * FA_HEAD_DIM + 2 * (size_t)G * FA_HEAD_DIM + FA_HEAD_DIM;
 }
 
 __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
@@ -497,8 +504,8 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
   float* lsum = mst + 8;                    // [8]
   float* sum = lsum + 8;                    // [G][payload] weighted sum of split payloads
   float* red = sum + G * payload;           // [8 warps][G][128] partial column sums
-  float* cvs = red + 8 * G * 128;           // [CB_KC][128] chunk of C_V
-  float* cpart = cvs + CB_KC * FA_HEAD_DIM; // [2][G][128] halves of u C_V
+  float* cvs = red + 8 * G * 128;           // [2][CB_KC][128] chunks of C_V (double buffer)
+  float* cpart = cvs + 2 * CB_KC * FA_HEAD_DIM; // [2][G][128] halves of u C_V
   int* inv = reinterpret_cast<int*>(cpart + 2 * G * FA_HEAD_DIM);  // [128]
   const long long bhq = (long long)p.B * p.Hq;
   const long long gh0 = (long long)b * p.Hq + (long long)g * G;
@@ -506,6 +513,25 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
     return p.rec + ((long long)r * bhq + gh0 + h) * p.rec_stride;
   };
 
+  // C_V does not depend on the split records: its first two CB_KC-row chunks are copied
+  // into shared memory (cp.async) while the records are merged. One commit group per chunk
+  // (empty past the last), so waiting for all but the newest group completes chunk i.
+  const float* CV = p.CV + (long long)b * p.c_batch + p.c_off[g];
+  const bool do_cv = k > 0 && dc > 0 && ns > 0;
+  auto load_cv_chunk = [&](int ci) {
+    const int j0 = ci * CB_KC;
+    if (do_cv && j0 < k) {
+      const int nj = min(CB_KC, k - j0), nq = dc_ld / 4;
+      float* buf = cvs + (ci & 1) * CB_KC * FA_HEAD_DIM;
+      for (int e = tid; e < nj * nq; e += CB_THREADS) {
+        const int jj = e / nq, c4 = e - jj * nq;
+        cp_async16(buf + jj * FA_HEAD_DIM + 4 * c4, CV + (long long)(j0 + jj) * dc_ld + 4 * c4);
+      }
+    }
+    cp_async_commit();
+  };
+  load_cv_chunk(0);
+  load_cv_chunk(1);
   if (tid < FA_HEAD_DIM) inv[p.perm[g][tid]] = tid;
   if (warp < G) {
     const int h = warp;
@@ -535,7 +561,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
 #pragma unroll
     for (int h = 0; h < HL; ++h) a[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     if (col < payload) {
-#pragma unroll 4  // several records' rows in flight per lane
+#pragma unroll 8  // several records' rows in flight per lane
       for (int r = warp; r < ns; r += 8) {
 #pragma unroll
         for (int h = 0; h < HL; ++h) {
@@ -565,34 +591,32 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
     }
     __syncthreads();
   }
-  // out_c = u C_V: C_V rows in chunks through shared memory; thread (half, column i) sums
-  // the rows of its parity
-  const float* CV = p.CV + (long long)b * p.c_batch + p.c_off[g];
+  // out_c = u C_V: C_V rows in double-buffered chunks; thread (half, column i) sums the rows
+  // of its parity
   const int colc = tid & (FA_HEAD_DIM - 1), half = tid >> 7;
   float acc[HL];
 #pragma unroll
   for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
-  for (int j0 = 0; j0 < k && dc > 0 && ns > 0; j0 += CB_KC) {
-    const int nj = min(CB_KC, k - j0);
-    __syncthreads();  // previous chunk consumed (first pass: sum written)
-    for (int e = tid; e < nj * (dc_ld / 4); e += CB_THREADS) {
-      const int jj = e / (dc_ld / 4), c4 = e - jj * (dc_ld / 4);
-      reinterpret_cast<float4*>(cvs + jj * FA_HEAD_DIM)[c4] =
-          reinterpret_cast<const float4*>(CV + (long long)(j0 + jj) * dc_ld)[c4];
-    }
-    __syncthreads();
+  for (int j0 = 0; j0 < k && do_cv; j0 += CB_KC) {
+    const int nj = min(CB_KC, k - j0), ci = j0 / CB_KC;
+    const float* cvb = cvs + (ci & 1) * CB_KC * FA_HEAD_DIM;
+    cp_async_wait<1>();  // this thread's copies of chunk ci have landed
+    __syncthreads();     // everyone's copies (first pass: sum written)
     if (colc < dc) {
       for (int jj = half; jj < nj; jj += 2) {
         const int j = j0 + jj, f = (j + 1) >> 1;
         const int slot = FA_HEAD_DIM + 2 * f + ((j > 0 && (j & 1) == 0) ? 1 : 0);
-        const float cv = cvs[jj * FA_HEAD_DIM + colc] *
+        const float cv = cvb[jj * FA_HEAD_DIM + colc] *
                          ((f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair);
 #pragma unroll
         for (int h = 0; h < HL; ++h)
           if (h < G) acc[h] += sum[h * payload + slot] * cv;
       }
     }
+    __syncthreads();     // chunk ci consumed: its buffer takes chunk ci + 2
+    load_cv_chunk(ci + 2);
   }
+  cp_async_wait<0>();
   __syncthreads();
 #pragma unroll
   for (int h = 0; h < HL; ++h)
@@ -796,28 +820,27 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   p.rec = reinterpret_cast<float*>(static_cast<char*>(workspace) + c.qw_bytes);
 
   cudaError_t e;
+  // On the tensor-core and warp-MMA paths the sink / recent rows run as extra CTAs of the
+  // prologue launch (small CTAs that need only q; the split kernels hold whole SMs).
+  const bool sr_with_prologue = p.M > 0 && (c.tc || c.hm);
   if (p.M > 0) {
-    decode_prologue_kernel<<<n_heads, DNT, plan->G * FA_HEAD_DIM * 4, stream>>>(p);
+    p.n_pro = n_heads;
+    const int pro_grid = n_heads + (sr_with_prologue ? n_heads * c.n_fsplits : 0);
+    size_t pro_smem = (size_t)plan->G * FA_HEAD_DIM * 4;
+    if (sr_with_prologue && sink_recent_smem_bytes() > pro_smem) pro_smem = sink_recent_smem_bytes();
+    decode_prologue_kernel<<<pro_grid, DNT, pro_smem, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // The sink / recent rows run either as extra CTAs of the tensor-core grid or, when
-  // kTcSinkRecentSeparate, in a CUDA-core launch of their own after it (small CTAs, two per
-  // SM, instead of holding a whole SM each).
-  constexpr bool kTcSinkRecentSeparate = true;
   if (c.tc) {
     p.e_row = plan->e_pitch[0];
-    p.tc_nf = kTcSinkRecentSeparate ? 0 : n_heads * c.n_fsplits;
+    p.tc_nf = 0;
     if ((e = launch_decode_tc(p, plan->de_ld[0], stream)) != cudaSuccess) return e;
-    p.n_mid = 0;
   } else if (plan->e_token_major && plan->M > 0) {
     return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only
   } else if (c.hm) {
-    // middle span on warp-level MMAs; the CUDA-core kernel below runs the sink / recent rows
     if ((e = launch_decode_hmma(p, c.hm_F2, stream)) != cudaSuccess) return e;
-    p.n_mid = 0;
   }
-  const int grid = c.tc ? (kTcSinkRecentSeparate ? n_heads * c.n_fsplits : 0)
-                        : p.n_mid + n_heads * c.n_fsplits;
+  const int grid = sr_with_prologue ? 0 : p.n_mid + n_heads * c.n_fsplits;
   if (grid > 0) {
     int occ = 0;
     if (c.SPT == 1) {

@@ -21,6 +21,7 @@ struct DecodeParams {
   int tc_F2, tc_tmem_cols;  // tensor-core split kernel: coefficient slots, TMEM columns
   int e_row;                // token-major E: elements per token row of a batch
   int tc_nf;                // sink / recent CTAs at the front of the tensor-core grid
+  int n_pro;                // prologue CTAs (the sink / recent CTAs of a prologue launch follow)
   float qscale, norm_single, norm_pair, two_over_P;
   long long e_batch, c_batch;
   long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
