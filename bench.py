@@ -214,10 +214,36 @@ def host_pairs(w, n_pairs, seed_shift=0):
     return out
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_workload(base, rank):
+    """Rank r's replica of the workload: the same shapes with its own seed (weak scaling: each
+    rank compresses and decodes its own batch; no data crosses ranks)."""
+    import workloads as wl
+    return wl.shrink(base, seed=base.seed + 1000 * rank) if rank else base
+
+
+def max_over_ranks(values, device=None):
+    """Element-wise max over all ranks of a list of floats (the slowest rank sets every
+    reported time). Every rank must call it, in the same order; one rank: returned as is."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def prints_line(rank):
+    """Only rank 0 prints the JSON line."""
+    return rank == 0
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
-    if rank != 0:
-        return
+    if not prints_line(rank):
+        return  # the reference arm runs on rank 0 alone
     w = workload_by_name(args.workload)
     pairs = host_pairs(w, 1)
     n_units = w.B * w.Hkv
@@ -263,7 +289,7 @@ def run_ours(args):
     base = workload_by_name(args.workload)
     if args.batch > 0:
         base = wl.shrink(base, B=args.batch)
-    w = wl.shrink(base, seed=base.seed + 1000 * rank) if rank else base
+    w = rank_workload(base, rank)
     mask = wl.dim_mask(base)
     dev = torch.device("cuda", local)
     K = wl.kv_cache(w, "K", device=dev)
@@ -333,10 +359,7 @@ def run_ours(args):
     comp_ms = statistics.mean(t_comp)
     dec_ms = statistics.mean(t_dec)
     basis_ms = statistics.mean(t_basis)
-    if world > 1:
-        t = torch.tensor([ms_step, comp_ms, dec_ms, basis_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, comp_ms, dec_ms, basis_ms = t.tolist()
+    ms_step, comp_ms, dec_ms, basis_ms = max_over_ranks([ms_step, comp_ms, dec_ms, basis_ms], dev)
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e_us = None
@@ -367,10 +390,7 @@ def run_ours(args):
         b.record(stream)
         barrier()
         e2e_ms = a.elapsed_time(b) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = t.item()
+        e2e_ms = max_over_ranks([e2e_ms], dev)[0]
         e2e_us = e2e_ms * 1e3
         h2d = Kh.numel() * 2 + Vh.numel() * 2 + qh.numel() * 2
         d2h = oh.numel() * 2
@@ -432,7 +452,7 @@ def run_ours(args):
             "kind": "oracle",
             "sample": f"2 of {n_units} (batch, KV head) pairs (fp64 compress K+V + decode), "
                       f"scaled x{n_units / 2:g}"}
-    if rank == 0:
+    if prints_line(rank):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])
