@@ -833,7 +833,6 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   }
   if (c.tc) {
     p.e_row = plan->e_pitch[0];
-    p.tc_nf = 0;
     if ((e = launch_decode_tc(p, plan->de_ld[0], stream)) != cudaSuccess) return e;
   } else if (plan->e_token_major && plan->M > 0) {
     return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only

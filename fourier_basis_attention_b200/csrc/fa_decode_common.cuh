@@ -1,6 +1,6 @@
 // fa_decode_common.cuh -- parameters and helpers shared by the decode kernels
 // (fa_decode.cu: prologue, CUDA-core split kernel, sink/recent, combine; fa_decode_tc.cu:
-// tensor-core split kernel).
+// tensor-core split kernel; fa_decode_hmma.cu: warp-MMA split kernel).
 #pragma once
 
 #include "fa_host.h"
@@ -20,7 +20,6 @@ struct DecodeParams {
   int NTU, TG, DEC, TGE;
   int tc_F2, tc_tmem_cols;  // tensor-core split kernel: coefficient slots, TMEM columns
   int e_row;                // token-major E: elements per token row of a batch
-  int tc_nf;                // sink / recent CTAs at the front of the tensor-core grid
   int n_pro;                // prologue CTAs (the sink / recent CTAs of a prologue launch follow)
   float qscale, norm_single, norm_pair, two_over_P;
   long long e_batch, c_batch;
@@ -54,7 +53,8 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&x)[8]) {
 // Sink / recent rows of one KV head, rows [fs * FT, fs * FT + FT) of its S + R exact rows
 // (all 128 dims): scores, softmax statistics and values of the G query heads, written as
 // split record n_splits + fs. All DNT threads of the CTA take part; `sm` holds
-// sink_recent_smem_bytes() bytes. Used by both split kernels as extra CTAs.
+// sink_recent_smem_bytes() bytes. Run as extra CTAs of the CUDA-core split kernel, or of the
+// prologue launch on the tensor-core and warp-MMA paths.
 __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float* sm, int fid) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kvh = fid / p.n_fsplits, fs = fid - (fid / p.n_fsplits) * p.n_fsplits;
@@ -187,7 +187,7 @@ cudaError_t launch_decode_hmma(const DecodeParams& p, int F2, cudaStream_t strea
 size_t decode_hmma_smem_bytes(int F2);
 
 // Tensor-core split kernel over token-major E with de_slot = 0, 8, 16 or 32 retained
-// elements per KV head and token (the grid also holds the sink / recent CTAs).
+// elements per KV head and token.
 // bf16 x 8 -> 4 fp32 pairs (element 2i in .x, 2i + 1 in .y) for paired FMAs.
 __device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};

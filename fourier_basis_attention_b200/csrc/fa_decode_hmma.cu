@@ -20,7 +20,7 @@
 //      CTA's KV heads fit in HM_EV_BYTES they are staged into shared memory with cp.async
 //      at the start of the tile, so their loads overlap phases A-E.
 // The split record (m, l, exact-dim values, U) has the layout of the other split kernels,
-// so the same combine merges it. Sink / recent rows run in the CUDA-core kernel.
+// so the same combine merges it. The sink / recent rows run in the prologue launch.
 #include "fa_decode_common.cuh"
 
 namespace fa {

@@ -34,8 +34,7 @@
 // accumulator stays distributed (lane = KV head, chunk, query head) until the record is
 // written. Softmax, P rows, U rescaling and (m, l) are per head lane.
 //
-// CTAs [0, tc_nf) of the grid may run the sink / recent rows on the CUDA cores
-// (decode_sink_recent); otherwise the CUDA-core kernel runs them in a launch of its own.
+// The sink / recent rows run on the CUDA cores as extra CTAs of the prologue launch.
 #include "fa_decode_common.cuh"
 
 namespace fa {
@@ -82,8 +81,7 @@ __host__ __device__ inline TcLayout tc_layout(int F2) {
 size_t decode_tc_smem_bytes(int F2, int de_slot, int G) {
   (void)de_slot;
   (void)G;
-  const size_t b = (size_t)tc_layout(F2).total;
-  return b > sink_recent_smem_bytes() ? b : sink_recent_smem_bytes();
+  return (size_t)tc_layout(F2).total;
 }
 
 __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
@@ -116,12 +114,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int n_f = p.tc_nf;  // sink / recent CTAs come first
-  if ((int)blockIdx.x < n_f) {
-    decode_sink_recent(p, reinterpret_cast<float*>(smem), blockIdx.x);
-    return;
-  }
-  const int cta = blockIdx.x - n_f;
+  const int cta = blockIdx.x;
   const int F2 = p.tc_F2;
   const TcLayout Ly = tc_layout(F2);
   uint8_t* Ws = smem + Ly.w;      // W_hi
@@ -723,7 +716,7 @@ static cudaError_t launch_tc_g(const DecodeParams& p, int grid, int smem, cudaSt
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream) {
   const int smem = (int)decode_tc_smem_bytes(p.tc_F2, de_slot, p.G);
   const int heads = p.B * p.Hq;
-  const int grid = p.tc_nf + ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
+  const int grid = ((heads + TC_NH - 1) / TC_NH) * p.n_splits;
   switch (de_slot) {
     case 0: return launch_tc_g<0>(p, grid, smem, stream);
     case 8: return launch_tc_g<1>(p, grid, smem, stream);
