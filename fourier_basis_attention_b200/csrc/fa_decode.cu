@@ -470,45 +470,65 @@ __global__ void __launch_bounds__(DNT, SPT == 1 ? 2 : 1)
 }
 
 // ------------------------------------------------------------------------- combine
-// One CTA per KV head (its G query heads share C_V), CB_THREADS threads = 8 warps.
-//  1. warp h: record weights w_r = 2^(m_r - m*) and the sum l of query head h;
+// One CTA per (KV head, group of GT of its G query heads; the heads of a group share C_V),
+// CB_THREADS threads = 8 warps. GT = G unless that leaves too few CTAs for the GPU.
+//  1. warp h < GT: record weights w_r = 2^(m_r - m*) and the sum l of query head h;
 //  2. the weighted sum over split records of their payload (retained-dim values, then u
-//     slots), 128 columns at a time: warp w takes records w, w + 8, ... and reads each
-//     record's 128 columns as one float4 per lane, so many loads are in flight; the eight
-//     partial rows are then added in a fixed order (deterministic);
+//     slots), CB_PW(GT) columns per pass: warp w takes records w, w + 8, ... and reads each
+//     record's columns as CB_NPW(GT) float4 per lane, CB_RB(GT) records per batch, so many
+//     loads are in flight; the eight partial rows are then added in a fixed order
+//     (deterministic);
 //  3. out_c = u C_V with u_j = basis scale of function j x its slot sum, C_V staged
-//     through shared memory in CB_KC-row chunks;
+//     through shared memory in double-buffered CB_KC-row chunks (cp.async, started before
+//     step 1: C_V does not depend on the records);
 //  4. sink / recent records (all 128 dims in natural order) are added per dim, the dims
 //     scattered back, normalised and stored.
 constexpr int CB_THREADS = 256;
 constexpr int CB_KC = 64;
 
+__host__ __device__ constexpr int CB_NPW(int GT) { return GT >= 8 ? 2 : 4; }
+__host__ __device__ constexpr int CB_PW(int GT) { return 128 * CB_NPW(GT); }
+__host__ __device__ constexpr int CB_RB(int GT) {
+  return 16 / (GT * CB_NPW(GT)) > 1 ? 16 / (GT * CB_NPW(GT)) : 1;
+}
+
 // Float offsets of the combine's shared arrays; every one a multiple of 4 (16 bytes), so
 // the float4 accesses stay aligned.
 __host__ __device__ inline int combine_wts_floats(int G, int nrec) { return (G * nrec + 3) & ~3; }
 
-__host__ __device__ inline size_t combine_smem_floats(int G, int nrec, int payload) {
-  return (size_t)combine_wts_floats(G, nrec) + 16 + (size_t)G * payload + (size_t)8 * G * 128 +
-         (size_t)2 * CB_KC * FA_HEAD_DIM + 2 * (size_t)G * FA_HEAD_DIM + FA_HEAD_DIM;
+// Columns of one pass actually used: the pass width, or the whole payload if narrower.
+__host__ __device__ inline int combine_pass_cols(int GT, int payload) {
+  return payload < CB_PW(GT) ? ((payload + 3) & ~3) : CB_PW(GT);
 }
 
+__host__ __device__ inline size_t combine_smem_floats(int GT, int nrec, int payload) {
+  return (size_t)combine_wts_floats(GT, nrec) + 16 + (size_t)GT * payload +
+         (size_t)8 * GT * combine_pass_cols(GT, payload) + (size_t)2 * CB_KC * FA_HEAD_DIM +
+         2 * (size_t)GT * FA_HEAD_DIM + FA_HEAD_DIM;
+}
+
+template <int GT>
 __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid_constant__ DecodeParams p) {
+  constexpr int NPW = CB_NPW(GT), RB = CB_RB(GT);
   extern __shared__ __align__(16) float cs[];
-  const int kvh = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_grp = p.G / GT;
+  const int kvh = blockIdx.x / n_grp, hg = blockIdx.x - (blockIdx.x / n_grp) * n_grp;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
-  const int G = p.G, dc = p.dc[g], dc_ld = p.dc_ld[g], nrec = p.n_rec, ns = p.n_splits;
+  const int dc = p.dc[g], dc_ld = p.dc_ld[g], nrec = p.n_rec, ns = p.n_splits;
   const int k = p.k;
   const int payload = p.rec_stride - 4;     // retained-dim values (128) + u slots (2 F_pad)
-  float* wts = cs;                          // [G][nrec]
-  float* mst = wts + combine_wts_floats(G, nrec);  // [8]
+  const int PWc = combine_pass_cols(GT, payload);
+  float* wts = cs;                          // [GT][nrec]
+  float* mst = wts + combine_wts_floats(GT, nrec);  // [8]
   float* lsum = mst + 8;                    // [8]
-  float* sum = lsum + 8;                    // [G][payload] weighted sum of split payloads
-  float* red = sum + G * payload;           // [8 warps][G][128] partial column sums
-  float* cvs = red + 8 * G * 128;           // [2][CB_KC][128] chunks of C_V (double buffer)
-  float* cpart = cvs + 2 * CB_KC * FA_HEAD_DIM; // [2][G][128] halves of u C_V
-  int* inv = reinterpret_cast<int*>(cpart + 2 * G * FA_HEAD_DIM);  // [128]
+  float* sum = lsum + 8;                    // [GT][payload] weighted sum of split payloads
+  float* red = sum + GT * payload;          // [8 warps][GT][PWc] partial column sums
+  float* cvs = red + 8 * GT * PWc;          // [2][CB_KC][128] chunks of C_V (double buffer)
+  float* cpart = cvs + 2 * CB_KC * FA_HEAD_DIM;  // [2][GT][128] halves of u C_V
+  int* inv = reinterpret_cast<int*>(cpart + 2 * GT * FA_HEAD_DIM);  // [128]
   const long long bhq = (long long)p.B * p.Hq;
-  const long long gh0 = (long long)b * p.Hq + (long long)g * G;
+  const long long gh0 = (long long)b * p.Hq + (long long)g * p.G + (long long)hg * GT;
   auto rec = [&](int r, int h) -> const float* {
     return p.rec + ((long long)r * bhq + gh0 + h) * p.rec_stride;
   };
@@ -533,7 +553,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
   load_cv_chunk(0);
   load_cv_chunk(1);
   if (tid < FA_HEAD_DIM) inv[p.perm[g][tid]] = tid;
-  if (warp < G) {
+  if (warp < GT) {
     const int h = warp;
     float mx = -INFINITY;
     for (int r = lane; r < nrec; r += 32) mx = fmaxf(mx, rec(r, h)[0]);
@@ -554,38 +574,58 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
     }
   }
   __syncthreads();
-  // weighted sum of the split records' payloads, 128 columns per pass
-  for (int c0 = 0; c0 < payload && ns > 0; c0 += 128) {
-    const int col = c0 + lane * 4;
-    float4 a[HL];
+  // weighted sum of the split records' payloads, PWc columns per pass; lane l, piece j
+  // covers columns c0 + 128 j + 4 l .. + 3
+  for (int c0 = 0; c0 < payload && ns > 0; c0 += PWc) {
+    float4 a[GT][NPW];
 #pragma unroll
-    for (int h = 0; h < HL; ++h) a[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    if (col < payload) {
-#pragma unroll 8  // several records' rows in flight per lane
-      for (int r = warp; r < ns; r += 8) {
+    for (int h = 0; h < GT; ++h)
 #pragma unroll
-        for (int h = 0; h < HL; ++h) {
-          if (h < G) {
-            const float w = wts[h * nrec + r];
-            const float4 v = *reinterpret_cast<const float4*>(rec(r, h) + 4 + col);
-            a[h].x += w * v.x;
-            a[h].y += w * v.y;
-            a[h].z += w * v.z;
-            a[h].w += w * v.w;
+      for (int j = 0; j < NPW; ++j) a[h][j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int r0 = warp; r0 < ns; r0 += 8 * RB) {
+      float4 v[RB][GT][NPW];
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const int r = r0 + 8 * u;
+#pragma unroll
+        for (int h = 0; h < GT; ++h)
+#pragma unroll
+          for (int j = 0; j < NPW; ++j) {
+            const int col = c0 + 128 * j + 4 * lane;
+            v[u][h][j] = (r < ns && col < payload && 128 * j + 4 * lane < PWc)
+                             ? *reinterpret_cast<const float4*>(rec(r, h) + 4 + col)
+                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          }
+      }
+#pragma unroll
+      for (int u = 0; u < RB; ++u) {
+        const int r = r0 + 8 * u;
+#pragma unroll
+        for (int h = 0; h < GT; ++h) {
+          const float w = r < ns ? wts[h * nrec + r] : 0.0f;
+#pragma unroll
+          for (int j = 0; j < NPW; ++j) {
+            a[h][j].x += w * v[u][h][j].x;
+            a[h][j].y += w * v[u][h][j].y;
+            a[h][j].z += w * v[u][h][j].z;
+            a[h][j].w += w * v[u][h][j].w;
           }
         }
       }
     }
 #pragma unroll
-    for (int h = 0; h < HL; ++h)
-      if (h < G) reinterpret_cast<float4*>(red + (warp * G + h) * 128)[lane] = a[h];
+    for (int h = 0; h < GT; ++h)
+#pragma unroll
+      for (int j = 0; j < NPW; ++j)
+        if (128 * j + 4 * lane < PWc)
+          *reinterpret_cast<float4*>(red + (warp * GT + h) * PWc + 128 * j + 4 * lane) = a[h][j];
     __syncthreads();
-    for (int idx = tid; idx < G * 128; idx += CB_THREADS) {
-      const int h = idx >> 7, cc = idx & 127;
+    for (int idx = tid; idx < GT * PWc; idx += CB_THREADS) {
+      const int h = idx / PWc, cc = idx - (idx / PWc) * PWc;
       if (c0 + cc < payload) {
         float v = 0.0f;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[(w * G + h) * 128 + cc];
+        for (int w = 0; w < 8; ++w) v += red[(w * GT + h) * PWc + cc];
         sum[h * payload + c0 + cc] = v;
       }
     }
@@ -594,9 +634,9 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
   // out_c = u C_V: C_V rows in double-buffered chunks; thread (half, column i) sums the rows
   // of its parity
   const int colc = tid & (FA_HEAD_DIM - 1), half = tid >> 7;
-  float acc[HL];
+  float acc[GT];
 #pragma unroll
-  for (int h = 0; h < HL; ++h) acc[h] = 0.0f;
+  for (int h = 0; h < GT; ++h) acc[h] = 0.0f;
   for (int j0 = 0; j0 < k && do_cv; j0 += CB_KC) {
     const int nj = min(CB_KC, k - j0), ci = j0 / CB_KC;
     const float* cvb = cvs + (ci & 1) * CB_KC * FA_HEAD_DIM;
@@ -609,8 +649,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
         const float cv = cvb[jj * FA_HEAD_DIM + colc] *
                          ((f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair);
 #pragma unroll
-        for (int h = 0; h < HL; ++h)
-          if (h < G) acc[h] += sum[h * payload + slot] * cv;
+        for (int h = 0; h < GT; ++h) acc[h] += sum[h * payload + slot] * cv;
       }
     }
     __syncthreads();     // chunk ci consumed: its buffer takes chunk ci + 2
@@ -619,10 +658,9 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
   cp_async_wait<0>();
   __syncthreads();
 #pragma unroll
-  for (int h = 0; h < HL; ++h)
-    if (h < G) cpart[(half * G + h) * FA_HEAD_DIM + colc] = acc[h];
+  for (int h = 0; h < GT; ++h) cpart[(half * GT + h) * FA_HEAD_DIM + colc] = acc[h];
   __syncthreads();
-  for (int idx = tid; idx < G * FA_HEAD_DIM; idx += CB_THREADS) {
+  for (int idx = tid; idx < GT * FA_HEAD_DIM; idx += CB_THREADS) {
     const int h = idx / FA_HEAD_DIM, d = idx - h * FA_HEAD_DIM;
     const int i = inv[d];
     float o = 0.0f;
@@ -630,7 +668,7 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
       if (i >= dc)
         o = sum[h * payload + (i - dc)];
       else
-        o = cpart[h * FA_HEAD_DIM + i] + cpart[(G + h) * FA_HEAD_DIM + i];
+        o = cpart[h * FA_HEAD_DIM + i] + cpart[(GT + h) * FA_HEAD_DIM + i];
     }
     const float* wh = wts + h * nrec;
     for (int r = ns; r < nrec; ++r) o += wh[r] * rec(r, h)[4 + d];
@@ -644,6 +682,26 @@ __global__ void __launch_bounds__(CB_THREADS) decode_combine_kernel(const __grid
 }
 
 // ------------------------------------------------------------------------- host side
+template <int GT>
+static cudaError_t launch_combine_t(const DecodeParams& p, const DecodeConfig& c, int n_heads,
+                                    cudaStream_t stream) {
+  cudaError_t e = raise_smem_limit(reinterpret_cast<const void*>(decode_combine_kernel<GT>),
+                                   (int)c.smem_combine);
+  if (e != cudaSuccess) return e;
+  decode_combine_kernel<GT><<<n_heads * (p.G / GT), CB_THREADS, c.smem_combine, stream>>>(p);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_combine(const DecodeParams& p, const DecodeConfig& c, int n_heads,
+                                  cudaStream_t stream) {
+  switch (c.cb_gt) {
+    case 1: return launch_combine_t<1>(p, c, n_heads, stream);
+    case 2: return launch_combine_t<2>(p, c, n_heads, stream);
+    case 4: return launch_combine_t<4>(p, c, n_heads, stream);
+    case 8: return launch_combine_t<8>(p, c, n_heads, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
 static int next_pow2(int x) {
   int v = 1;
   while (v < x) v <<= 1;
@@ -755,7 +813,16 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   const long long bhq = (long long)sh.B * sh.Hq;
   c->qw_bytes = (size_t)(bhq * c->qw_stride * 4);
   c->rec_bytes = (size_t)((long long)c->n_rec * bhq * c->rec_stride * 4);
-  c->smem_combine = combine_smem_floats(plan->G, c->n_rec, c->rec_stride - 4) * 4;
+  // query heads per combine CTA: all G of a KV head (they share C_V) unless that leaves
+  // fewer than two CTAs per SM, then halved (each CTA re-reads C_V)
+  {
+    int sms = 148;
+    if (device_sm_count(&sms) != cudaSuccess) sms = 148;  // no device: sizes only
+    int gt = plan->G;
+    while (gt > 1 && (long long)n_heads * (plan->G / gt) < 2LL * sms) gt >>= 1;
+    c->cb_gt = gt;
+  }
+  c->smem_combine = combine_smem_floats(c->cb_gt, c->n_rec, c->rec_stride - 4) * 4;
   return c->smem_combine <= 227 * 1024 ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -854,10 +921,7 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  e = raise_smem_limit(reinterpret_cast<const void*>(decode_combine_kernel), (int)c.smem_combine);
-  if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<n_heads, CB_THREADS, c.smem_combine, stream>>>(p);
-  return cudaGetLastError();
+  return launch_combine(p, c, n_heads, stream);
 }
 
 }  // namespace fa

@@ -13,6 +13,7 @@ struct DecodeConfig {
   int n_splits, split_len, n_fsplits, n_rec, F, F_pad, SPT, NTU, TG, DEC, TGE, NKV;
   int tc, tc_F2, tc_tmem_cols, de_ld_max;  // tensor-core split kernel chosen, its slots / TMEM
   int hm, hm_F2;  // warp-MMA split kernel chosen (blocked E, large k), its slots
+  int cb_gt;      // query heads per combine CTA (a divisor of G)
   size_t qw_bytes, rec_bytes, smem_main, smem_combine;
   int rec_stride, qw_stride;
 };
