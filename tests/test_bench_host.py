@@ -1,0 +1,49 @@
+"""Host-side accounting of bench.py: the algorithmic work model, the launch count and the
+append byte count, checked against independent hand counts (no GPU)."""
+import numpy as np
+
+import bench
+import fourier_basis_attention_b200 as fa
+import workloads as wl
+
+
+def _plan(w, mask=None):
+    mask = wl.dim_mask(w) if mask is None else mask
+    return fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+
+
+def test_work_model_bench_workload_by_hand():
+    """LLaMA-2-7B MHA, B=8, L=32768, k=255, 96 of 128 dims compressed in every head."""
+    w = wl.LLAMA2_7B_MHA_32K
+    p = _plan(w)
+    assert all(p.dc[g] == 96 for g in range(w.Hkv))
+    M, k, SR = 32768 - 96, 255, 96
+    heads = 8 * 32
+    per_head_c = 2 * (2 * M * 128 + 4 * k * 96 + 2 * M * 32 + 4 * SR * 128)   # K and V
+    per_head_d = 2 * (2 * SR * 128 + 2 * M * 32 + 4 * k * 96)
+    wm = bench.work_model(w, p)
+    assert wm["compress_bytes"] == heads * per_head_c
+    assert wm["compress_flops"] == heads * 2 * 2 * k * M * 96
+    assert wm["decode_bytes"] == heads * per_head_d + 2 * 2 * 8 * 32 * 128
+    # the figures quoted with the bench line
+    assert wm["compress_bytes"] == 5428281344 and wm["decode_bytes"] == 1133445120
+
+
+def test_launches_per_step_each_path():
+    """6 launches on the tensor-core and warp-MMA paths (sink / recent rows ride in the
+    prologue launch) and on the CUDA-core path (they ride in the split kernel)."""
+    tc = wl.LLAMA2_7B_MHA_32K
+    hm = wl.LLAMA3_8B_GQA_128K
+    cc = wl.llama3_8b_layer(1, 8192, 0)
+    assert _plan(tc).e_token_major == 1 and bench.launches_per_step(tc, _plan(tc)) == 6
+    assert _plan(hm).e_token_major == 0 and bench.launches_per_step(hm, _plan(hm)) == 6
+    assert _plan(cc).e_token_major == 0 and bench.launches_per_step(cc, _plan(cc)) == 6
+
+
+def test_append_bytes_by_hand():
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=2, Hkv=4, Hq=4, L=5000)
+    mask = np.zeros((4, 128), dtype=np.uint8)
+    mask[:, :96] = 1                                  # dc = 96, de = 32 in every head
+    p = _plan(w, mask)
+    per = 2 * 255 * 96 * 4 + 32 * 2 + 3 * 256
+    assert bench.append_bytes(p) == 2 * 2 * 4 * per
