@@ -271,7 +271,10 @@ int fa_decode_noalloc(const fa_plan* plan, const void* q, const fa_cache* cache,
  * The result equals fa_compress of the longer sequence with the same period, up to fp32
  * rounding of the coefficients (E and F are bit-exact).
  * Returns FA_ERR_UNSUPPORTED when no room is left (M == P) or the plan has no middle
- * span; argument errors as for the other entry points. Launches one kernel.
+ * span; argument errors as for the other entry points. Launches one kernel (two when the
+ * fold is split into row chunks to fill the GPU). The position (t = M, the ring head) is
+ * taken from the plan when the call is made, so a CUDA graph that captured this call
+ * replays that same position.
  */
 int fa_append(fa_plan* plan, const void* k_new, const void* v_new, const fa_cache* cache,
               void* stream);
