@@ -41,7 +41,7 @@ struct AppendParams {
 __global__ void __launch_bounds__(AP_THREADS) append_kernel(const __grid_constant__ AppendParams p) {
   __shared__ float xc[FA_HEAD_DIM];               // compressed dims of x, in C column order
   __shared__ __nv_bfloat16 xb[FA_HEAD_DIM];       // x, all dims
-  __shared__ float ub[FA_MAX_K_DECODE + 1];       // phi_j(t), j < k
+  __shared__ float ub[FA_MAX_K_DECODE + 1];       // phi_j(t) of this chunk's rows j0 <= j < j1
   const int tid = threadIdx.x;
   const int head = blockIdx.x, which = blockIdx.y, z = blockIdx.z;
   const int j0 = z * p.chunk_rows, j1 = min(p.k, j0 + p.chunk_rows);

@@ -11,6 +11,9 @@ GOLDEN = os.path.join(ROOT, "tests", "golden")
 
 
 def pytest_configure(config):
+    # temporary files (compiled C probes of the ABI) stay inside the repository
+    if not config.option.basetemp:
+        config.option.basetemp = os.path.join(ROOT, ".pytest_tmp")
     config.addinivalue_line("markers", "gpu: needs a CUDA device (sm_100a)")
     config.addinivalue_line("markers", "slow: large parity case (full-size workload)")
 

@@ -338,3 +338,16 @@ def test_select_dims_rejections():
     r = fa.LIB.fa_dim_sensitivity(ctypes.byref(shape), 0x1000, 0x1000, 0x1000, 0x1000, 0x1000,
                                   1 << 20, None)
     assert r == fa.FA_ERR_UNSUPPORTED
+
+
+def test_c_program_uses_the_abi(tmp_path):
+    """A plain C program (gcc, no C++ or torch) links the library and runs the host-only
+    entry points: plan, reservation, append refusal, dim selection."""
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    exe = tmp_path / "c_abi_host"
+    libdir = os.path.dirname(fa.LIB_PATH)
+    subprocess.run(["gcc", "-std=c11", "-I", os.path.join(root, "include"),
+                    os.path.join(root, "tests", "c_abi_host.c"), "-o", str(exe),
+                    "-L", libdir, "-lfourier_attention", f"-Wl,-rpath,{libdir}"], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
