@@ -165,7 +165,8 @@ int fa_plan_reserve(fa_plan* plan, int32_t L_max);
 /*
  * fa_build_basis -- the orthonormal real Fourier basis over a span of M tokens, transposed.
  * ([abstract] "orthogonal Fourier bases"; [skill] Step 2 keeps the leading spectral
- * terms of a real FFT along the sequence.)
+ * terms of a real FFT along the sequence.) M is the basis period: pass the plan's P (which
+ * equals the middle length unless fa_plan_reserve made room).
  *   phi_0(t) = 1/sqrt(M); for j >= 1, f = (j + 1) / 2 and phi_j is sqrt(2/M) cos(2 pi f t / M)
  *   (j odd) or sqrt(2/M) sin(2 pi f t / M) (j even); the cosine at f = M/2 (M even) uses
  *   1/sqrt(M). The phase f*t is reduced modulo M exactly in integers first.
