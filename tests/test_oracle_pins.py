@@ -432,3 +432,31 @@ def test_sensitivity_pin_rejects_planted_mistakes():
                                                   for b in range(2)]))
     for wrong in (keys, good / 0.1):
         assert np.abs(wrong - ref).max() > 1e-6 * ref.max()
+
+
+# ----------------------------------------------------------------------------- properties
+
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=40, deadline=None)
+@given(M=st.integers(1, 300), extra=st.integers(0, 200), kfrac=st.floats(0.0, 1.0),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_period_projection_bessel_and_linearity(M, extra, kfrac, seed):
+    """For any period P >= M and k <= P the coefficients are an orthogonal projection of the
+    middle zero-padded to P samples: Bessel's inequality holds (equality at k = P), and the
+    map is linear."""
+    P = M + extra
+    k = max(1, min(P, int(round(kfrac * P))))
+    rng = np.random.default_rng(seed)
+    x, y = rng.standard_normal((M, 3)), rng.standard_normal((M, 3))
+    mask = np.ones(3)
+    cx = fo.compress(x, mask, 0, 0, k, period=P).C
+    cy = fo.compress(y, mask, 0, 0, k, period=P).C
+    energy = (x ** 2).sum(0)
+    assert np.all((cx ** 2).sum(0) <= energy * (1 + 1e-12))
+    if k == P:
+        assert np.allclose((cx ** 2).sum(0), energy, rtol=1e-10)
+    a, b = rng.standard_normal(2)
+    cxy = fo.compress(a * x + b * y, mask, 0, 0, k, period=P).C
+    assert np.abs(cxy - (a * cx + b * cy)).max() <= 1e-10 * max(1.0, np.abs(cxy).max())
