@@ -351,3 +351,60 @@ def test_c_program_uses_the_abi(tmp_path):
                     "-L", libdir, "-lfourier_attention", f"-Wl,-rpath,{libdir}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0 and out.stdout.strip() == "ok", out.stdout + out.stderr
+
+
+# ----------------------------------------------------------------------------- layout properties
+
+from hypothesis import given, settings, strategies as st
+
+
+@settings(max_examples=60, deadline=None)
+@given(B=st.integers(1, 40), Hkv=st.sampled_from([1, 2, 4, 8]), G=st.sampled_from([1, 2, 4, 8]),
+       L=st.integers(1, 3000), S=st.integers(0, 40), R=st.integers(0, 80),
+       k=st.integers(1, 300), extra=st.integers(0, 500), seed=st.integers(0, 2 ** 31 - 1))
+def test_plan_layout_properties(B, Hkv, G, L, S, R, k, extra, seed):
+    """Every plan the host derives (with or without reserved room) has disjoint, in-bounds
+    E and C blocks, the documented token-major rule, padded row widths and sorted dim lists."""
+    rng = np.random.default_rng(seed)
+    mask = (rng.random((Hkv, 128)) < rng.random()).astype(np.uint8)
+    Hq = Hkv * G
+    try:
+        p = fa.fa_plan_init(B, Hq, Hkv, L, S, R, k, mask)
+    except fa.FaError as e:
+        assert e.code == fa.FA_ERR_UNSUPPORTED and k > L - min(S, L) - min(R, L - min(S, L))
+        return
+    if p.M > 0 and extra > 0:
+        fa.fa_plan_reserve(p, L + extra)
+    assert p.S + p.M + p.R == L and p.P >= p.M
+    assert p.f_elems == B * Hkv * (p.S + p.R) * 128
+    de = [p.de[g] for g in range(Hkv)]
+    tm = (p.M > 0 and k <= 255 and G in (1, 2, 4) and max(de) <= 32 and k * G >= 255
+          and B * Hq >= 128)
+    assert p.e_token_major == int(tm)
+    for g in range(Hkv):
+        cd, ed = fa.perm_lists(p, g)
+        assert list(cd) == sorted(cd) and list(ed) == sorted(ed)
+        assert sorted(list(cd) + list(ed)) == list(range(128))
+        assert p.dc_ld[g] % 8 == 0 and p.dc_ld[g] >= p.dc[g]
+        assert p.de_ld[g] >= p.de[g] and (p.de_ld[g] == 0 or p.de_ld[g] % 8 == 0)
+    # E: element intervals [start, start + de_ld) of every (b, g, t < P) row are disjoint and
+    # inside e_elems; C: the [kk][dc_ld] blocks likewise inside c_elems
+    rows = []
+    for b in range(min(B, 3)):
+        for g in range(Hkv):
+            if p.de_ld[g] == 0:
+                continue
+            for t in {t for t in (0, 1, p.P // 2, p.P - 1) if 0 <= t < p.P}:
+                start = b * p.e_batch + p.e_off[g] + t * p.e_pitch[g]
+                rows.append((start, start + p.de_ld[g]))
+    rows.sort()
+    for (a0, a1), (b0, _) in zip(rows, rows[1:]):
+        assert a1 <= b0
+    if rows:
+        assert rows[0][0] >= 0 and max(r[1] for r in rows) <= p.e_elems
+    blocks = sorted((b * p.c_batch + p.c_off[g], b * p.c_batch + p.c_off[g] + p.kk * p.dc_ld[g])
+                    for b in range(B) for g in range(Hkv) if p.kk * p.dc_ld[g] > 0)
+    for (a0, a1), (b0, _) in zip(blocks, blocks[1:]):
+        assert a1 <= b0
+    if blocks:
+        assert blocks[-1][1] <= p.c_elems
