@@ -11,15 +11,18 @@
 //
 // Three launches on the caller's stream:
 //   prologue  per KV head: q_c / q_e gathered by the dim mask, w = C_K^T q_c, with the
-//             softmax scale, log2(e) and the basis normalisation folded in.
-//   main      split-L: CTA (head set, split) streams its token range of E_K / E_V in
-//             tiles of 64 tokens for 8 query heads at once, regenerating cos/sin of the
-//             basis by a rotation recurrence (re-seeded from sincospif of the exactly
-//             reduced phase), with an fp32 online softmax. Extra CTAs do the sink /
-//             recent rows of each KV head. Every CTA writes a partial record
-//             (running max, running sum, value accumulator, u).
-//   combine   per KV head: merges the records, out_c = u C_V, scatters the dims back,
-//             normalises and stores fp32 or bf16.
+//             softmax scale, log2(e) and the basis normalisation folded in. On the
+//             tensor-core and warp-MMA paths the same launch runs the sink / recent rows.
+//   split     the middle span, split-L: the tensor-core kernel (fa_decode_tc.cu, token-major
+//             E, k <= 255), the warp-MMA kernel (fa_decode_hmma.cu, 256 <= k <= 1023) or the
+//             CUDA-core kernel below: CTA (head set, split) streams its token range of
+//             E_K / E_V in tiles of 64 tokens for 8 query heads at once, regenerating
+//             cos/sin of the basis by a rotation recurrence (re-seeded from sincospif of the
+//             exactly reduced phase), with an fp32 online softmax; its extra CTAs do the
+//             sink / recent rows. Every CTA writes a partial record (running max, running
+//             sum, value accumulator, u).
+//   combine   per (KV head, group of its query heads): merges the records, out_c = u C_V,
+//             scatters the dims back, normalises and stores fp32 or bf16.
 #include "fa_decode_common.cuh"
 
 namespace fa {
