@@ -460,3 +460,14 @@ def test_period_projection_bessel_and_linearity(M, extra, kfrac, seed):
     a, b = rng.standard_normal(2)
     cxy = fo.compress(a * x + b * y, mask, 0, 0, k, period=P).C
     assert np.abs(cxy - (a * cx + b * cy)).max() <= 1e-10 * max(1.0, np.abs(cxy).max())
+
+
+def test_period_hand_example(hand_cases):
+    """A middle of 2 tokens under period 4, then one appended token (hand-derived values)."""
+    x = np.array(hand_cases["period4_x"])[:, None]
+    h = fo.compress(x, np.ones(1), 0, 0, 4, period=4)
+    assert h.P == 4 and h.M == 2
+    assert np.abs(h.C[:, 0] - hand_cases["period4_C"]).max() < 1e-15
+    x3 = np.array(hand_cases["period4_x_appended"])[:, None]
+    h3 = fo.compress(x3, np.ones(1), 0, 0, 4, period=4)
+    assert np.abs(h3.C[:, 0] - hand_cases["period4_C_appended"]).max() < 1e-15
