@@ -255,6 +255,17 @@ class Cache:
         t = self.F_K if which == "K" else self.F_V
         return t[:p.f_elems].view(p.shape.B, p.shape.Hkv, p.S + p.R, HEAD_DIM)
 
+    def F_tokens(self, which: str):
+        """[B, Hkv, S + R, 128]: the sink rows, then the recent rows in token order (the ring
+        rotated so that its oldest row comes first). A copy, not a view."""
+        import torch
+        p = self.plan
+        F = self.F(which)
+        if p.R == 0 or p.recent_head == 0:
+            return F.clone()
+        idx = list(range(p.S)) + [p.S + (p.recent_head + a) % p.R for a in range(p.R)]
+        return F[:, :, torch.tensor(idx, device=F.device)]
+
     def E(self, which: str, b: int, g: int):
         return self.E_raw(which, b, g)[:, :self.plan.de[g]]
 

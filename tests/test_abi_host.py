@@ -408,3 +408,26 @@ def test_plan_layout_properties(B, Hkv, G, L, S, R, k, extra, seed):
         assert a1 <= b0
     if blocks:
         assert blocks[-1][1] <= p.c_elems
+
+
+def test_cache_views_on_host_memory():
+    """The Cache views follow the documented layouts (checked on CPU tensors; no kernel)."""
+    import torch
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=2, Hq=4, Hkv=2, L=400, S=4, R=6, k=15)
+    mask = np.zeros((2, 128), dtype=np.uint8)
+    mask[:, ::2] = 1                                      # 64 compressed, 64 retained
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    c = fa.Cache(p, device="cpu")
+    # F: write each row's token index, then rotate the ring by hand
+    F = c.F("K")
+    for i in range(p.S + p.R):
+        F[:, :, i] = i
+    p.recent_head = 2
+    got = c.F_tokens("K")[0, 0, :, 0].tolist()
+    assert got == [0, 1, 2, 3] + [4 + (2 + a) % 6 for a in range(6)]
+    # E: row t of head (b, g) at b * e_batch + e_off[g] + t * e_pitch[g]
+    c.E_K.zero_()
+    c.E_K[1 * p.e_batch + p.e_off[1] + 7 * p.e_pitch[1] + 3] = 5.0
+    assert c.E("K", 1, 1)[7, 3].item() == 5.0 and c.E("K", 1, 1).sum().item() == 5.0
+    # C: [kk][dc_ld] block of (b, g), padding columns past dc
+    assert c.C("V", 0, 1).shape == (15, 64) and c.C_raw("V", 0, 1).shape == (15, p.dc_ld[1])
