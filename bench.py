@@ -30,6 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "fa_decode μs/step & HBM GB/s; fa_compress TFLOP/s; % of B200 roofline"
+L2_BYTES = 126 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -41,6 +42,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama2_7b_mha_b8_L32768_k255")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload measurements added to the default line")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--no-clock-probe", action="store_true",
@@ -71,23 +74,58 @@ def workload_by_name(name):
 # ----------------------------------------------------------------------------- algorithmic work
 
 def work_model(w, plan):
-    """Algorithmic bytes / flops per step, from the plan's per-head dim split."""
+    """Algorithmic bytes / flops per step, from the plan's per-head dim split.
+
+    Two byte counts per half of the path:
+    * ``*_bytes``: what this implementation moves by design: C stored in fp32, and
+      fa_compress also copies the sink / recent rows into F;
+    * ``*_bytes_alg``: the method's minimum (bf16 C; compress reads the middle rows once
+      and writes C and E, decode reads F, E and C of K and V plus q and writes out).
+    Rooflines are reported against ``*_bytes_alg`` (the smaller, so the harder, figure)."""
     B, Hkv, G, D = w.B, w.Hkv, w.G, 128
     S, R, M, k = plan.S, plan.R, plan.M, w.k
     dcs = [plan.dc[g] for g in range(Hkv)]
     des = [plan.de[g] for g in range(Hkv)]
+    kk = k if M > 0 else 0
     # compress: read the middle rows once, write C (fp32) and E, copy the sink/recent rows
     # (K and V)
-    c_bytes = 2 * B * sum(2 * M * D + 4 * k * dc + 2 * M * de + 2 * 2 * (S + R) * D
+    c_bytes = 2 * B * sum(2 * M * D + 4 * kk * dc + 2 * M * de + 2 * 2 * (S + R) * D
                           for dc, de in zip(dcs, des))
-    c_flops = 2 * 2 * B * sum(k * M * dc for dc in dcs)
-    # decode: read F, E (bf16) and C (fp32) of K and V, the queries, write the outputs
-    d_bytes = 2 * B * sum(2 * (S + R) * D + 2 * M * de + 4 * k * dc for dc, de in zip(dcs, des)) \
-        + 2 * 2 * B * w.Hq * D
-    d_flops = B * G * sum(4 * D * (S + R) + 4 * de * M + 4 * k * dc + 4 * M * k
+    c_bytes_alg = 2 * B * sum(2 * M * D + 2 * kk * dc + 2 * M * de for dc, de in zip(dcs, des))
+    c_flops = 2 * 2 * B * sum(kk * M * dc for dc in dcs)
+    # decode: read F, E (bf16) and C of K and V, the queries, write the outputs
+    qo = 2 * 2 * B * w.Hq * D
+    d_bytes = 2 * B * sum(2 * (S + R) * D + 2 * M * de + 4 * kk * dc for dc, de in zip(dcs, des)) + qo
+    d_bytes_alg = 2 * B * sum(2 * (S + R) * D + 2 * M * de + 2 * kk * dc
+                              for dc, de in zip(dcs, des)) + qo
+    d_flops = B * G * sum(4 * D * (S + R) + 4 * de * M + 4 * kk * dc + 4 * M * kk
                           for dc, de in zip(dcs, des))
-    return dict(compress_bytes=c_bytes, compress_flops=c_flops, decode_bytes=d_bytes,
-                decode_flops=d_flops)
+    return dict(compress_bytes=c_bytes, compress_bytes_alg=c_bytes_alg, compress_flops=c_flops,
+                decode_bytes=d_bytes, decode_bytes_alg=d_bytes_alg, decode_flops=d_flops)
+
+
+def decode_path(w, plan):
+    """Which split kernel fa_decode runs for this plan (mirrors the library's choice)."""
+    if plan.M == 0:
+        return "none (no middle span)"
+    if plan.e_token_major:
+        return "tcgen05 (decode_tc_kernel)"
+    if 256 <= w.k <= 1023:
+        return "warp MMA (decode_hmma_kernel)"
+    return "CUDA cores (decode_main_kernel)"
+
+
+def config_dict(w, world=1):
+    """The ``config`` object of the JSON line; both arms print exactly this."""
+    import workloads as wl
+    mask = wl.dim_mask(w)
+    dcs = sorted({int(x) for x in mask.sum(axis=1)})
+    return {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L, "Hq": w.Hq,
+            "Hkv": w.Hkv, "k": w.k, "S": w.S, "R": w.R,
+            "dims_compressed_per_head": dcs[0] if len(dcs) == 1 else dcs,
+            "parallelism": f"replica x{world}",
+            "l2": ("inputs larger than L2 (K+V %.2f GB per replica)" if 2 * K_bytes(w) > L2_BYTES
+                   else "inputs fit in L2 (K+V %.4f GB per replica)") % (2 * K_bytes(w) / 1e9)}
 
 
 def load_peaks():
@@ -111,6 +149,23 @@ def compress_traffic():
         return None
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     return rec if digest == rec.get("source_sha256_16") else None
+
+
+def decode_traffic():
+    """Measured DRAM traffic of one fa_decode on the bench workload (profiles/), if it was
+    taken on the current decode sources."""
+    path = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as fh:
+        rec = json.load(fh)
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        src = os.path.join(ROOT, "fourier_basis_attention_b200", "csrc", name)
+        if not os.path.exists(src):
+            return None
+        h.update(open(src, "rb").read())
+    return rec.get("bytes_per_step") if h.hexdigest()[:16] == rec.get("sources_sha256_16") else None
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -178,15 +233,37 @@ def summarize_clocks(rows):
 
 # ----------------------------------------------------------------------------- oracle timing
 
-def oracle_sample(w, K_pairs, V_pairs, q_pairs, masks):
-    """Time the fp64 oracle on whole (batch, KV head) pairs; returns seconds per pair."""
+ORACLE_PAIRS = 4  # (batch, KV head) pairs the oracle runs per sampled step
+
+
+def oracle_step_seconds(w, pairs):
+    """One sampled oracle step, scaled to the whole workload, in seconds.
+
+    The same policy serves the GPU arm's ``cpu_baseline`` and ``--impl reference``: the
+    oracle's basis cache is cleared, the basis is built once (timed: the GPU step rebuilds
+    its table every step too), then len(pairs) whole (batch, KV head) pairs run fp64
+    compress of K and V and the decode step; the pair time is scaled to all B * Hkv pairs."""
     from oracle import fourier_oracle as fo
+    fo._basis_full.cache_clear()
+    S_, R_, M = fo.partition(w.L, w.S, w.R)
     t0 = time.perf_counter()
-    for (Kh, Vh, qh, m) in zip(K_pairs, V_pairs, q_pairs, masks):
+    if M > 0:
+        fo._basis_full(M, w.k, M)
+    t_basis = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    for (Kh, Vh, qh, m) in pairs:
         hk = fo.compress(Kh, m, w.S, w.R, w.k)
         hv = fo.compress(Vh, m, w.S, w.R, w.k)
         fo.decode(qh, hk, hv)
-    return (time.perf_counter() - t0) / len(K_pairs)
+    t_pairs = time.perf_counter() - t0
+    return t_basis + t_pairs / len(pairs) * (w.B * w.Hkv)
+
+
+def oracle_sample_note(w, n_pairs):
+    n_units = w.B * w.Hkv
+    return (f"{n_pairs} of {n_units} (batch, KV head) pairs per step (fp64 compress of K and V + "
+            f"decode), scaled x{n_units / n_pairs:g}, plus one basis build per step (the oracle's "
+            f"basis cache cleared before every step)")
 
 
 def blas_threads():
@@ -245,23 +322,24 @@ def run_reference(args):
     if not prints_line(rank):
         return  # the reference arm runs on rank 0 alone
     w = workload_by_name(args.workload)
-    pairs = host_pairs(w, 1)
-    n_units = w.B * w.Hkv
+    if args.batch > 0:
+        import workloads as wl
+        w = wl.shrink(w, B=args.batch)
+    pairs = host_pairs(w, ORACLE_PAIRS)
     for _ in range(args.warmup):
-        oracle_sample(w, *zip(*pairs))
-    times = [oracle_sample(w, *zip(*pairs)) for _ in range(args.steps)]
-    us = statistics.mean(times) * n_units * 1e6
+        oracle_step_seconds(w, pairs)
+    times = [oracle_step_seconds(w, pairs) for _ in range(args.steps)]
+    us = statistics.mean(times) * 1e6
     cores = blas_threads()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {
         "impl": "reference", "metric": METRIC, "value": us, "unit": "us/step",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": us / 1e3,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.L, "k": w.k,
-                   "S": w.S, "R": w.R, "parallelism": "host"},
+        "config": config_dict(w, world),
         "cpu_baseline": {"value": us, "unit": "us/step", "cores": cores, "kind": "oracle",
-                         "sample": f"1 of {n_units} (batch, KV head) pairs per step, fp64 "
-                                   f"compress K+V + decode, scaled x{n_units}"},
+                         "sample": oracle_sample_note(w, len(pairs))},
         "e2e": {"value": us, "unit": "us/step", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -269,8 +347,160 @@ def run_reference(args):
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def roofline_entry(kind, bytes_, flops, ms, peaks, peak_src, kernel, traffic=None):
+    """A roofline object: HBM-bound unless the path's arithmetic intensity is above the
+    ridge of the bf16 tensor peak over the HBM peak (compress at large k)."""
+    hbm = peaks["hbm_gbs"]
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    ridge = tc * 1e12 / (hbm * 1e9)
+    gbs = bytes_ / (ms * 1e-3) / 1e9
+    tfl = flops / (ms * 1e-3) / 1e12
+    if kind == "compress" and flops / bytes_ >= ridge:
+        roof = {"bound": "tensor", "achieved": tfl, "peak": tc, "unit": "TFLOP/s", "frac": tfl / tc}
+    else:
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+    roof.update({"kernel": kernel, "traffic": traffic,
+                 "algorithmic_bytes": bytes_,
+                 "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)"
+                                 if peak_src == "measured" else
+                                 "fallback (6.65 TB/s, 1.59 PFLOP/s: no MEASURED_PEAKS.json)")})
+    return roof
+
+
+def timed_loop(fn, stream, min_s=0.6, max_iter=4000):
+    """Average device time (ms) of fn() over a loop of back-to-back calls lasting about
+    min_s seconds (long enough for the clock sampler), CUDA events on ``stream``."""
+    import torch
+    t_one = _time(fn, 3, stream)
+    n = int(min(max_iter, max(10, min_s * 1e3 / max(t_one, 1e-3))))
+    return _time(fn, n, stream), n
+
+
+def measure_workload(w, dev, stream, peaks, peak_src, gpu_index):
+    """Per-workload figures for the bench line: compress and decode timed in loops of
+    about 0.6 s each (decode also as CUDA-graph replays), with the SM clocks sampled during
+    each loop."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+    mask = wl.dim_mask(w)
+    K = wl.kv_cache(w, "K", device=dev)
+    V = wl.kv_cache(w, "V", device=dev)
+    q = wl.queries(w, device=dev)
+    plan = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    cache = fa.Cache(plan, device=dev)
+    phiT = torch.empty(w.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(fa.fa_decode_workspace_size(plan), dtype=torch.uint8, device=dev)
+    out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+    fa.fa_build_basis(plan.P, w.k, phiT, plan.phi_ld, False, stream)
+    comp = lambda: fa.fa_compress(plan, K, V, phiT, cache, stream)
+    dec = lambda: fa.fa_decode(plan, q, cache, out, ws, 0, stream)
+    for f in (comp, dec):
+        f(); f(); f()
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.25)
+    t_c, n_c = timed_loop(comp, stream)
+    t_d, n_d = timed_loop(dec, stream)
+    rows = sampler.stop()
+    t_dg = _time_graph(lambda s: fa.fa_decode(plan, q, cache, out, ws, 0, s), max(10, n_d // 4))
+    fa.fa_device_status(stream)
+    wm = work_model(w, plan)
+    rc = roofline_entry("compress", wm["compress_bytes_alg"], wm["compress_flops"], t_c, peaks,
+                        peak_src, "fa_compress")
+    rd = roofline_entry("decode", wm["decode_bytes_alg"], wm["decode_flops"], t_d, peaks,
+                        peak_src, "fa_decode")
+    rdg = roofline_entry("decode", wm["decode_bytes_alg"], wm["decode_flops"], t_dg, peaks,
+                         peak_src, "fa_decode")
+    hbm = peaks["hbm_gbs"]
+    tcp = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    res = {
+        "shape": {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "L": w.L, "S": w.S, "R": w.R, "k": w.k},
+        "fa_compress": {"us": t_c * 1e3, "iterations": n_c,
+                        "tflops": wm["compress_flops"] / t_c / 1e9,
+                        "frac_tensor": wm["compress_flops"] / t_c / 1e9 / tcp,
+                        "hbm_gbs": wm["compress_bytes_alg"] / t_c / 1e6,
+                        "frac_hbm": wm["compress_bytes_alg"] / t_c / 1e6 / hbm,
+                        "bound": rc["bound"], "frac_of_bound": rc["frac"]},
+        "fa_decode": {"us": t_d * 1e3, "iterations": n_d, "us_graph_replay": t_dg * 1e3,
+                      "path": decode_path(w, plan),
+                      "hbm_gbs": wm["decode_bytes_alg"] / t_d / 1e6, "frac_hbm": rd["frac"],
+                      "frac_hbm_graph_replay": rdg["frac"],
+                      "algorithmic_bytes": wm["decode_bytes_alg"]},
+        "clocks": summarize_clocks(rows),
+    }
+    del K, V, q, cache, phiT, ws, out
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_layers(B, L, dev, stream, peaks, gpu_index, layers=32):
+    """One point of the 32-layer LLaMA-3-8B cache: fa_compress of every layer (distinct
+    seeded masks) and one decode step over all layers (32 fa_decode calls), each timed in
+    loops of about 0.6 s, clocks sampled."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+    w0 = wl.llama3_8b_layer(B, L, 0)
+    K = wl.kv_cache(w0, "K", device=dev)
+    V = wl.kv_cache(w0, "V", device=dev)
+    q = wl.queries(w0, device=dev)
+    plans, caches, wms = [], [], []
+    phiT = None
+    for layer in range(layers):
+        wlay = wl.llama3_8b_layer(B, L, layer)
+        plan = fa.fa_plan_init(B, 32, 8, L, wlay.S, wlay.R, wlay.k, wl.dim_mask(wlay))
+        plans.append(plan)
+        caches.append(fa.Cache(plan, device=dev))
+        wms.append(work_model(wlay, plan))
+        if phiT is None:
+            phiT = torch.empty(wlay.k, plan.phi_ld, dtype=torch.bfloat16, device=dev)
+            fa.fa_build_basis(plan.P, wlay.k, phiT, plan.phi_ld, False, stream)
+
+    def comp():  # the K / V of every layer are one synthetic draw; the masks differ
+        for p, c in zip(plans, caches):
+            fa.fa_compress(p, K, V, phiT, c, stream)
+    ws = torch.empty(max(fa.fa_decode_workspace_size(p) for p in plans), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty(B, 32, 128, dtype=torch.bfloat16, device=dev)
+
+    def dec(s=stream):
+        for p, c in zip(plans, caches):
+            fa.fa_decode(p, q, c, out, ws, 0, s)
+    comp(); dec()
+    sampler = ClockSampler(gpu_index)
+    sampler.start()
+    time.sleep(0.25)
+    t_c, n_c = timed_loop(comp, stream)
+    t_d, n_d = timed_loop(dec, stream)
+    rows = sampler.stop()
+    t_dg = _time_graph(dec, max(5, n_d // 4))
+    fa.fa_device_status(stream)
+    hbm = peaks["hbm_gbs"]
+    tcp = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    cfl = sum(m["compress_flops"] for m in wms)
+    cby = sum(m["compress_bytes_alg"] for m in wms)
+    dby = sum(m["decode_bytes_alg"] for m in wms)
+    res = {
+        "shape": {"layers": layers, "B": B, "Hq": 32, "Hkv": 8, "L": L, "S": w0.S, "R": w0.R,
+                  "k": w0.k},
+        "fa_compress": {"us": t_c * 1e3, "iterations": n_c, "tflops": cfl / t_c / 1e9,
+                        "frac_tensor": cfl / t_c / 1e9 / tcp, "hbm_gbs": cby / t_c / 1e6,
+                        "frac_hbm": cby / t_c / 1e6 / hbm},
+        "fa_decode": {"us": t_d * 1e3, "iterations": n_d, "us_graph_replay": t_dg * 1e3,
+                      "path": decode_path(w0, plans[0]), "hbm_gbs": dby / t_d / 1e6,
+                      "frac_hbm": dby / t_d / 1e6 / hbm,
+                      "frac_hbm_graph_replay": dby / t_dg / 1e6 / hbm, "algorithmic_bytes": dby},
+        "clocks": summarize_clocks(rows),
+    }
+    del K, V, q, caches, plans, ws, out, phiT
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args):
-    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -394,64 +624,70 @@ def run_ours(args):
         e2e_us = e2e_ms * 1e3
         h2d = Kh.numel() * 2 + Vh.numel() * 2 + qh.numel() * 2
         d2h = oh.numel() * 2
+        del Kh, Vh, Kd, Vd
+    else:
+        del K, V
+    del cache, ws
+    torch.cuda.empty_cache()
 
     # ---------------------------------------------------------------- roofline
     wm = work_model(w, plan)
     peaks, peak_src = load_peaks()
     hbm = peaks["hbm_gbs"]
     tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    ridge = tc * 1e12 / (hbm * 1e9)
-    c_ai = wm["compress_flops"] / wm["compress_bytes"]
-    c_gbs = wm["compress_bytes"] / (comp_ms * 1e-3) / 1e9
-    c_tflops = wm["compress_flops"] / (comp_ms * 1e-3) / 1e12
-    d_gbs = wm["decode_bytes"] / (dec_ms * 1e-3) / 1e9
-    d_tflops = wm["decode_flops"] / (dec_ms * 1e-3) / 1e12
     traffic = compress_traffic()
-    if c_ai < ridge:
-        roof = {"bound": "hbm", "achieved": c_gbs, "peak": hbm, "unit": "GB/s", "frac": c_gbs / hbm}
-    else:
-        roof = {"bound": "tensor", "achieved": c_tflops, "peak": tc, "unit": "TFLOP/s",
-                "frac": c_tflops / tc}
-    roof.update({"kernel": "fa_compress (compress_kernel + copy_sink_recent_kernel)",
-                 "traffic": (traffic["bytes_per_launch_scaled"] if traffic else None),
-                 "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs / bf16_tflops)"
-                 if peak_src == "measured" else "fallback"})
+    roof = roofline_entry("compress", wm["compress_bytes_alg"], wm["compress_flops"], comp_ms,
+                          peaks, peak_src, "fa_compress (compress_kernel + copy_sink_recent_kernel)",
+                          traffic["bytes_per_launch_scaled"] if traffic else None)
+    roof_dec = roofline_entry("decode", wm["decode_bytes_alg"], wm["decode_flops"], dec_ms, peaks,
+                              peak_src, "fa_decode (prologue + %s + combine)" % decode_path(w, plan),
+                              decode_traffic())
+    c_gbs = wm["compress_bytes_alg"] / (comp_ms * 1e-3) / 1e9
+    c_tflops = wm["compress_flops"] / (comp_ms * 1e-3) / 1e12
+    d_gbs = wm["decode_bytes_alg"] / (dec_ms * 1e-3) / 1e9
 
     line = {
         "metric": METRIC, "value": ms_step * 1e3, "unit": "us/step", "n_gpus": world,
         "steps": args.steps, "warmup": max(args.warmup, 3), "ms_per_step": ms_step,
         "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": w.name, "global_batch": w.B * world, "seq_len": w.L,
-                   "Hq": w.Hq, "Hkv": w.Hkv, "k": w.k, "S": w.S, "R": w.R,
-                   "dims_compressed_per_head": int(plan.dc[0]), "parallelism": f"replica x{world}",
-                   "l2": "inputs larger than L2 (K+V %.2f GB, E %.2f GB per step)" % (
-                       2 * K_bytes(w) / 1e9, 2 * plan.e_elems * 2 / 1e9)},
+        "config": config_dict(base, world),
         "components": {
             "fa_build_basis": {"us": basis_ms * 1e3},
             "fa_compress": {"us": comp_ms * 1e3, "tflops": c_tflops, "hbm_gbs": c_gbs,
-                            "arith_intensity": c_ai, "algorithmic_bytes": wm["compress_bytes"],
+                            "algorithmic_bytes": wm["compress_bytes_alg"],
+                            "bytes_moved_fp32_C_and_F_copy": wm["compress_bytes"],
                             "algorithmic_flops": wm["compress_flops"],
                             "frac_hbm": c_gbs / hbm, "frac_tensor": c_tflops / tc},
             "fa_decode": {"us": dec_ms * 1e3, "hbm_gbs": d_gbs, "frac_hbm": d_gbs / hbm,
-                          "tflops_fp32": d_tflops, "algorithmic_bytes": wm["decode_bytes"],
+                          "path": decode_path(w, plan),
+                          "algorithmic_bytes": wm["decode_bytes_alg"],
+                          "bytes_moved_fp32_C": wm["decode_bytes"],
                           "algorithmic_flops": wm["decode_flops"]},
         },
         "roofline": roof,
+        "roofline_fa_decode": roof_dec,
         "clocks": {**summarize_clocks(rows), "note": clock_note},
         "gpu_launches": launches_per_step(w, plan) * args.steps,
         "e2e": {"value": e2e_us, "unit": "us/step", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
     }
+    if world == 1 and not args.no_configs:
+        # every single-layer workload and one point of the 32-layer cache, measured apart
+        # from the timed step above (not part of ``value``)
+        per = {}
+        for cw in wl.CONFIGS:
+            per[cw.name] = measure_workload(cw, dev, stream, peaks, peak_src, gpu_index)
+        per["llama3_8b_32_layers_b8_L32768_k255"] = measure_layers(8, 32768, dev, stream, peaks,
+                                                                  gpu_index)
+        line["per_workload"] = per
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        pairs = host_pairs(base, 2)
-        n_units = base.B * base.Hkv
-        per_pair = oracle_sample(base, *zip(*pairs))
+        pairs = host_pairs(base, ORACLE_PAIRS)
+        est = [oracle_step_seconds(base, pairs) for _ in range(3)]
         line["cpu_baseline"] = {
-            "value": per_pair * n_units * 1e6, "unit": "us/step", "cores": blas_threads(),
+            "value": statistics.mean(est) * 1e6, "unit": "us/step", "cores": blas_threads(),
             "kind": "oracle",
-            "sample": f"2 of {n_units} (batch, KV head) pairs (fp64 compress K+V + decode), "
-                      f"scaled x{n_units / 2:g}"}
+            "sample": oracle_sample_note(base, len(pairs)) + "; mean of 3 sampled steps"}
     if prints_line(rank):
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -228,10 +228,22 @@ static int decode_checks(const fa_plan* plan) {
   return FA_OK;
 }
 
+}  // extern "C"
+
+int fa::decode_setup(const fa_plan* plan, int requested, fa::DecodeConfig* c) {
+  if (int r = decode_checks(plan)) return r;
+  const char* why = nullptr;
+  cudaError_t e = fa::decode_configure(plan, requested, c, &why);
+  if (e == cudaSuccess) return FA_OK;
+  if (why) return fail(FA_ERR_UNSUPPORTED, "fa_decode: %s", why);
+  return cuda_fail(e, "fa_decode: configure");
+}
+
+extern "C" {
+
 size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits) {
-  if (decode_checks(plan) != FA_OK) return 0;
   fa::DecodeConfig c;
-  if (fa::decode_configure(plan, num_splits, &c) != cudaSuccess) return 0;
+  if (fa::decode_setup(plan, num_splits, &c) != FA_OK) return 0;
   return c.qw_bytes + c.rec_bytes;
 }
 
@@ -252,13 +264,12 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
   if (int r = check_ptr(cache->C_V, "cache->C_V", plan->c_elems > 0)) return r;
   if (int r = check_ptr(workspace, "workspace", true)) return r;
   fa::DecodeConfig c;
-  cudaError_t e = fa::decode_configure(plan, num_splits, &c);
-  if (e != cudaSuccess) return cuda_fail(e, "fa_decode: configure");
+  if (int r = fa::decode_setup(plan, num_splits, &c)) return r;
   if (workspace_bytes < c.qw_bytes + c.rec_bytes)
     return fail(FA_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
                 workspace_bytes, c.qw_bytes + c.rec_bytes);
-  e = fa::launch_decode(plan, c, q, cache, out, out_dtype, workspace,
-                        static_cast<cudaStream_t>(stream));
+  cudaError_t e = fa::launch_decode(plan, c, q, cache, out, out_dtype, workspace,
+                                    static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "fa_decode: launch");
   return FA_OK;
 }
@@ -292,9 +303,7 @@ static int sensitivity_setup(const fa_shape* shape, fa_plan* plan, fa::DecodeCon
                              size_t* bytes) {
   if (!shape) return fail(FA_ERR_INVALID, "shape is NULL");
   if (int r = fa::sensitivity_plan(shape, plan)) return r;  // fa_plan_init set the message
-  if (int r = decode_checks(plan)) return r;
-  cudaError_t e = fa::decode_configure(plan, 0, c);
-  if (e != cudaSuccess) return cuda_fail(e, "fa_dim_sensitivity: configure");
+  if (int r = fa::decode_setup(plan, 0, c)) return r;
   *bytes = fa::sensitivity_out_offset(*c) +
            (size_t)plan->shape.B * plan->shape.Hq * FA_HEAD_DIM * sizeof(float);
   return FA_OK;

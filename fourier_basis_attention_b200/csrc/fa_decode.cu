@@ -725,8 +725,10 @@ static cudaError_t occupancy(int* blocks, size_t smem) {
 }
 
 // Derive the launch configuration. `requested` <= 0 selects the split count from a
-// wave-quantisation cost model for the current device.
-cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c) {
+// wave-quantisation cost model for the current device. A plan the kernels cannot serve
+// returns cudaErrorInvalidValue with *why naming the limit.
+cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c,
+                             const char** why) {
   const fa_shape& sh = plan->shape;
   const int M = plan->M;
   c->F = sh.k / 2 + 1;
@@ -803,6 +805,11 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
     const long long nfs = (plan->S + plan->R + FT - 1) / FT;
     const long long fixed = (long long)combine_smem_floats(plan->G, 0, FA_HEAD_DIM + 2 * c->F_pad) + 4;
     const long long ns_max = ((227 * 1024) / 4 - fixed) / plan->G - nfs;
+    if (ns_max < 1) {
+      // the sink / recent records alone fill the combine's shared memory
+      if (why) *why = "too many sink + recent rows for the combine (S + R too large for this k and G)";
+      return cudaErrorInvalidValue;
+    }
     if (ns > ns_max) ns = (int)ns_max;
     const int per = (ntiles + ns - 1) / ns;
     c->n_splits = (ntiles + per - 1) / per;
@@ -826,7 +833,11 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
     c->cb_gt = gt;
   }
   c->smem_combine = combine_smem_floats(c->cb_gt, c->n_rec, c->rec_stride - 4) * 4;
-  return c->smem_combine <= 227 * 1024 ? cudaSuccess : cudaErrorInvalidValue;
+  if (c->smem_combine > 227 * 1024) {
+    if (why) *why = "the combine's shared memory would exceed 227 KB (too many split records)";
+    return cudaErrorInvalidValue;
+  }
+  return cudaSuccess;
 }
 
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,

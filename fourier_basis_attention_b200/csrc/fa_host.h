@@ -23,7 +23,11 @@ cudaError_t launch_build_basis(int M, int k, long long ld, int dtype, int normal
 cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
                             const void* phiT, const fa_cache* cache, cudaStream_t stream,
                             const char** why);
-cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c);
+cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c,
+                             const char** why = nullptr);
+// Decode checks + configuration as the entry points run them: FA_OK, or a status with
+// fa_last_error() set (argument checks, unsupported shapes, configuration limits).
+int decode_setup(const fa_plan* plan, int requested, DecodeConfig* c);
 cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void* q,
                           const fa_cache* cache, void* out, int out_dtype, void* workspace,
                           cudaStream_t stream);

@@ -19,10 +19,35 @@ constexpr int kMaxDevices = 64;
 // its device address comes from cudaGetSymbolAddress (see scratch_address below).
 static __device__ __align__(256) unsigned char g_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_mu;
-void* g_addr[kMaxDevices] = {};
+typedef int (*PFN_ctxGetCurrent)(void** ctx);  // CUresult cuCtxGetCurrent(CUcontext*)
 
-// Device address of g_scratch on the current device, looked up once per device.
+std::mutex g_mu;
+struct ScratchEntry {
+  void* ctx;   // the CUDA context the address belongs to
+  void* addr;  // device address of g_scratch in that context
+};
+ScratchEntry g_addr[kMaxDevices] = {};
+
+// Current CUDA context (the driver's handle), or nullptr if it cannot be read.
+void* current_context() {
+  static PFN_ctxGetCurrent fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_ctxGetCurrent>(p);
+    looked = true;
+  }
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of g_scratch on the current device. It is looked up once per device and
+// context: after cudaDeviceReset the library's module is loaded into a new context with a
+// new address, so a changed context handle triggers a fresh lookup.
 int scratch_address(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -30,7 +55,9 @@ int scratch_address(void** out) {
   if (dev < 0 || dev >= kMaxDevices)
     return fa::set_last_error(FA_ERR_UNSUPPORTED, "fa_decode_noalloc: device index out of range");
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_addr[dev]) {
+  void* ctx = current_context();
+  ScratchEntry& ent = g_addr[dev];
+  if (!ent.addr || !ctx || ent.ctx != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_scratch);
     if (e != cudaSuccess || !p) {
@@ -39,9 +66,11 @@ int scratch_address(void** out) {
                cudaGetErrorString(e));
       return fa::set_last_error(FA_ERR_CUDA, msg);
     }
-    g_addr[dev] = p;
+    // the context handle is read after the lookup, which may have created the context
+    ent.ctx = current_context();
+    ent.addr = p;
   }
-  *out = g_addr[dev];
+  *out = ent.addr;
   return FA_OK;
 }
 
@@ -50,20 +79,15 @@ int scratch_address(void** out) {
 extern "C" int fa_decode_noalloc(const fa_plan* plan, const void* q, const fa_cache* cache,
                                  void* out, int32_t out_dtype, int32_t num_splits,
                                  void* stream) {
-  size_t need = fa_decode_workspace_size(plan, num_splits);
-  if (need == 0) {
-    // unusable plan: let fa_decode report the precise reason
-    return fa_decode(plan, q, cache, out, out_dtype, nullptr, 0, num_splits, stream);
-  }
+  fa::DecodeConfig c;
+  if (int r = fa::decode_setup(plan, num_splits, &c)) return r;  // precise reason recorded
+  size_t need = c.qw_bytes + c.rec_bytes;
   int splits = num_splits;
   if (need > FA_NOALLOC_SCRATCH_BYTES && num_splits <= 0) {
     // lower the automatic split count until the partial records fit
-    fa::DecodeConfig c;
-    if (fa::decode_configure(plan, 0, &c) != cudaSuccess)
-      return fa::set_last_error(FA_ERR_CUDA, "fa_decode_noalloc: configure failed");
     for (splits = c.n_splits - 1; splits >= 1; --splits) {
       need = fa_decode_workspace_size(plan, splits);
-      if (need <= FA_NOALLOC_SCRATCH_BYTES) break;
+      if (need != 0 && need <= FA_NOALLOC_SCRATCH_BYTES) break;
     }
     if (splits < 1) splits = 1;
   }

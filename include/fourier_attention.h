@@ -244,7 +244,11 @@ int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* o
  *   Calls no cudaMalloc / cudaFree and no allocating library routine.
  *   Set-up: the first call on each device (with that device current) looks up the
  *   device address of the scratch array; make that first call before any stream
- *   capture begins.
+ *   capture begins. The address is kept per device and CUDA context: after
+ *   cudaDeviceReset the next call looks it up again (in the new context), so that call
+ *   too belongs before any capture.
+ *   Errors: the plan checks and configuration limits of fa_decode, reported with their
+ *   own message.
  *   All calls in the process share one scratch array per device and it keeps the last
  *   call's contents; the kernels write every scratch word before reading it, so nothing
  *   needs clearing. Calls whose kernels overlap on the same GPU (different streams, no

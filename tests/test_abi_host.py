@@ -155,6 +155,22 @@ def test_decode_rejects_unsupported_group_and_k():
     assert fa.fa_decode_workspace_size(p, 4) > 0
 
 
+def test_decode_rejects_too_many_sink_recent_records():
+    """S + R so large that the combine's sink/recent record weights alone fill its shared
+    memory: the size query answers 0 and both decode entry points return
+    FA_ERR_UNSUPPORTED with the reason (host checks only; nothing is launched)."""
+    p = fa.fa_plan_init(1, 8, 1, 32 + 460000 + 2048, 32, 460000, 1023, np.ones((1, 128)))
+    assert p.M == 2048
+    assert fa.fa_decode_workspace_size(p, 1) == 0
+    cache = fa.fa_cache(0x1000, 0x1000, 0x1000, 0x1000, 0x1000, 0x1000)
+    r = fa.LIB.fa_decode(ctypes.byref(p), 0x1000, ctypes.byref(cache), 0x1000, fa.FA_F32,
+                         0x1000, 1 << 30, 1, None)
+    assert r == fa.FA_ERR_UNSUPPORTED and "sink + recent" in fa.fa_last_error()
+    r = fa.LIB.fa_decode_noalloc(ctypes.byref(p), 0x1000, ctypes.byref(cache), 0x1000,
+                                 fa.FA_F32, 1, None)
+    assert r == fa.FA_ERR_UNSUPPORTED and "sink + recent" in fa.fa_last_error()
+
+
 def test_workspace_size_formula():
     w = wl.LLAMA2_7B_MHA_32K
     p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))

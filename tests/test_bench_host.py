@@ -29,6 +29,34 @@ def test_work_model_bench_workload_by_hand():
     assert wm["compress_bytes"] == 5428281344 and wm["decode_bytes"] == 1133445120
 
 
+def test_algorithmic_bytes_are_the_method_minimum_by_hand():
+    """The method's minimum bytes (bf16 coefficients; compress reads the middle rows once
+    and writes C and E; decode reads F, E and C of K and V, the queries, writes out):
+    decode 4 B Hkv [(S+R) D + M De + k Dc] + q + out, compress 4 B Hkv (M D + k Dc + M De)."""
+    w = wl.LLAMA2_7B_MHA_32K
+    wm = bench.work_model(w, _plan(w))
+    B, Hkv, D, M, k, SR = 8, 32, 128, 32768 - 96, 255, 96
+    assert wm["decode_bytes_alg"] == 4 * B * Hkv * (SR * D + M * 32 + k * 96) + 2 * 2 * B * 32 * D
+    assert wm["compress_bytes_alg"] == 4 * B * Hkv * (M * D + k * 96 + M * 32)
+    assert wm["compress_bytes_alg"] == 5378048000 and wm["decode_bytes_alg"] == 1108377600
+    # no middle span: nothing to project, decode reads only the sink / recent rows
+    w0 = wl.shrink(w, B=1, Hq=2, Hkv=2, L=90)
+    wm0 = bench.work_model(w0, _plan(w0))
+    assert wm0["compress_flops"] == 0 and wm0["compress_bytes_alg"] == 0
+    assert wm0["decode_bytes_alg"] == 4 * 2 * 90 * 128 + 2 * 2 * 2 * 128
+
+
+def test_config_dict_is_shared_by_both_arms():
+    """Both arms print config_dict(workload, world): the same keys and values."""
+    w = wl.LLAMA3_8B_GQA_32K
+    c = bench.config_dict(w, 1)
+    assert c == bench.config_dict(w, 1)
+    assert c["dims_compressed_per_head"] == [64, 96] and c["workload"] == w.name
+    assert bench.config_dict(wl.LLAMA2_7B_MHA_32K)["dims_compressed_per_head"] == 96
+    assert bench.config_dict(wl.SINGLE_HEAD_2K)["l2"].startswith("inputs fit in L2")
+    assert "reference" not in c and c["parallelism"] == "replica x1"
+
+
 def test_launches_per_step_each_path():
     """6 launches on the tensor-core and warp-MMA paths (sink / recent rows ride in the
     prologue launch) and on the CUDA-core path (they ride in the split kernel)."""

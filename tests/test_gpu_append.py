@@ -163,11 +163,15 @@ def test_append_until_full_then_refused():
     fa.fa_device_status()
 
 
-@pytest.mark.parametrize("w", [wl.LLAMA2_7B_MHA_32K, wl.LLAMA3_8B_GQA_128K], ids=lambda w: w.name)
-def test_append_full_size_sampled_heads(w):
-    """The bench-sized caches (tensor-core and warp-MMA decode paths): 16 appends, then the
-    first and last (batch, KV head) against the oracle of the longer sequence."""
-    p, cache, K, V = run_append(w, 16, 8, heads=[(0, 0), (w.B - 1, w.Hkv - 1)], gen_device="cuda")
-    assert p.M == w.L - w.S - w.R + 16
+@pytest.mark.parametrize("w,n_app", [(wl.LLAMA2_7B_MHA_32K, 16), (wl.LLAMA3_8B_GQA_128K, 16),
+                                       (wl.llama3_8b_layer(64, 131072, 30), 1)],
+                         ids=lambda x: getattr(x, "name", str(x)))
+def test_append_full_size_sampled_heads(w, n_app):
+    """The bench-sized caches and the largest point of the 32-layer cache (B = 64,
+    L = 128K): appends, then the first and last (batch, KV head) against the oracle of the
+    longer sequence."""
+    p, cache, K, V = run_append(w, n_app, 8, heads=[(0, 0), (w.B - 1, w.Hkv - 1)],
+                                gen_device="cuda")
+    assert p.M == w.L - w.S - w.R + n_app
     idx = [p.S + (p.recent_head + a) % p.R for a in range(p.R)]
     assert torch.equal(cache.F("K")[:, :, idx], K[:, :, p.shape.L - p.R:])

@@ -310,8 +310,25 @@ def test_repeat_calls_are_deterministic():
 
 # ----------------------------------------------------------------------------- full-size workloads
 
+def sample_pairs(w):
+    """Four distinct (batch row, KV head) pairs spread over the cache: the first, the last
+    (largest offsets into every buffer), and two between them."""
+    cand = [(0, 0), (w.B - 1, w.Hkv - 1), (w.B // 2, w.Hkv // 2), (w.B - 1, 0),
+            (0, w.Hkv - 1), ((w.B - 1) // 3, 1 % w.Hkv), (0, 1 % w.Hkv)]
+    out = []
+    for c in cand:
+        if c not in out:
+            out.append(c)
+    return out[:4]
+
+
+# The single-layer workloads at full size, and points of the 32-layer LLaMA-3-8B cache
+# sweep: B = 8 at L = 32K (tensor-core decode), B = 64 at L = 128K (k = 1023; E offsets of
+# the last batch row near 2^31 elements), B = 64 at L = 8K (k = 63, CUDA-core decode) and
+# B = 1 at L = 32K (32 query heads, CUDA-core decode).
 FULL = [wl.LLAMA2_7B_MHA_32K, wl.LLAMA3_8B_GQA_32K, wl.LLAMA3_8B_GQA_128K,
-        wl.llama3_8b_layer(8, 32768, 3)]
+        wl.llama3_8b_layer(8, 32768, 3), wl.llama3_8b_layer(64, 131072, 31),
+        wl.llama3_8b_layer(64, 8192, 17), wl.llama3_8b_layer(1, 32768, 9)]
 
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
@@ -321,13 +338,15 @@ def test_full_size_sampled_heads(w):
     V = wl.kv_cache(w, "V", device="cuda")
     q = wl.queries(w, device="cuda")
     p, cache, out = run_path(w, K, V, q, mask)
-    for b, g in [(0, 0), (w.B - 1, w.Hkv - 1)]:
+    for b, g in sample_pairs(w):
         check_head(w, p, cache, out, K[b, g].cpu(), V[b, g].cpu(),
                    q[b, g * w.G:(g + 1) * w.G].cpu(), mask[g], b, g)
     # every output is finite and every head's F rows are exact copies
     assert torch.isfinite(out.float()).all().item()
     idx = torch.cat([torch.arange(p.S), torch.arange(w.L - p.R, w.L)]).cuda()
     assert torch.equal(cache.F("K"), K[:, :, idx]) and torch.equal(cache.F("V"), V[:, :, idx])
+    del cache, K, V
+    torch.cuda.empty_cache()
 
 
 # ----------------------------------------------------------------------------- failure detection

@@ -2,7 +2,9 @@
 
 The oracle runs the skill page's loop (one perturbed attention per dim, values perturbed);
 the library uses one attention pass over (K, noise). Scores meet the 3e-3 bound per KV
-head; the selected masks agree wherever the choice is decided by more than that bound.
+head; the mask selected from the GPU scores is a valid selection under the oracle's scores
+(no compressed dim scores above a retained one by more than the bound), which makes it
+the oracle's mask wherever the oracle's cut is wider than the bound.
 """
 import numpy as np
 import pytest
@@ -27,14 +29,17 @@ def gpu_scores(q, K, noise):
 
 
 def check_masks_agree(sg, so, n_compressed):
-    """Masks from GPU and oracle scores may differ only where the oracle's scores of the
-    swapped dims lie within the tolerance of each other."""
+    """The mask selected from the GPU scores is a valid selection under the oracle's
+    scores: every dim it compresses scores (by the oracle) no higher than every dim it
+    retains, up to the score tolerance. Where the oracle's scores separate the two sets
+    by more than that tolerance, this forces the masks to be identical."""
     mg = fo.select_dims(sg, n_compressed)
-    mo = fo.select_dims(so, n_compressed)
-    diff = np.nonzero(mg != mo)[0]
-    if diff.size:
-        cut = np.sort(so)[n_compressed - 1:n_compressed + 1]
-        assert np.all(np.abs(so[diff] - cut.mean()) <= TOL * so.max() + np.ptp(cut)), diff
+    comp, kept = so[mg == 1], so[mg == 0]
+    if comp.size and kept.size:
+        assert comp.max() <= kept.min() + TOL * so.max(), (comp.max(), kept.min())
+    srt = np.sort(so)
+    if 0 < n_compressed < so.size and srt[n_compressed] - srt[n_compressed - 1] > TOL * so.max():
+        assert np.array_equal(mg, fo.select_dims(so, n_compressed))
 
 
 @pytest.mark.parametrize("G,L", [(4, 700), (1, 300), (8, 1000), (2, 1)], ids=str)
@@ -66,3 +71,4 @@ def test_sensitivity_full_size_sampled_heads():
         so = fo.dim_sensitivity(q[:, g:g + 1].double().cpu().numpy(), Kg, np.zeros_like(Kg),
                                 n[:, g].double().cpu().numpy())
         assert np.abs(sg[g] - so).max() <= TOL * so.max()
+        check_masks_agree(sg[g], so, 96)

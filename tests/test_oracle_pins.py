@@ -471,3 +471,21 @@ def test_period_hand_example(hand_cases):
     x3 = np.array(hand_cases["period4_x_appended"])[:, None]
     h3 = fo.compress(x3, np.ones(1), 0, 0, 4, period=4)
     assert np.abs(h3.C[:, 0] - hand_cases["period4_C_appended"]).max() < 1e-15
+
+
+def test_mask_agreement_check_rejects_a_swap_across_a_wide_cut():
+    """The GPU mask check (tests/test_gpu_sensitivity.py) must reject a selection that swaps
+    two dims whose oracle scores differ by more than the tolerance, and accept one that
+    swaps only dims tied within it. The mistake is planted in the scores on the CPU."""
+    from test_gpu_sensitivity import TOL, check_masks_agree
+    so = np.linspace(1.0, 2.0, 128)            # cut gaps 1/127 > TOL * max
+    check_masks_agree(so.copy(), so, 96)
+    swapped = so.copy()
+    swapped[[95, 96]] = swapped[[96, 95]]       # dim 96 compressed, dim 95 retained
+    with pytest.raises(AssertionError):
+        check_masks_agree(swapped, so, 96)
+    tied = so.copy()
+    tied[96] = tied[95] + 0.5 * TOL * tied.max()
+    near = tied.copy()
+    near[[95, 96]] = near[[96, 95]]
+    check_masks_agree(near, tied, 96)

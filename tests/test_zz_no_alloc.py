@@ -48,6 +48,10 @@ def _reference(p, cache, q, w, num_splits):
 ], ids=["small_auto", "small_forced_splits", "llama2_7b_full_auto"])
 def test_noalloc_matches_fa_decode_on_two_calls(w, num_splits):
     p, cache, q = _setup(w)
+    if w is wl.LLAMA2_7B_MHA_32K:
+        # the automatic split count's records exceed the built-in scratch here, so this
+        # case runs the branch that lowers the split count until they fit
+        assert fa.fa_decode_workspace_size(p, 0) > fa.NOALLOC_SCRATCH_BYTES
     ref = _reference(p, cache, q, w, num_splits)
     scale = ref.abs().max().item()
     for call in range(2):
