@@ -105,14 +105,11 @@ def work_model(w, plan):
 
 
 def decode_path(w, plan):
-    """Which split kernel fa_decode runs for this plan (mirrors the library's choice)."""
-    if plan.M == 0:
-        return "none (no middle span)"
-    if plan.e_token_major:
-        return "tcgen05 (decode_tc_kernel)"
-    if 256 <= w.k <= 1023:
-        return "warp MMA (decode_hmma_kernel)"
-    return "CUDA cores (decode_main_kernel)"
+    """Which split kernel fa_decode runs for this plan (the library's own answer)."""
+    import fourier_basis_attention_b200 as fa
+    info = fa.fa_decode_describe(plan, 1)
+    name = fa.SPLIT_KERNELS[info.split_kernel]
+    return name + (f", clusters of {info.cluster}" if info.cluster > 1 else "")
 
 
 def config_dict(w, world=1):
@@ -696,20 +693,12 @@ def run_ours(args):
 
 
 def launches_per_step(w, plan):
-    """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel and
-    compress_kernel; then fa_decode's prologue (middle span present; on the tensor-core and
-    warp-MMA paths its launch also runs the sink / recent rows), the split kernel (the
-    tensor-core one when the plan laid E out token-major, the warp-MMA one for other plans
-    with 256 <= k <= 1023, else the CUDA-core one, which then also runs the sink / recent
-    rows), and the combine."""
-    n = 1 + 2
-    n += 1 if plan.M > 0 else 0          # prologue (+ sink / recent rows)
-    hm = plan.M > 0 and not plan.e_token_major and 256 <= w.k <= 1023
-    if (plan.e_token_major or hm) and plan.M > 0:
-        n += 1                           # tensor-core or warp-MMA split kernel
-    elif plan.M > 0 or plan.S + plan.R > 0:
-        n += 1                           # CUDA-core split kernel (+ sink / recent rows)
-    return n + 1                         # combine
+    """Kernels one step launches: build_basis_kernel; copy_sink_recent_kernel (when there
+    are sink / recent rows) and compress_kernel (when there is a middle span); then what
+    fa_decode launches (the library's count: prologue, split kernel, combine)."""
+    import fourier_basis_attention_b200 as fa
+    n = 1 + (1 if plan.S + plan.R > 0 else 0) + (1 if plan.M > 0 else 0)
+    return n + fa.fa_decode_describe(plan, 1).launches
 
 
 def K_bytes(w):

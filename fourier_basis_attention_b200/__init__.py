@@ -5,7 +5,7 @@ Argument marshalling only: every step of the hot path runs in the CUDA kernels o
 PyTorch is used for device memory and streams. The functions keep the C names:
 
     fa_plan_init, fa_plan_reserve, fa_build_basis, fa_compress, fa_decode_workspace_size,
-    fa_decode, fa_decode_noalloc, fa_append, fa_dim_sensitivity_workspace_size,
+    fa_decode_describe, fa_decode, fa_decode_noalloc, fa_append, fa_dim_sensitivity_workspace_size,
     fa_dim_sensitivity, fa_select_dims, fa_device_status, fa_last_error
 
 There is no CPU fallback: if the shared library is missing or fails to load, importing
@@ -25,11 +25,13 @@ MAX_KV_HEADS = 64
 MAX_K_DECODE = 2047
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_DEVICE = range(5)
 FA_BF16, FA_F32 = 0, 1
+(FA_SPLIT_NONE, FA_SPLIT_CUDA_CORES, FA_SPLIT_TC_TOKEN_MAJOR, FA_SPLIT_WARP_MMA,
+ FA_SPLIT_TC_CLUSTER) = range(5)
 
 EXPORTED = ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress",
             "fa_decode_workspace_size", "fa_decode", "fa_decode_noalloc", "fa_append",
             "fa_dim_sensitivity_workspace_size", "fa_dim_sensitivity", "fa_select_dims",
-            "fa_device_status", "fa_watchdog_selftest", "fa_last_error")
+            "fa_device_status", "fa_watchdog_selftest", "fa_last_error", "fa_decode_describe")
 NOISE_SCALE = 0.1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -63,6 +65,16 @@ class fa_plan(ctypes.Structure):
     ]
 
 
+class fa_decode_info(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("split_kernel", "num_splits", "cluster", "launches")]
+
+
+SPLIT_KERNELS = {0: "none (no middle span)", 1: "CUDA cores (decode_main_kernel)",
+                 2: "tcgen05, token-major E (decode_tc_kernel)",
+                 3: "warp MMA (decode_hmma_kernel)",
+                 4: "tcgen05, slot-split cluster (decode_cl_kernel)"}
+
+
 class fa_cache(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in ("F_K", "F_V", "E_K", "E_V", "C_K", "C_V")]
 
@@ -90,6 +102,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_compress.argtypes = [ctypes.POINTER(fa_plan), P, P, P, ctypes.POINTER(fa_cache), P]
     lib.fa_decode_workspace_size.argtypes = [ctypes.POINTER(fa_plan), I32]
     lib.fa_decode_workspace_size.restype = SZ
+    lib.fa_decode_describe.argtypes = [ctypes.POINTER(fa_plan), I32, ctypes.POINTER(fa_decode_info)]
     lib.fa_decode.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32, P, SZ,
                               I32, P]
     lib.fa_decode_noalloc.argtypes = [ctypes.POINTER(fa_plan), P, ctypes.POINTER(fa_cache), P, I32,
@@ -100,7 +113,7 @@ def configure(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.fa_last_error.restype = ctypes.c_char_p
     for name in ("fa_plan_init", "fa_plan_reserve", "fa_build_basis", "fa_compress", "fa_decode",
                  "fa_decode_noalloc", "fa_append", "fa_dim_sensitivity", "fa_select_dims",
-                 "fa_device_status", "fa_watchdog_selftest"):
+                 "fa_device_status", "fa_watchdog_selftest", "fa_decode_describe"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -169,6 +182,13 @@ def fa_compress(plan: fa_plan, K, V, phiT, cache: "Cache", stream=None) -> None:
 
 def fa_decode_workspace_size(plan: fa_plan, num_splits: int = 0) -> int:
     return int(LIB.fa_decode_workspace_size(ctypes.byref(plan), num_splits))
+
+
+def fa_decode_describe(plan: fa_plan, num_splits: int = 0) -> fa_decode_info:
+    """How fa_decode runs this plan: split kernel, split count, cluster size, launches."""
+    info = fa_decode_info()
+    _check(LIB.fa_decode_describe(ctypes.byref(plan), num_splits, ctypes.byref(info)))
+    return info
 
 
 def fa_decode(plan: fa_plan, q, cache: "Cache", out, workspace, num_splits: int = 0,

@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfourier_attention.so")
-SOURCES = ["fa_abi.cu", "fa_basis.cu", "fa_compress.cu", "fa_decode.cu", "fa_decode_tc.cu", "fa_decode_hmma.cu", "fa_runtime.cu", "fa_append.cu", "fa_sensitivity.cu",
+SOURCES = ["fa_abi.cu", "fa_basis.cu", "fa_compress.cu", "fa_decode.cu", "fa_decode_tc.cu", "fa_decode_hmma.cu", "fa_decode_cl.cu", "fa_runtime.cu", "fa_append.cu", "fa_sensitivity.cu",
            "fa_noalloc.cu"]
 HEADERS = ["fa_internal.cuh", "fa_host.h", "fa_decode_common.cuh"]
 PUBLIC_HEADER = os.path.join(ROOT, "include", "fourier_attention.h")

@@ -247,6 +247,25 @@ size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits) {
   return c.qw_bytes + c.rec_bytes;
 }
 
+int fa_decode_describe(const fa_plan* plan, int32_t num_splits, fa_decode_info* info) {
+  if (!info) return fail(FA_ERR_INVALID, "info is NULL");
+  fa::DecodeConfig c;
+  if (int r = fa::decode_setup(plan, num_splits, &c)) return r;
+  const bool mid = plan->M > 0;
+  info->split_kernel = !mid ? FA_SPLIT_NONE
+                       : c.tc ? FA_SPLIT_TC_TOKEN_MAJOR
+                       : c.cl ? FA_SPLIT_TC_CLUSTER
+                       : c.hm ? FA_SPLIT_WARP_MMA
+                              : FA_SPLIT_CUDA_CORES;
+  info->num_splits = c.n_splits;
+  info->cluster = c.cl ? c.cl_C : 1;
+  // prologue (with the sink / recent rows on the tensor-core and warp-MMA paths), the split
+  // kernel (with the sink / recent rows on the CUDA-core path), the combine
+  const bool split_launch = mid || plan->S + plan->R > 0;
+  info->launches = (mid ? 1 : 0) + (split_launch ? 1 : 0) + 1;
+  return FA_OK;
+}
+
 int fa_decode(const fa_plan* plan, const void* q, const fa_cache* cache, void* out,
               int32_t out_dtype, void* workspace, size_t workspace_bytes, int32_t num_splits,
               void* stream) {

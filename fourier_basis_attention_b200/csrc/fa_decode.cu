@@ -724,11 +724,62 @@ static cudaError_t occupancy(int* blocks, size_t smem) {
   return cached_occupancy(reinterpret_cast<const void*>(decode_main_kernel<SPT>), DNT, smem, blocks);
 }
 
+// Ring and buffer sizes of the cluster tensor-core kernel for a plan, cluster size C and
+// 2 F_pad slots; leaves c->cl = 0 when its buffers do not fit in shared memory.
+static void cl_configure(const fa_plan* plan, int C, int slots, DecodeConfig* c) {
+  const fa_shape& sh = plan->shape;
+  const int G = plan->G, nown = 4 / C, nkq = 32 / G;
+  const int SL = ((slots + C - 1) / C + 63) / 64 * 64;
+  // bytes one token of a ring slot takes for the worst CTA (sum of its exact KV heads'
+  // row pitches) and the number of those heads with exact dims (each padded in a slot)
+  long long worst_row = 0, worst_pad = 0;
+  const long long bhq = (long long)sh.B * sh.Hq;
+  const long long n_hs = (bhq + 127) / 128;
+  for (long long hs = 0; hs < n_hs; ++hs)
+    for (int r = 0; r < C; ++r) {
+      long long row = 0, pad = 0;
+      for (int li = 0; li < nown; ++li)
+        for (int j = 0; j < nkq; ++j) {
+          const long long gh = hs * 128 + 32 * (r * nown + li) + (long long)j * G;
+          if (gh >= bhq) continue;
+          const int g = (int)((gh % sh.Hq) / G);
+          row += 2LL * plan->de_ld[g];
+          pad += plan->de_ld[g] > 0 ? 64 : 0;
+        }
+      worst_row = row > worst_row ? row : worst_row;
+      worst_pad = pad > worst_pad ? pad : worst_pad;
+    }
+  const size_t fixed = decode_cl_smem_bytes(C, SL, 0, 0);
+  const size_t budget = 227 * 1024;
+  if (fixed >= budget) return;
+  int TB = 32;
+  int slot = 0, stages = 0;
+  for (; TB >= 8; TB >>= 1) {
+    slot = (int)((TB * worst_row + worst_pad + 127) / 128 * 128);
+    if (slot < 128) slot = 128;
+    stages = (int)((budget - fixed) / (size_t)slot);
+    if (stages > 8) stages = 8;
+    if (stages >= 3 || (TB == 8 && stages >= 2)) break;
+  }
+  if (TB < 8 || stages < 2) return;
+  int cols = 32;
+  while (cols < SL + 64 + SL / 2) cols <<= 1;
+  c->cl = 1;
+  c->cl_C = C;
+  c->cl_SL = SL;
+  c->cl_TB = TB;
+  c->cl_stages = stages;
+  c->cl_slot_bytes = slot;
+  c->cl_tmem_cols = cols;
+  c->cl_smem = (int)decode_cl_smem_bytes(C, SL, slot, stages);
+}
+
 // Derive the launch configuration. `requested` <= 0 selects the split count from a
 // wave-quantisation cost model for the current device. A plan the kernels cannot serve
 // returns cudaErrorInvalidValue with *why naming the limit.
 cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c,
                              const char** why) {
+  memset(c, 0, sizeof(*c));
   const fa_shape& sh = plan->shape;
   const int M = plan->M;
   c->F = sh.k / 2 + 1;
@@ -759,8 +810,23 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   int cols = 32;  // U (2F slots), S (2 x 32 tokens), W_lo (2F / 2 columns of slot pairs)
   while (cols < c->tc_F2 + 64 + c->tc_F2 / 2) cols <<= 1;
   c->tc_tmem_cols = cols;
-  const int unit_tokens = c->tc ? 32 : DT;  // tokens per tile (64 for the warp-MMA kernel)
-  const int n_headsets = c->tc ? (sh.B * sh.Hq + 127) / 128
+  // The cluster tensor-core split kernel takes the plans with 256 <= k <= 1023 on
+  // per-KV-head E blocks when G is 2, 4 or 8 and its per-CTA buffers fit (it replaces the
+  // warp-MMA kernel there).
+  c->cl = 0;
+  if (!c->tc && M > 0 && (plan->G == 2 || plan->G == 4 || plan->G == 8)) {
+    const int slots = 2 * c->F_pad;
+    const int C = slots <= 256 ? 1 : (slots <= 512 ? 2 : (slots <= 1024 ? 4 : 0));
+    if (C >= 2 && de_ld_max <= 32 * C) cl_configure(plan, C, slots, c);
+    // a device on which no cluster of it can be resident keeps the warp-MMA kernel (with no
+    // device to ask, the plan's choice stands)
+    int nclu = 0;
+    if (c->cl && decode_cl_max_clusters(c->cl_C, c->cl_smem, &nclu) == cudaSuccess && nclu < 1)
+      c->cl = 0;
+  }
+  if (c->cl) c->hm = 0;
+  const int unit_tokens = (c->tc || c->cl) ? 32 : DT;  // tokens per tile (64: warp-MMA, CUDA cores)
+  const int n_headsets = (c->tc || c->cl) ? (sh.B * sh.Hq + 127) / 128
                                : (c->hm ? (sh.B * sh.Hq + 15) / 16 : (n_heads + c->NKV - 1) / c->NKV);
   const int ntiles = (M + unit_tokens - 1) / unit_tokens;
   if (M == 0) {
@@ -774,7 +840,14 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
       int sms = 148, occ = 1;
       cudaError_t e = device_sm_count(&sms);
       if (e != cudaSuccess) return e;
-      if (c->tc || c->hm) {
+      if (c->cl) {
+        // slots = resident clusters (each cluster serves one head set and split)
+        int nclu = 0;
+        e = decode_cl_max_clusters(c->cl_C, c->cl_smem, &nclu);
+        if (e != cudaSuccess) return e;
+        sms = nclu > 0 ? nclu : 1;
+        occ = 1;
+      } else if (c->tc || c->hm) {
         occ = 1;  // one CTA per SM (shared memory)
       } else {
         e = c->SPT == 1 ? occupancy<1>(&occ, c->smem_main)
@@ -869,6 +942,12 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   p.TG = c.TG;
   p.tc_F2 = c.tc_F2;
   p.tc_tmem_cols = c.tc_tmem_cols;
+  p.cl_C = c.cl_C;
+  p.cl_SL = c.cl_SL;
+  p.cl_TB = c.cl_TB;
+  p.cl_stages = c.cl_stages;
+  p.cl_slot_bytes = c.cl_slot_bytes;
+  p.cl_tmem_cols = c.cl_tmem_cols;
   p.DEC = c.DEC;
   p.TGE = c.TGE;
   p.qscale = (float)(1.4426950408889634 / sqrt((double)FA_HEAD_DIM));
@@ -903,7 +982,7 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
   cudaError_t e;
   // On the tensor-core and warp-MMA paths the sink / recent rows run as extra CTAs of the
   // prologue launch (small CTAs that need only q; the split kernels hold whole SMs).
-  const bool sr_with_prologue = p.M > 0 && (c.tc || c.hm);
+  const bool sr_with_prologue = p.M > 0 && (c.tc || c.hm || c.cl);
   if (p.M > 0) {
     p.n_pro = n_heads;
     const int pro_grid = n_heads + (sr_with_prologue ? n_heads * c.n_fsplits : 0);
@@ -917,6 +996,8 @@ cudaError_t launch_decode(const fa_plan* plan, const DecodeConfig& c, const void
     if ((e = launch_decode_tc(p, plan->de_ld[0], stream)) != cudaSuccess) return e;
   } else if (plan->e_token_major && plan->M > 0) {
     return cudaErrorInvalidValue;  // the CUDA-core kernel reads per-KV-head E blocks only
+  } else if (c.cl) {
+    if ((e = launch_decode_cl(p, stream)) != cudaSuccess) return e;
   } else if (c.hm) {
     if ((e = launch_decode_hmma(p, c.hm_F2, stream)) != cudaSuccess) return e;
   }

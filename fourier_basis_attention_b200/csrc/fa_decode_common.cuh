@@ -21,6 +21,7 @@ struct DecodeParams {
   int tc_F2, tc_tmem_cols;  // tensor-core split kernel: coefficient slots, TMEM columns
   int e_row;                // token-major E: elements per token row of a batch
   int n_pro;                // prologue CTAs (the sink / recent CTAs of a prologue launch follow)
+  int cl_C, cl_SL, cl_TB, cl_stages, cl_slot_bytes, cl_tmem_cols;  // cluster tensor-core kernel
   float qscale, norm_single, norm_pair, two_over_P;
   long long e_batch, c_batch;
   long long e_off[FA_MAX_KV_HEADS], c_off[FA_MAX_KV_HEADS];
@@ -197,6 +198,10 @@ __device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
 }
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream);
+
+// Cluster tensor-core split kernel (fa_decode_cl.cu): per-KV-head E blocks, coefficient
+// slots split over a cluster of C CTAs (C = 1, 2 or 4).
+cudaError_t launch_decode_cl(const DecodeParams& p, cudaStream_t stream);
 size_t decode_tc_smem_bytes(int F2, int de_slot, int G);
 
 }  // namespace fa

@@ -13,6 +13,9 @@ struct DecodeConfig {
   int n_splits, split_len, n_fsplits, n_rec, F, F_pad, SPT, NTU, TG, DEC, TGE, NKV;
   int tc, tc_F2, tc_tmem_cols, de_ld_max;  // tensor-core split kernel chosen, its slots / TMEM
   int hm, hm_F2;  // warp-MMA split kernel chosen (blocked E, large k), its slots
+  // cluster tensor-core split kernel chosen (blocked E), its cluster size, slots per CTA,
+  // ring token block, ring stages and slot bytes, TMEM columns, shared-memory bytes
+  int cl, cl_C, cl_SL, cl_TB, cl_stages, cl_slot_bytes, cl_tmem_cols, cl_smem;
   int cb_gt;      // query heads per combine CTA (a divisor of G)
   size_t qw_bytes, rec_bytes, smem_main, smem_combine;
   int rec_stride, qw_stride;
@@ -47,6 +50,12 @@ cudaError_t device_sm_count(int* sms);
 cudaError_t raise_smem_limit(const void* func, int bytes);
 // Resident blocks per SM of `func` at `threads` threads and `smem` dynamic shared bytes.
 cudaError_t cached_occupancy(const void* func, int threads, size_t smem, int* blocks);
+// Clusters of `cluster` CTAs of `func` that can be resident at once on the current device.
+cudaError_t cached_max_clusters(const void* func, int threads, size_t smem, int cluster, int* n);
+// Cluster tensor-core decode kernel (fa_decode_cl.cu): shared-memory bytes of a layout,
+// and resident clusters of it.
+size_t decode_cl_smem_bytes(int C, int SL, int slot_bytes, int stages);
+cudaError_t decode_cl_max_clusters(int C, int smem, int* n);
 
 // Records `msg` as the calling thread's fa_last_error() text and returns `code`.
 int set_last_error(int code, const char* msg);

@@ -101,4 +101,42 @@ cudaError_t cached_occupancy(const void* func, int threads, size_t smem, int* bl
   return cudaSuccess;
 }
 
+cudaError_t cached_max_clusters(const void* func, int threads, size_t smem, int cluster, int* n) {
+  int dev = 0;
+  cudaError_t e = device_index(&dev);
+  if (e != cudaSuccess) return e;
+  // keyed like the occupancy table, with the cluster size in the thread count's high bits
+  const int key_threads = threads | (cluster << 16);
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < g_n_occ; ++i) {
+      const OccEntry& o = g_occ[i];
+      if (o.func == func && o.dev == dev && o.threads == key_threads && o.smem == smem) {
+        *n = o.blocks;
+        return cudaSuccess;
+      }
+    }
+  }
+  if ((e = raise_smem_limit(func, (int)smem)) != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)cluster, 1, 1);
+  cfg.blockDim = dim3((unsigned)threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int c = 0;
+  e = cudaOccupancyMaxActiveClusters(&c, func, &cfg);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const int slot = g_n_occ < kMaxEntries ? g_n_occ++ : (g_occ_next++ % kMaxEntries);
+  g_occ[slot] = OccEntry{func, dev, key_threads, smem, c};
+  *n = c;
+  return cudaSuccess;
+}
+
 }  // namespace fa

@@ -208,6 +208,28 @@ int fa_compress(const fa_plan* plan, const void* K, const void* V, const void* p
 size_t fa_decode_workspace_size(const fa_plan* plan, int32_t num_splits);
 
 /*
+ * fa_decode_describe -- how fa_decode would run a plan (no counterpart in the paper; a
+ * host-side query for callers that size launches, graphs or profiles).
+ *   info->split_kernel  which kernel runs the middle span (enum fa_split_kernel);
+ *   info->num_splits    split-L partitions (num_splits <= 0: the automatic choice for the
+ *                       current device, as fa_decode makes it);
+ *   info->cluster       CTAs per thread-block cluster of the split kernel (1 = no cluster);
+ *   info->launches      kernels one fa_decode call launches.
+ * Returns the status fa_decode_workspace_size would imply (message in fa_last_error()).
+ */
+enum fa_split_kernel {
+  FA_SPLIT_NONE = 0,        /* no middle span: only the sink / recent rows */
+  FA_SPLIT_CUDA_CORES = 1,  /* fp32 CUDA-core split kernel */
+  FA_SPLIT_TC_TOKEN_MAJOR = 2, /* tcgen05 split kernel over token-major E (k <= 255) */
+  FA_SPLIT_WARP_MMA = 3,    /* warp-level MMA split kernel (256 <= k <= 1023) */
+  FA_SPLIT_TC_CLUSTER = 4   /* tcgen05 split kernel, coefficient slots split over a cluster */
+};
+typedef struct fa_decode_info {
+  int32_t split_kernel, num_splits, cluster, launches;
+} fa_decode_info;
+int fa_decode_describe(const fa_plan* plan, int32_t num_splits, fa_decode_info* info);
+
+/*
  * fa_decode -- one decode step: every query attends to all L tokens of the hybrid cache.
  * ([skill] Step 4, restore during decoding; [abstract].)
  *   q     device bf16 [B][Hq][128], one query per sequence and head.

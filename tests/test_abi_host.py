@@ -39,7 +39,8 @@ def test_library_exports_every_declared_function():
 def test_plan_struct_matches_header_layout(tmp_path):
     """The ctypes mirrors have the C layout of the header: gcc compiles the header and
     prints sizeof and every field's offsetof, which must equal the ctypes ones."""
-    structs = {"fa_shape": fa.fa_shape, "fa_plan": fa.fa_plan, "fa_cache": fa.fa_cache}
+    structs = {"fa_shape": fa.fa_shape, "fa_plan": fa.fa_plan, "fa_cache": fa.fa_cache,
+               "fa_decode_info": fa.fa_decode_info}
     lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "fourier_attention.h"',
              "int main(void) {"]
     for name, cls in structs.items():

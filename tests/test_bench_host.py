@@ -58,14 +58,26 @@ def test_config_dict_is_shared_by_both_arms():
 
 
 def test_launches_per_step_each_path():
-    """6 launches on the tensor-core and warp-MMA paths (sink / recent rows ride in the
-    prologue launch) and on the CUDA-core path (they ride in the split kernel)."""
+    """6 launches on every path with a middle span and sink / recent rows: basis table,
+    sink / recent copy, projection; then prologue (carrying the sink / recent rows on the
+    tensor-core and warp-MMA paths), split kernel (carrying them on the CUDA-core path) and
+    combine. The split kernel each workload takes is the library's documented choice."""
     tc = wl.LLAMA2_7B_MHA_32K
-    hm = wl.LLAMA3_8B_GQA_128K
+    cl = wl.LLAMA3_8B_GQA_128K
     cc = wl.llama3_8b_layer(1, 8192, 0)
-    assert _plan(tc).e_token_major == 1 and bench.launches_per_step(tc, _plan(tc)) == 6
-    assert _plan(hm).e_token_major == 0 and bench.launches_per_step(hm, _plan(hm)) == 6
-    assert _plan(cc).e_token_major == 0 and bench.launches_per_step(cc, _plan(cc)) == 6
+    hm = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=3, Hq=4, Hkv=4, L=2000, k=511)   # G = 1, k = 511
+    kinds = {w.name + str(w.B): fa.fa_decode_describe(_plan(w), 1) for w in (tc, cl, cc, hm)}
+    assert kinds[tc.name + "8"].split_kernel == 2 and _plan(tc).e_token_major == 1
+    assert kinds[cl.name + "4"].split_kernel == 4 and kinds[cl.name + "4"].cluster == 4
+    assert kinds[cc.name + "1"].split_kernel == 1
+    assert kinds[hm.name + "3"].split_kernel == 3
+    for w in (tc, cl, cc, hm):
+        assert bench.launches_per_step(w, _plan(w)) == 6
+    # no middle span: basis table, sink / recent copy, the split kernel with the sink /
+    # recent rows, combine
+    w0 = wl.shrink(tc, B=1, Hq=2, Hkv=2, L=90)
+    assert fa.fa_decode_describe(_plan(w0), 1).split_kernel == 0
+    assert bench.launches_per_step(w0, _plan(w0)) == 4
 
 
 def test_append_bytes_by_hand():

@@ -276,6 +276,25 @@ def _ragged_hkv(dcs, Hkv):
     return mask
 
 
+# Plans with 256 <= k <= 1023, G in {2, 4, 8} and per-KV-head E blocks run the middle span
+# on the cluster tensor-core kernel: the coefficient slots are split over 2 (k <= 511) or 4
+# CTAs of a thread-block cluster, partial scores summed by each quadrant's owner CTA.
+@pytest.mark.parametrize("G,Hkv,k,B,dcs,cluster", [
+    (4, 2, 511, 3, [96, 64], 2),             # ragged exact dims (32 / 64 per KV head)
+    (2, 4, 511, 5, [96, 64, 90, 120], 2),    # G = 2: 32 exact KV heads per CTA
+    (8, 2, 1023, 2, [96, 100], 4),           # G = 8
+    (4, 8, 1023, 5, None, 4),                # 160 query heads: a second, partial head set
+    (4, 2, 257, 2, [96, 96], 2),             # 2 F_pad = 264 slots: 192 per CTA
+], ids=["C2_G4_ragged", "C2_G2", "C4_G8", "C4_two_head_sets", "C2_192_slots"])
+def test_cluster_decode(G, Hkv, k, B, dcs, cluster):
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=B, Hq=Hkv * G, Hkv=Hkv, L=k + 96 + 333, k=k)
+    mask = wl.dim_mask(w) if dcs is None else _ragged_hkv(dcs, Hkv)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    info = fa.fa_decode_describe(p, 1)
+    assert info.split_kernel == fa.FA_SPLIT_TC_CLUSTER and info.cluster == cluster
+    run_small(w, mask=mask)
+
+
 @pytest.mark.parametrize("ns", [1, 5, 1000])
 def test_split_counts_warp_mma(ns):
     run_small(wl.shrink(wl.LLAMA3_8B_GQA_128K, B=1, Hq=32, Hkv=8, L=3300), num_splits=ns,
