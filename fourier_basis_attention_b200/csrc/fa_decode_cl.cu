@@ -181,10 +181,10 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
     tmem_alloc(tmem_slot, p.cl_tmem_cols);
     tmem_relinquish();
   }
-  // ring zeroed (rows past a split's end are read by the score MMAs but never copied);
-  // exact-dim query rows (bf16, unscaled, zero past de) of the owned quadrants
-  for (int o = threadIdx.x * 16; o < stages * slot_bytes; o += CL_THREADS * 16)
-    *reinterpret_cast<uint4*>(ring + o) = make_uint4(0, 0, 0, 0);
+  // exact-dim query rows (bf16, unscaled, zero past de) of the owned quadrants. (The ring
+  // is not cleared: rows past a split's end are never copied, but the score MMA gives each
+  // token its own output column and those tokens' scores are replaced by -inf before use,
+  // and the value loops stop at the last token.)
   for (int idx = threadIdx.x; idx < NOWN * 32 * FA_HEAD_DIM; idx += CL_THREADS) {
     const int li = idx / (32 * FA_HEAD_DIM), rem = idx - li * 32 * FA_HEAD_DIM;
     const int row = rem >> 7, d = rem & 127;
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
           const uint8_t* slotp = ring + s * slot_bytes;
           for (int e = wq; e < n_exact; e += 4) {
             const ClExact& me = meta[e];
-            if (!me.valid || me.de_ld == 0) continue;
+            if (!me.valid) continue;  // a KV head without exact dims gets zero scores (nk = 0)
             const uint8_t* blk = slotp + me.off;
             const __nv_bfloat16* qrow = qes + (me.li * 32 + me.row0 + ar) * CL_QE_LD;
             const int nk = (me.de_ld + 15) >> 4;
