@@ -383,11 +383,21 @@ cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream) 
   return cudaGetLastError();
 }
 
+FA_WATCHDOG_READER(read_watchdog_compress)
+
+// The first nonzero word of the units whose kernels wait on mbarriers (compress, the
+// tensor-core decode, the cluster decode); every word is cleared.
 cudaError_t read_and_clear_watchdog(unsigned int* word) {
-  cudaError_t e = cudaMemcpyFromSymbol(word, g_watchdog, sizeof(unsigned int));
-  if (e != cudaSuccess) return e;
-  const unsigned int zero = 0;
-  return cudaMemcpyToSymbol(g_watchdog, &zero, sizeof(unsigned int));
+  cudaError_t (*readers[])(unsigned int*) = {read_watchdog_compress, read_watchdog_decode_tc,
+                                             read_watchdog_decode_cl};
+  *word = 0;
+  for (auto rd : readers) {
+    unsigned int w = 0;
+    cudaError_t e = rd(&w);
+    if (e != cudaSuccess) return e;
+    if (*word == 0) *word = w;
+  }
+  return cudaSuccess;
 }
 
 typedef CUresult (*PFN_encodeTiled)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

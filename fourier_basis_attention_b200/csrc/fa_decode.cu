@@ -817,7 +817,7 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   if (!c->tc && M > 0 && (plan->G == 2 || plan->G == 4 || plan->G == 8)) {
     const int slots = 2 * c->F_pad;
     const int C = slots <= 256 ? 1 : (slots <= 512 ? 2 : (slots <= 1024 ? 4 : 0));
-    if (C >= 2 && de_ld_max <= 32 * C) cl_configure(plan, C, slots, c);
+    if (C >= 2 && de_ld_max <= 64) cl_configure(plan, C, slots, c);
     // a device on which no cluster of it can be resident keeps the warp-MMA kernel (with no
     // device to ask, the plan's choice stands)
     int nclu = 0;

@@ -43,9 +43,8 @@ constexpr float CL_LAZY = 8.0f;
 constexpr float CL_P_SCALE = 128.0f;
 constexpr float CL_P_UNSCALE = 1.0f / 128.0f;
 constexpr int CL_XS_LD = 33;     // fp32 row pitch of the [head][token] score / p buffers
-constexpr int CL_XR_LD = 36;     // fp32 row pitch of a received partial-score block
-constexpr int CL_PR_LD = 20;     // words per head of a received P row (16 P words + alpha)
-constexpr int CL_QE_LD = 136;    // bf16 row pitch of the exact-dim query rows
+constexpr int CL_XB = 32 * CL_T * 4;  // bytes of one quadrant's partial-score block (4 KB):
+                                 // row = head, 16-byte chunk j of row h at (j ^ (h & 7))
 constexpr int CL_MAX_EXACT = 32; // exact KV heads per CTA (owned query heads / G)
 constexpr int CL_MAX_STAGES = 8;
 constexpr int CL_EPAD = 64;      // bytes between two KV heads' blocks in a ring slot
@@ -61,7 +60,7 @@ struct ClExact {   // one exact KV head of the CTA (32 bytes)
 };
 
 struct ClLayout {
-  int w, phi, ps, ring, xr, pr, xs, qe, al, meta, bars, total;  // byte offsets
+  int w, phi, ps, ring, xr, xsend, xs, al, meta, bars, total;  // byte offsets
 };
 
 __host__ __device__ inline ClLayout cl_layout(int C, int SL, int slot_bytes, int stages) {
@@ -71,11 +70,10 @@ __host__ __device__ inline ClLayout cl_layout(int C, int SL, int slot_bytes, int
   L.phi = L.w + CL_NH * SL * 2;                     // 2 x [SL/64][32 tokens][64 fp16] SW128
   L.ps = L.phi + 2 * CL_T * SL * 2;                 // 2 x [128 heads][32 fp16] SW64
   L.ring = L.ps + 2 * CL_NH * CL_T * 2;             // stages x slot_bytes
-  L.xr = L.ring + stages * slot_bytes;              // [2][nown][C-1][32][CL_XR_LD] fp32
-  L.pr = L.xr + 2 * nown * (C - 1) * 32 * CL_XR_LD * 4;  // [2][4-nown][32][CL_PR_LD] words
-  L.xs = L.pr + 2 * (4 - nown) * 32 * CL_PR_LD * 4;       // [2][nown][32][CL_XS_LD] fp32
-  L.qe = L.xs + 2 * nown * 32 * CL_XS_LD * 4;             // [nown][32][CL_QE_LD] bf16
-  L.al = L.qe + nown * 32 * CL_QE_LD * 2;                 // [2][128] fp32 rescale factors
+  L.xr = L.ring + stages * slot_bytes;              // [2][nown][C-1] partial-score blocks
+  L.xsend = L.xr + 2 * nown * (C - 1) * CL_XB;      // [4 - nown] outgoing blocks
+  L.xs = L.xsend + (4 - nown) * CL_XB;              // [2][nown][32][CL_XS_LD] fp32
+  L.al = L.xs + 2 * nown * 32 * CL_XS_LD * 4;             // [2][128] fp32 rescale factors
   L.meta = L.al + 2 * CL_NH * 4;                          // [CL_MAX_EXACT] ClExact
   L.bars = L.meta + CL_MAX_EXACT * (int)sizeof(ClExact);  // mbarriers, TMEM slot, flags
   L.total = L.bars + 64 * 8 + 64 + 1024;                  // + alignment slack
@@ -92,8 +90,9 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
     decode_cl_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int NOWN = 4 / C;  // quadrants owned by each CTA
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, formed by pointer arithmetic on smem_raw so that the compiler
+  // keeps it (and everything derived from it) in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int SL = p.cl_SL;
   const int stages = p.cl_stages, slot_bytes = p.cl_slot_bytes, TB = p.cl_TB;
   const ClLayout Ly = cl_layout(C, SL, slot_bytes, stages);
@@ -101,10 +100,9 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
   uint8_t* PHI = smem + Ly.phi;
   uint8_t* PS = smem + Ly.ps;
   uint8_t* ring = smem + Ly.ring;
-  float* xr = reinterpret_cast<float*>(smem + Ly.xr);
-  uint32_t* pr = reinterpret_cast<uint32_t*>(smem + Ly.pr);
+  uint8_t* xr = smem + Ly.xr;
+  uint8_t* xsend = smem + Ly.xsend;
   float* xs = reinterpret_cast<float*>(smem + Ly.xs);
-  __nv_bfloat16* qes = reinterpret_cast<__nv_bfloat16*>(smem + Ly.qe);
   float* al = reinterpret_cast<float*>(smem + Ly.al);
   ClExact* meta = reinterpret_cast<ClExact*>(smem + Ly.meta);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bars);
@@ -116,7 +114,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
   uint64_t* r_full = bars + 9;      // [stages] producer -> head warps (expect_tx)
   uint64_t* r_empty = r_full + CL_MAX_STAGES;  // [stages] head warps -> producer (count 4)
   uint64_t* xr_full = r_empty + CL_MAX_STAGES; // [2][NOWN] partial scores received
-  uint64_t* pr_full = xr_full + 2 * 4;         // [2][4 - NOWN] P rows received
+  uint64_t* pr_full = xr_full + 2 * 4;         // [2][4 - NOWN] P rows + factors received
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pr_full + 2 * 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* n_exact_s = const_cast<int*>(abort_flag) + 1;
@@ -181,21 +179,9 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
     tmem_alloc(tmem_slot, p.cl_tmem_cols);
     tmem_relinquish();
   }
-  // exact-dim query rows (bf16, unscaled, zero past de) of the owned quadrants. (The ring
-  // is not cleared: rows past a split's end are never copied, but the score MMA gives each
-  // token its own output column and those tokens' scores are replaced by -inf before use,
-  // and the value loops stop at the last token.)
-  for (int idx = threadIdx.x; idx < NOWN * 32 * FA_HEAD_DIM; idx += CL_THREADS) {
-    const int li = idx / (32 * FA_HEAD_DIM), rem = idx - li * 32 * FA_HEAD_DIM;
-    const int row = rem >> 7, d = rem & 127;
-    const long long gh = (long long)hs * CL_NH + 32 * (q_first + li) + row;
-    __nv_bfloat16 v = __float2bfloat16_rn(0.0f);
-    if (gh < bhq) {
-      const int bb = (int)(gh / p.Hq), gg = (int)(gh - (long long)bb * p.Hq) / G;
-      if (d < p.de[gg]) v = p.q[gh * FA_HEAD_DIM + p.perm[gg][p.dc[gg] + d]];
-    }
-    qes[(li * 32 + row) * CL_QE_LD + d] = v;
-  }
+  // (The exact-dim ring is not cleared: rows past a split's end are never copied, but their
+  // tokens' scores are replaced by -inf before use and the value loops stop at the last
+  // token.)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -309,40 +295,51 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
       const unsigned long long w0 = globaltimer_ns();
       while (!mbar_try_wait(u_done, 0) && globaltimer_ns() - w0 < kWaitLimitNs) {
       }
+      if constexpr (C > 1) {
+        // MMA 2's commits arrive on phi_free in every CTA of the cluster. Nothing else waits
+        // for the last two tiles' phases, so this CTA waits for them here: once they complete,
+        // no peer's arrive is still on its way to this CTA's shared memory when it leaves.
+        for (int i = ntiles >= 2 ? ntiles - 2 : 0; i < ntiles; ++i)
+          mbar_wait(&phi_free[i & 1], (uint32_t)(i >> 1) & 1u, abort_flag, WD_DECODE | 43u);
+      }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------------- exact-dim producer
     if (lane == 0 && has_exact) {
+      // chunks in the head warps' order: K(0); then per tile i: V(i - 1), K(i + 1); V(last)
       int cc = 0;
       bool ok = true;
-      for (int i = 0; i < ntiles && ok; ++i) {
-        const int t0 = lo + i * CL_T;
-        for (int ph = 0; ph < 2 && ok; ++ph) {
-          const __nv_bfloat16* E = ph ? p.EV : p.EK;
-          for (int sb = 0; sb < nsb; ++sb, ++cc) {
-            const int s = cc % stages;
-            if (cc >= stages &&
-                !mbar_wait(&r_empty[s], (uint32_t)((cc / stages) - 1) & 1u, abort_flag,
-                           WD_DECODE | 34u)) {
-              ok = false;
-              break;
-            }
-            const int tok0 = t0 + sb * TB;
-            const int rows = max(0, min(TB, hi - tok0));
-            uint32_t bytes = 0;
-            for (int e = 0; e < n_exact; ++e)
-              if (meta[e].valid) bytes += (uint32_t)(rows * meta[e].de_ld * 2);
-            mbar_arrive_expect_tx(&r_full[s], bytes);
-            for (int e = 0; e < n_exact; ++e) {
-              const ClExact& m = meta[e];
-              if (m.valid && m.de_ld > 0 && rows > 0)
-                bulk_load_cta(ring + s * slot_bytes + m.off,
-                              E + m.gbase + (long long)tok0 * m.de_ld,
-                              (uint32_t)(rows * m.de_ld * 2), &r_full[s]);
-            }
+      auto issue = [&](int ti, int ph) {
+        const int t0 = lo + ti * CL_T;
+        const __nv_bfloat16* E = ph ? p.EV : p.EK;
+        for (int sb = 0; sb < nsb && ok; ++sb, ++cc) {
+          const int s = cc % stages;
+          if (cc >= stages &&
+              !mbar_wait(&r_empty[s], (uint32_t)((cc / stages) - 1) & 1u, abort_flag,
+                         WD_DECODE | 34u)) {
+            ok = false;
+            break;
+          }
+          const int tok0 = t0 + sb * TB;
+          const int rows = max(0, min(TB, hi - tok0));
+          uint32_t bytes = 0;
+          for (int e = 0; e < n_exact; ++e)
+            if (meta[e].valid) bytes += (uint32_t)(rows * meta[e].de_ld * 2);
+          mbar_arrive_expect_tx(&r_full[s], bytes);
+          for (int e = 0; e < n_exact; ++e) {
+            const ClExact& m = meta[e];
+            if (m.valid && m.de_ld > 0 && rows > 0)
+              bulk_load_cta(ring + s * slot_bytes + m.off, E + m.gbase + (long long)tok0 * m.de_ld,
+                            (uint32_t)(rows * m.de_ld * 2), &r_full[s]);
           }
         }
+      };
+      if (ntiles > 0) issue(0, 0);
+      for (int i = 0; i < ntiles && ok; ++i) {
+        if (i >= 1) issue(i - 1, 1);
+        if (i + 1 < ntiles) issue(i + 1, 0);
       }
+      if (ntiles > 0 && ok) issue(ntiles - 1, 1);
     }
   } else if (warp < 4) {
     // -------------------------------------------------------------------- basis generators
@@ -361,7 +358,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
     }
     for (int i = 0; i < ntiles; ++i) {
       const int b = i & 1;
-      if (i >= 2 && !mbar_wait_cluster(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag,
+      if (i >= 2 && !mbar_wait(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag,
                                        WD_DECODE | 35u))
         break;
       const long long tm0 = (long long)lo + i * CL_T;
@@ -422,6 +419,44 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
       }
       n_items += it_e[u] >= 0 ? 1 : 0;
     }
+    // exact-dim scores: lane = (query head sh of the warp's KV heads, token group sg); the
+    // warp's 32 / C query heads (its KV heads e = wq, wq + 4, ... times G) take SGN = C
+    // token groups. q_e of the lane's head in registers (unscaled, 8-dim chunks as pairs).
+    const int SGN = C;
+    const int HW = 32 / SGN;
+    const int shi = lane % HW, sg = lane / HW;
+    int sh_off = 0, sh_pitch = 0, sh_c8 = 0, sh_row = 0;
+    bool sh_ok = false;  // the lane has a valid query head (its KV head may have no exact dims)
+    float2 qv[8][4];
+    {
+      const int el = shi / G, jq = shi % G;
+      const int e = wq + 4 * el;
+      if (e < n_exact && meta[e].valid) {
+        const ClExact& me = meta[e];
+        sh_ok = true;
+        sh_off = me.off;
+        sh_pitch = me.de_ld * 2;
+        sh_c8 = me.de_ld / 8;
+        sh_row = me.li * 32 + me.row0 + jq;
+        const long long ghs = (long long)hs * CL_NH + 32 * (q_first + me.li) + me.row0 + jq;
+        const int bb = (int)(ghs / p.Hq), gg = (int)(ghs - (long long)bb * p.Hq) / G;
+#pragma unroll
+        for (int d8 = 0; d8 < 8; ++d8)
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            float2 v = make_float2(0.0f, 0.0f);
+            const int d = 8 * d8 + 2 * e2;
+            if (d < me.de) v.x = __bfloat162float(p.q[ghs * FA_HEAD_DIM + p.perm[gg][p.dc[gg] + d]]);
+            if (d + 1 < me.de) v.y = __bfloat162float(p.q[ghs * FA_HEAD_DIM + p.perm[gg][p.dc[gg] + d + 1]]);
+            qv[d8][e2] = v;
+          }
+      } else {
+#pragma unroll
+        for (int d8 = 0; d8 < 8; ++d8)
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) qv[d8][e2] = make_float2(0.0f, 0.0f);
+      }
+    }
     float acc[CL_MAX_IPL][8];
 #pragma unroll
     for (int u = 0; u < CL_MAX_IPL; ++u)
@@ -430,7 +465,6 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
     float m = -INFINITY, l = 0.0f;  // softmax state of head h (owned quadrant)
     bool ok = true;
     int cc = 0;  // ring slot counter (same sequence as the producer's)
-    const int ar = lane >> 2, ac = (lane & 3) * 2;  // MMA fragment row / column pair
 
     auto ring_wait = [&](int s) -> bool {
       return mbar_wait(&r_full[s], (uint32_t)(cc / stages) & 1u, abort_flag, WD_DECODE | 36u);
@@ -440,50 +474,120 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
       if (lane == 0) mbar_arrive(&r_empty[s]);
     };
 
-    for (int i = 0; i < ntiles; ++i) {
-      const int b = i & 1;
-      const int t0 = lo + i * CL_T;
-      const int nt = min(CL_T, hi - t0);
-      float* xsb = xs + b * NOWN * 32 * CL_XS_LD;
-      // ---- exact-dim scores of this warp's KV heads into xs[b] (scaled by sigma log2 e)
-      if (has_exact) {
+    // A(i): exact-dim scores of tile i into xs[i & 1] (scaled by sigma log2 e); lane (query
+    // head sh, token group sg) takes tokens sg, sg + SGN, ... of each ring slot
+    auto scores = [&](int i) {
+      float* xsb = xs + (i & 1) * NOWN * 32 * CL_XS_LD;
+      {
         for (int sb = 0; sb < nsb; ++sb, ++cc) {
           const int s = cc % stages;
           ok = ring_wait(s) && ok;
-          const uint8_t* slotp = ring + s * slot_bytes;
-          for (int e = wq; e < n_exact; e += 4) {
-            const ClExact& me = meta[e];
-            if (!me.valid) continue;  // a KV head without exact dims gets zero scores (nk = 0)
-            const uint8_t* blk = slotp + me.off;
-            const __nv_bfloat16* qrow = qes + (me.li * 32 + me.row0 + ar) * CL_QE_LD;
-            const int nk = (me.de_ld + 15) >> 4;
-            for (int tg = 0; tg < TB / 8; ++tg) {
-              float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-              const uint8_t* rowp = blk + (tg * 8 + (lane & 7)) * me.de_ld * 2;
-              for (int ks = 0; ks < nk; ++ks) {
-                uint32_t bq[4];
-                const int grp = 2 * ks + ((lane >> 3) & 1);
-                if (2 * ks + 1 < me.de_ld / 8)
-                  ldmatrix_x2(bq, rowp + grp * 16);
-                else
-                  ldmatrix_x1(bq, rowp + 2 * ks * 16);
-                uint32_t a0 = 0, a2 = 0;
-                if (ar < G) {
-                  a0 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + ac);
-                  a2 = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 8 + ac);
+          if (sh_ok) {
+            const uint8_t* blk = ring + s * slot_bytes + sh_off;
+            float* xrw = xsb + sh_row * CL_XS_LD + sb * TB;
+            const int ntb = TB;  // tokens past the split's end are masked by the owner
+            for (int t0 = sg; t0 < ntb; t0 += 4 * SGN) {
+              float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+              for (int d8 = 0; d8 < 8; ++d8) {
+                if (d8 < sh_c8) {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u) {
+                    const int t = t0 + u * SGN;
+                    if (t < ntb) {
+                      float2 x2[4];
+                      bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(blk + t * sh_pitch + d8 * 16), x2);
+                      float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+                      for (int e = 0; e < 4; ++e) a = __ffma2_rn(qv[d8][e], x2[e], a);
+                      acc4[u] += a.x + a.y;
+                    }
+                  }
                 }
-                mma_bf16_16816_rows8(d, a0, a2, bq[0], bq[1]);
               }
-              if (ar < G) {
-                float* xrw = xsb + (me.li * 32 + me.row0 + ar) * CL_XS_LD + sb * TB + tg * 8 + ac;
-                xrw[0] = d[0] * p.qscale;
-                xrw[1] = d[1] * p.qscale;
-              }
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                if (t0 + u * SGN < ntb) xrw[t0 + u * SGN] = acc4[u] * p.qscale;
             }
           }
           ring_release(s);
         }
       }
+    };
+    // G(i): exact-dim values of tile i, acc = alpha acc + p E_V over this warp's items (p in
+    // xs[i & 1], rescale factors in al[i & 1])
+    auto values = [&](int i) {
+      const int b = i & 1;
+      const int nt = min(CL_T, hi - (lo + i * CL_T));
+      const float* xsb = xs + b * NOWN * 32 * CL_XS_LD;
+#pragma unroll
+      for (int u = 0; u < CL_MAX_IPL; ++u) {
+        if (u < n_items) {
+          const ClExact& me = meta[it_e[u]];
+          const float a = al[b * CL_NH + 32 * (q_first + me.li) + me.row0 + it_jq[u]];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[u][e] *= a;
+        }
+      }
+      for (int sb = 0; sb < nsb; ++sb, ++cc) {
+        const int s = cc % stages;
+        ok = ring_wait(s) && ok;
+        const uint8_t* slotp = ring + s * slot_bytes;
+        const int ntb = min(TB, nt - sb * TB);
+#pragma unroll
+        for (int u = 0; u < CL_MAX_IPL; ++u) {
+          if (u < n_items) {
+            const ClExact& me = meta[it_e[u]];
+            const float* prw = xsb + (me.li * 32 + me.row0 + it_jq[u]) * CL_XS_LD + sb * TB;
+            const uint8_t* col = slotp + me.off + it_c[u] * 16;
+            const int pitch = me.de_ld * 2;
+            float2 a2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a2[e] = make_float2(acc[u][2 * e], acc[u][2 * e + 1]);
+            int t = 0;
+            for (; t + 4 <= ntb; t += 4) {  // four tokens' loads issued together
+              uint4 xv[4];
+              float pt[4];
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                xv[v] = *reinterpret_cast<const uint4*>(col + (t + v) * pitch);
+                pt[v] = prw[t + v];
+              }
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                float2 x2[4];
+                bf16x8_to_f32x2(xv[v], x2);
+                const float2 pp = make_float2(pt[v], pt[v]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) a2[e] = __ffma2_rn(pp, x2[e], a2[e]);
+              }
+            }
+            for (; t < ntb; ++t) {
+              float2 x2[4];
+              bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(col + t * pitch), x2);
+              const float2 pp = make_float2(prw[t], prw[t]);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) a2[e] = __ffma2_rn(pp, x2[e], a2[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              acc[u][2 * e] = a2[e].x;
+              acc[u][2 * e + 1] = a2[e].y;
+            }
+          }
+        }
+        ring_release(s);
+      }
+    };
+    // Software-pipelined tile loop: the partial scores of tile i travel to their owners
+    // while the values of tile i - 1 are accumulated, and the P rows of tile i travel back
+    // while the exact-dim scores of tile i + 1 are computed.
+    float sc[CL_T];
+    if (ntiles > 0 && has_exact) scores(0);
+    for (int i = 0; i < ntiles; ++i) {
+      const int b = i & 1;
+      const int nt = min(CL_T, hi - (lo + i * CL_T));
+      float* xsb = xs + b * NOWN * 32 * CL_XS_LD;
       // ---- partial S of quadrant `quad` over this CTA's slots
       ok = mbar_wait(&s_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, WD_DECODE | 37u) && ok;
       __syncwarp();
@@ -491,42 +595,49 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
       uint32_t sr[32];
       tmem_ld_32x32b_x32(tmem_s + lanebase + 32 * b, sr);
       tmem_ld_wait();
-      float sc[CL_T];
 #pragma unroll
       for (int t = 0; t < CL_T; ++t) sc[t] = hvalid ? __uint_as_float(sr[t]) * w_unscale : 0.0f;
       if constexpr (C > 1) {
         if (!own_q) {
-          // to the owner: row lane of block [b][its quadrant index][this CTA's sender slot]
-          const int oli = quad - owner * NOWN;
-          const int sslot = (int)rank < owner ? (int)rank : (int)rank - 1;
-          const uint32_t dst = mapa_shared(
-              smem_u32(xr + (((b * NOWN + oli) * (C - 1) + sslot) * 32 + lane) * CL_XR_LD),
-              (uint32_t)owner);
-          const uint32_t rb = mapa_shared(smem_u32(&xr_full[b * 4 + oli]), (uint32_t)owner);
+          // to the owner, as one bulk copy of the quadrant's block into slot [b][its quadrant
+          // index][this CTA's sender slot]. The staging block is free again: its previous copy
+          // landed before the owner answered the previous tile.
+          uint8_t* stg = xsend + npi * CL_XB;
 #pragma unroll
-          for (int t = 0; t < CL_T; t += 4)
-            st_async_v4(dst + 4 * t, __float_as_uint(sc[t]), __float_as_uint(sc[t + 1]),
-                        __float_as_uint(sc[t + 2]), __float_as_uint(sc[t + 3]), rb);
+          for (int j = 0; j < CL_T / 4; ++j)
+            *reinterpret_cast<float4*>(stg + lane * 128 + ((j ^ (lane & 7)) << 4)) =
+                make_float4(sc[4 * j], sc[4 * j + 1], sc[4 * j + 2], sc[4 * j + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int oli = quad - owner * NOWN;
+            const int sslot = (int)rank < owner ? (int)rank : (int)rank - 1;
+            const uint32_t dst = mapa_shared(
+                smem_u32(xr + ((b * NOWN + oli) * (C - 1) + sslot) * CL_XB), (uint32_t)owner);
+            const uint32_t rb = mapa_shared(smem_u32(&xr_full[b * 4 + oli]), (uint32_t)owner);
+            bulk_copy_s2s(dst, stg, CL_XB, rb);
+          }
         }
       }
-      asm volatile("bar.sync 2, 128;" ::: "memory");  // exact-dim scores of xs[b] complete
+      if (i > 0 && has_exact) values(i - 1);
+      asm volatile("bar.sync 2, 128;" ::: "memory");  // scores of tile i in xs[b]; xs[b ^ 1] free
       float alpha = 1.0f;
       if (own_q) {
         // ---- owner: full scores, online softmax, P rows to every CTA
         if constexpr (C > 1) {
           if (lane == 0)
-            mbar_arrive_expect_tx(&xr_full[b * 4 + li_q], (uint32_t)((C - 1) * 32 * CL_T * 4));
-          ok = mbar_wait_cluster(&xr_full[b * 4 + li_q], (uint32_t)(i >> 1) & 1u, abort_flag,
+            mbar_arrive_expect_tx(&xr_full[b * 4 + li_q], (uint32_t)((C - 1) * CL_XB));
+          ok = mbar_wait(&xr_full[b * 4 + li_q], (uint32_t)(i >> 1) & 1u, abort_flag,
                                  WD_DECODE | 38u) && ok;
           for (int s2 = 0; s2 < C - 1; ++s2) {
-            const float* src = xr + (((b * NOWN + li_q) * (C - 1) + s2) * 32 + lane) * CL_XR_LD;
+            const uint8_t* src = xr + ((b * NOWN + li_q) * (C - 1) + s2) * CL_XB + lane * 128;
 #pragma unroll
-            for (int t = 0; t < CL_T; t += 4) {
-              const float4 v = *reinterpret_cast<const float4*>(src + t);
-              sc[t] += hvalid ? v.x : 0.0f;
-              sc[t + 1] += hvalid ? v.y : 0.0f;
-              sc[t + 2] += hvalid ? v.z : 0.0f;
-              sc[t + 3] += hvalid ? v.w : 0.0f;
+            for (int j = 0; j < CL_T / 4; ++j) {
+              const float4 v = *reinterpret_cast<const float4*>(src + ((j ^ (lane & 7)) << 4));
+              sc[4 * j] += hvalid ? v.x : 0.0f;
+              sc[4 * j + 1] += hvalid ? v.y : 0.0f;
+              sc[4 * j + 2] += hvalid ? v.z : 0.0f;
+              sc[4 * j + 3] += hvalid ? v.w : 0.0f;
             }
           }
         }
@@ -553,7 +664,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
         m = m_new;
         // P buffers of tile i - 2 are free in every CTA once their MMA 2 completed
         if (i >= 2)
-          ok = mbar_wait_cluster(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag,
+          ok = mbar_wait(&phi_free[b], (uint32_t)((i >> 1) - 1) & 1u, abort_flag,
                                  WD_DECODE | 39u) && ok;
         uint32_t pv[16];
 #pragma unroll
@@ -564,42 +675,41 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
         for (int c = 0; c < 4; ++c)
           *reinterpret_cast<uint4*>(prow + ((c ^ ((h >> 1) & 3)) << 4)) =
               make_uint4(pv[4 * c], pv[4 * c + 1], pv[4 * c + 2], pv[4 * c + 3]);
+        al[b * CL_NH + h] = alpha;
         if constexpr (C > 1) {
-          for (int peer = 0; peer < C; ++peer) {
-            if (peer == (int)rank) continue;
-            // this quadrant's received-P slot in the peer
-            const int pq = quad < peer * NOWN ? quad : quad - NOWN;
-            const uint32_t dst = mapa_shared(smem_u32(pr + ((b * (4 - NOWN) + pq) * 32 + lane) * CL_PR_LD),
-                                             (uint32_t)peer);
-            const uint32_t rb = mapa_shared(smem_u32(&pr_full[b * 4 + pq]), (uint32_t)peer);
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              st_async_v4(dst + 16 * c, pv[4 * c], pv[4 * c + 1], pv[4 * c + 2], pv[4 * c + 3], rb);
-            st_async_b32(dst + 64, __float_as_uint(alpha), rb);
+          // the quadrant's 32 P rows (2 KB, already in the peers' swizzled layout) and its 32
+          // rescale factors go to the same places in every peer, by two bulk copies each
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            for (int peer = 0; peer < C; ++peer) {
+              if (peer == (int)rank) continue;
+              const int pq = quad < peer * NOWN ? quad : quad - NOWN;  // peer's slot for it
+              const uint32_t rb = mapa_shared(smem_u32(&pr_full[b * 4 + pq]), (uint32_t)peer);
+              const uint8_t* prows = PS + b * p_bytes + quad * 32 * 64;
+              const float* alq = al + b * CL_NH + quad * 32;
+              bulk_copy_s2s(mapa_shared(smem_u32(prows), (uint32_t)peer), prows, 32 * 64, rb);
+              bulk_copy_s2s(mapa_shared(smem_u32(alq), (uint32_t)peer), alq, 32 * 4, rb);
+            }
           }
         }
-        // p (fp32) of this head for the exact-dim values, and its rescale factor
+        // p (fp32) of this head for the exact-dim values
 #pragma unroll
         for (int t = 0; t < CL_T; ++t) xrow[t] = sc[t];
-        al[b * CL_NH + h] = alpha;
-      } else {
-        // ---- P row and rescale factor of this head from the quadrant's owner
-        if (lane == 0) mbar_arrive_expect_tx(&pr_full[b * 4 + npi], (uint32_t)(32 * 68));
-        ok = mbar_wait_cluster(&pr_full[b * 4 + npi], (uint32_t)(i >> 1) & 1u, abort_flag,
+      }
+      if (i + 1 < ntiles && has_exact) scores(i + 1);
+      if (!own_q) {
+        // ---- the owner's P rows of this quadrant land in PS, its factors in al
+        if (lane == 0) mbar_arrive_expect_tx(&pr_full[b * 4 + npi], (uint32_t)(32 * 64 + 32 * 4));
+        ok = mbar_wait(&pr_full[b * 4 + npi], (uint32_t)(i >> 1) & 1u, abort_flag,
                                WD_DECODE | 40u) && ok;
-        const uint32_t* src = pr + ((b * (4 - NOWN) + npi) * 32 + lane) * CL_PR_LD;
-        uint8_t* prow = PS + b * p_bytes + h * 64;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ ((h >> 1) & 3)) << 4)) =
-              *reinterpret_cast<const uint4*>(src + 4 * c);
-        alpha = __uint_as_float(src[16]);
+        alpha = al[b * CL_NH + h];
       }
       // a head whose reference max rose rescales its U^T row (after the previous tile's
       // MMA 2 of this CTA)
       const bool need = i > 0 && alpha < 1.0f;
       if (__any_sync(0xffffffffu, need)) {
-        ok = mbar_wait_cluster(&phi_free[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag,
+        ok = mbar_wait(&phi_free[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u, abort_flag,
                                WD_DECODE | 41u) && ok;
         __syncwarp();
         tc_fence_after();
@@ -619,53 +729,9 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[b]);
-      asm volatile("bar.sync 2, 128;" ::: "memory");  // p and alpha of the owned heads
-      // ---- exact-dim values: acc += p E_V over this warp's items
-      if (has_exact) {
-#pragma unroll
-        for (int u = 0; u < CL_MAX_IPL; ++u) {
-          if (u < n_items) {
-            const ClExact& me = meta[it_e[u]];
-            const float a = al[b * CL_NH + 32 * (q_first + me.li) + me.row0 + it_jq[u]];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[u][e] *= a;
-          }
-        }
-        for (int sb = 0; sb < nsb; ++sb, ++cc) {
-          const int s = cc % stages;
-          ok = ring_wait(s) && ok;
-          const uint8_t* slotp = ring + s * slot_bytes;
-          const int ntb = min(TB, nt - sb * TB);
-#pragma unroll
-          for (int u = 0; u < CL_MAX_IPL; ++u) {
-            if (u < n_items) {
-              const ClExact& me = meta[it_e[u]];
-              const float* prw = xsb + (me.li * 32 + me.row0 + it_jq[u]) * CL_XS_LD + sb * TB;
-              const uint8_t* col = slotp + me.off + it_c[u] * 16;
-              const int pitch = me.de_ld * 2;
-              float2 a2[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) a2[e] = make_float2(acc[u][2 * e], acc[u][2 * e + 1]);
-#pragma unroll 4
-              for (int t = 0; t < ntb; ++t) {
-                float2 x2[4];
-                bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(col + t * pitch), x2);
-                const float pt = prw[t];
-                const float2 pp = make_float2(pt, pt);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) a2[e] = __ffma2_rn(pp, x2[e], a2[e]);
-              }
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                acc[u][2 * e] = a2[e].x;
-                acc[u][2 * e + 1] = a2[e].y;
-              }
-            }
-          }
-          ring_release(s);
-        }
-      }
+      asm volatile("bar.sync 2, 128;" ::: "memory");  // p and alpha of tile i visible
     }
+    if (ntiles > 0 && has_exact) values(ntiles - 1);
     // ---- split record: running max, sum (owned heads), exact-dim values, U slice
     const bool done = ntiles == 0 || mbar_wait(u_done, 0, abort_flag, WD_DECODE | 42u);
     const bool all_ok = __all_sync(0xffffffffu, ok && done);
@@ -789,5 +855,7 @@ cudaError_t decode_cl_max_clusters(int C, int smem, int* n) {
   }
   return cached_max_clusters(fn, CL_THREADS, (size_t)smem, C, n);
 }
+
+FA_WATCHDOG_READER(read_watchdog_decode_cl)
 
 }  // namespace fa

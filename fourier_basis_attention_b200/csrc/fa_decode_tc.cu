@@ -112,8 +112,9 @@ template <int CPS, int G>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     decode_tc_kernel(const __grid_constant__ DecodeParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base, formed by pointer arithmetic on smem_raw so that the compiler
+  // keeps it (and everything derived from it) in the shared address space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int cta = blockIdx.x;
   const int F2 = p.tc_F2;
   const TcLayout Ly = tc_layout(F2);
@@ -725,5 +726,7 @@ cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t st
     default: return cudaErrorInvalidValue;
   }
 }
+
+FA_WATCHDOG_READER(read_watchdog_decode_tc)
 
 }  // namespace fa

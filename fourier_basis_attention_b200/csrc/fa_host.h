@@ -42,6 +42,8 @@ cudaError_t launch_sensitivity(const fa_plan* plan, const DecodeConfig& c, const
                                const void* K, const void* noise, float* scores, void* workspace,
                                cudaStream_t stream);
 cudaError_t read_and_clear_watchdog(unsigned int* word);
+cudaError_t read_watchdog_decode_tc(unsigned int* word);  // per-unit readers
+cudaError_t read_watchdog_decode_cl(unsigned int* word);
 cudaError_t launch_watchdog_selftest(unsigned int wait_ns, cudaStream_t stream);
 
 // Per-device launch facts, queried once and cached (fa_runtime.cu).

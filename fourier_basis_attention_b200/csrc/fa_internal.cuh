@@ -17,9 +17,18 @@
 namespace fa {
 
 // Watchdog word: 0 = fine; otherwise (kernel id << 8) | wait site. Each translation unit
-// has its own copy; only the compress kernel waits on mbarriers, and fa_device_status
-// reads that unit's copy through read_and_clear_watchdog().
+// has its own copy (a static device variable); every unit whose kernels wait on mbarriers
+// defines a reader with FA_WATCHDOG_READER, and fa_device_status reads all of them.
 static __device__ unsigned int g_watchdog = 0;
+
+// Reads and clears this translation unit's watchdog word (host side).
+#define FA_WATCHDOG_READER(name)                                                     \
+  cudaError_t name(unsigned int* word) {                                             \
+    cudaError_t e_ = cudaMemcpyFromSymbol(word, g_watchdog, sizeof(unsigned int));   \
+    if (e_ != cudaSuccess) return e_;                                                \
+    const unsigned int zero_ = 0;                                                    \
+    return cudaMemcpyToSymbol(g_watchdog, &zero_, sizeof(unsigned int));             \
+  }
 
 enum : unsigned int {
   WD_COMPRESS = 1u << 8,
@@ -434,6 +443,18 @@ __device__ __forceinline__ void mma_commit_mc(uint64_t* bar, uint16_t cta_mask) 
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
       "[%0], %1;" ::"r"(smem_u32(bar)),
       "h"(cta_mask)
+      : "memory");
+}
+
+// Bulk copy of `bytes` from this CTA's shared memory to another CTA's shared memory in the
+// cluster (no multicast), completing on that CTA's mbarrier; dst and rbar from mapa_shared,
+// addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_copy_s2s(uint32_t rdst, const void* ssrc, uint32_t bytes,
+                                              uint32_t rbar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          rdst),
+      "r"(smem_u32(ssrc)), "r"(bytes), "r"(rbar)
       : "memory");
 }
 

@@ -285,7 +285,8 @@ def _ragged_hkv(dcs, Hkv):
     (8, 2, 1023, 2, [96, 100], 4),           # G = 8
     (4, 8, 1023, 5, None, 4),                # 160 query heads: a second, partial head set
     (4, 2, 257, 2, [96, 96], 2),             # 2 F_pad = 264 slots: 192 per CTA
-], ids=["C2_G4_ragged", "C2_G2", "C4_G8", "C4_two_head_sets", "C2_192_slots"])
+    (2, 4, 1023, 3, [100, 64, 96, 128], 4),  # G = 2, a KV head without exact dims
+], ids=["C2_G4_ragged", "C2_G2", "C4_G8", "C4_two_head_sets", "C2_192_slots", "C4_G2_ragged"])
 def test_cluster_decode(G, Hkv, k, B, dcs, cluster):
     w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=B, Hq=Hkv * G, Hkv=Hkv, L=k + 96 + 333, k=k)
     mask = wl.dim_mask(w) if dcs is None else _ragged_hkv(dcs, Hkv)
