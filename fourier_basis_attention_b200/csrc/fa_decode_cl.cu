@@ -13,19 +13,22 @@
 // tensor memory, and it generates only its frequencies of Phi_t. Its MMA 1 then gives a
 // partial S over its slots. The 128 heads form four quadrants of 32 (the TMEM lane
 // quarters); quadrant q is owned by CTA q C / 4. For each tile:
-//   1. every CTA reads its partial S of each quadrant out of tensor memory and sends the
-//      quadrants it does not own to their owners (asynchronous DSMEM stores counted on the
-//      owner's mbarrier);
+//   1. every CTA reads its partial S of each quadrant out of tensor memory, stages the
+//      quadrants it does not own in its shared memory and sends each to its owner as one
+//      bulk shared-to-shared copy across the cluster (counted on the owner's mbarrier);
 //   2. the owner adds the C partials and the exact-dim scores, runs the online softmax
-//      (fp32, lazily raised reference max) and writes the P rows (fp16, 2^7 p) and the
-//      rescale factors of its heads into every CTA of the cluster;
+//      (fp32, lazily raised reference max) and sends the P rows (fp16, 2^7 p) and the
+//      rescale factors of its heads to every CTA of the cluster by bulk copies;
 //   3. each CTA rescales its U^T rows where the reference max rose and issues MMA 2 on its
 //      slots. MMA 2's commit arrives on the same barrier in every CTA of the cluster, which
 //      tells the owners when P buffers may be rewritten.
 // The exact (retained) dims of the owned quadrants' KV heads are streamed by TMA bulk
 // copies (one per KV head and token block, per-KV-head E blocks as stored) into a ring of
-// shared-memory slots fed by one producer thread; exact-dim scores run on warp-level bf16
-// MMAs (query rows x 8 tokens), values on the CUDA cores with fp32 accumulators.
+// shared-memory slots fed by one producer thread. Exact-dim scores run on the CUDA cores
+// (each lane holds its query head's retained q values in registers and serves a group of
+// tokens), values on the CUDA cores with fp32 accumulators. The head warps are software-
+// pipelined: while the partial scores of tile i cross the cluster, they accumulate the
+// values of tile i - 1 and, after the softmax, compute the exact-dim scores of tile i + 1.
 //
 // Warp roles (8 warps): 0 = TMEM owner and MMA issuer; 1 = exact-dim producer; 2-3 = basis
 // generators (thread = frequency, rotation along the tile's tokens from the exactly
