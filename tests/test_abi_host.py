@@ -448,3 +448,19 @@ def test_cache_views_on_host_memory():
     assert c.E("K", 1, 1)[7, 3].item() == 5.0 and c.E("K", 1, 1).sum().item() == 5.0
     # C: [kk][dc_ld] block of (b, g), padding columns past dc
     assert c.C("V", 0, 1).shape == (15, 64) and c.C_raw("V", 0, 1).shape == (15, p.dc_ld[1])
+
+
+def test_c_gpu_program_builds():
+    """The plain-C GPU program (run by the -m gpu tests) compiles and links against the
+    header, the library and the CUDA runtime."""
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location(
+        "gpu_c_program", os.path.join(root, "tests", "test_gpu_c_program.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        exe = os.path.join(d, "c_abi_gpu")
+        mod.build_c_program(exe)
+        assert os.path.getsize(exe) > 0

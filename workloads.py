@@ -175,3 +175,31 @@ def value_noise(w: Workload, device="cpu") -> torch.Tensor:
     """bf16 [B, Hkv, L, D] N(0, 1) draws: the noise of the head-dimension analysis."""
     gen = _gen(device, (w.seed * 1_000_003 + 777_767) & 0x7FFFFFFF)
     return torch.randn(w.B, w.Hkv, w.L, D, generator=gen, device=device).to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------- counter-based draws
+
+_SM64_GAMMA = 0x9E3779B97F4A7C15
+_M64 = (1 << 64) - 1
+
+
+def splitmix64(seed: int, n: int) -> np.ndarray:
+    """The first n outputs (uint64) of SplitMix64 started at state ``seed`` (Steele, Lea
+    and Flood, "Fast splittable pseudorandom number generators", OOPSLA 2014, in the
+    64-bit finaliser form Vigna distributes as splitmix64.c): output i mixes the state
+    seed + (i + 1) * gamma. Counter-based, so a C program reproduces the same stream
+    from the same published definition without sharing code with this module."""
+    i = np.arange(1, n + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed & _M64) + i * np.uint64(_SM64_GAMMA)
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(0xBF58476D1CE4E5B9)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(0x94D049BB133111EB)
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def grid_values(seed: int, n: int) -> np.ndarray:
+    """n values on the grid {-128, ..., 127} / 64 (exact in bf16), from the top byte of
+    each SplitMix64 output read as a signed 8-bit integer."""
+    top = (splitmix64(seed, n) >> np.uint64(56)).astype(np.int64)
+    return np.where(top >= 128, top - 256, top).astype(np.float64) / 64.0
