@@ -54,6 +54,7 @@ struct CkCfg {
 
 struct CompressParams {
   int M, P, k, S, L, Hkv, n_ktiles, n_pairs;
+  int nsplit;  // CTAs (one cluster) that split each unit's token stages; 1 = no split
   const void* K;
   const void* V;
   float norm_single, norm_pair;
@@ -94,19 +95,27 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   uint64_t* drain = accum + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* acc_flag = abort_flag + 1;  // the split epilogue's "accumulators valid"
   unsigned char* perm_s = reinterpret_cast<unsigned char*>(misc + 256);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int pair = blockIdx.x % p.n_pairs;
-  const int head = blockIdx.x / p.n_pairs;  // flattened b * Hkv + g
+  // unit = (head, coefficient-tile pair); with nsplit > 1 the nsplit CTAs of a cluster share
+  // one unit and take contiguous thirds / quarters / ... of its token stages (rank = the
+  // CTA's rank in its one-dimensional cluster)
+  const int unit = blockIdx.x / p.nsplit;
+  const int rank = blockIdx.x - unit * p.nsplit;
+  const int pair = unit % p.n_pairs;
+  const int head = unit / p.n_pairs;  // flattened b * Hkv + g
   const int b = head / p.Hkv;
   const int g = head - b * p.Hkv;
   const int dc = p.dc[g];
   const int kt0 = pair * KT;                       // first coefficient tile of this CTA
   const int kt_n = min(KT, p.n_ktiles - kt0);       // tiles present (>= 1)
   const bool do_pack = (pair == 0);
-  const int nk = (p.M + CK_BK - 1) / CK_BK;
+  const int nk_all = (p.M + CK_BK - 1) / CK_BK;
+  const int st0 = (int)((long long)rank * nk_all / p.nsplit);  // first stage of this CTA
+  const int nk = (int)((long long)(rank + 1) * nk_all / p.nsplit) - st0;  // >= 1 (host rule)
   // A head with no compressed dims needs only the packing pass of the first pair.
   if (dc == 0 && pair != 0) return;
 
@@ -142,7 +151,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       const char* k_rows = static_cast<const char*>(p.K) + (long long)head * p.L * (FA_HEAD_DIM * 2);
       const char* v_rows = static_cast<const char*>(p.V) + (long long)head * p.L * (FA_HEAD_DIM * 2);
       auto prefetch_stage = [&](int st) {
-        const int t = p.S + st * CK_BK;
+        const int t = p.S + (st0 + st) * CK_BK;
         const int n = min(CK_BK, p.L - t);
         if (n > 0) {
           prefetch_l2_bulk(k_rows + (long long)t * (FA_HEAD_DIM * 2), (uint32_t)n * (FA_HEAD_DIM * 2));
@@ -160,10 +169,11 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
           break;
         uint8_t* a_s = stages + s * Cfg::STAGE_BYTES;
         uint8_t* b_s = a_s + Cfg::A_BYTES;
-        const int t = p.S + it * CK_BK;
+        const int t = p.S + (st0 + it) * CK_BK;
         mbar_arrive_expect_tx(&full[s], tx);
         for (int kt = 0; kt < kt_n; ++kt)
-          tma_load_2d(a_s + kt * CK_A_TILE, &tm_phi, &full[s], it * CK_BK, (kt0 + kt) * CK_BM);
+          tma_load_2d(a_s + kt * CK_A_TILE, &tm_phi, &full[s], (st0 + it) * CK_BK,
+                      (kt0 + kt) * CK_BM);
         tma_load_3d(b_s, &tm_k, &full[s], 0, t, head);
         tma_load_3d(b_s + CK_B_BOX, &tm_k, &full[s], 64, t, head);
         tma_load_3d(b_s + 2 * CK_B_BOX, &tm_v, &full[s], 0, t, head);
@@ -243,7 +253,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
         if (!mbar_wait(&full[s], (uint32_t)(it / STAGES) & 1u, abort_flag, WD_COMPRESS | 3u))
           break;
         const uint8_t* b_s = stages + s * Cfg::STAGE_BYTES + Cfg::A_BYTES;
-        const int ntok = min(CK_BK, p.M - it * CK_BK);
+        const int ntok = min(CK_BK, p.M - (st0 + it) * CK_BK);
         for (int c = 0; c < ngrp; ++c) {
           const int i = lane + 32 * c;
           int boff = -1, cbit = 0;
@@ -271,7 +281,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
                 const int tau = pw + j * CK_PACK_WARPS;
                 if (tau < ntok)
                   reinterpret_cast<unsigned short*>((x ? E1 : E0) +
-                                                    (long long)(it * CK_BK + tau) * e_pitch)[i] =
+                                                    (long long)((st0 + it) * CK_BK + tau) * e_pitch)[i] =
                       v[x][j];
               }
           }
@@ -285,7 +295,10 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
     asm volatile("bar.sync 1, 256;" ::: "memory");
     const int acc_ready =
         (dc > 0 && !*abort_flag) ? (mbar_wait(accum, 0, abort_flag, WD_COMPRESS | 4u) ? 1 : 0) : 0;
-    if (dc > 0 && bar1_and_256(acc_ready)) {
+    const int acc_all = bar1_and_256(acc_ready);
+    if (p.nsplit > 1) {
+      if (et == 0) *acc_flag = acc_all;  // read by every thread after the __syncthreads below
+    } else if (dc > 0 && acc_all) {
       tc_fence_after();
       float* stage_f = reinterpret_cast<float*>(stages);
       const int rb = warp & 3;       // TMEM lanes this warp may access: 32*rb .. 32*rb+31
@@ -332,6 +345,83 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
               make_float4(v[0], v[1], v[2], v[3]);
         }
       }
+    }
+  }
+
+  if (p.nsplit > 1 && dc > 0) {
+    // Token-split reduction. Per coefficient tile: every CTA stages its partial sums
+    // (TMEM -> fp32 staging rows, as above); after a cluster barrier, rank r sums rows
+    // [r 128 / nsplit, (r + 1) 128 / nsplit) of the tile over the cluster's CTAs in rank
+    // order 0, 1, ..., nsplit - 1 (distributed shared memory reads), scales and writes them;
+    // a second barrier keeps every staging buffer alive until its readers are done. All
+    // threads of every CTA take both barriers of every tile, aborted or not.
+    __syncthreads();
+    const int acc_ok = *acc_flag;
+    float* stage_f = reinterpret_cast<float*>(stages);
+    const int rows_per = CK_BM / p.nsplit;
+    const int r0 = rank * rows_per;
+    const int dc_ld = p.dc_ld[g];
+    const int nchunk = dc_ld >> 2;
+    const int per_x = rows_per * nchunk;
+    float* const C0 = p.C[0] + (long long)b * p.c_batch + p.c_off[g];
+    float* const C1 = p.C[1] + (long long)b * p.c_batch + p.c_off[g];
+    uint32_t peer[16];
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      peer[r] = r < p.nsplit ? mapa_shared(smem_u32(stage_f), (uint32_t)r) : 0u;
+    for (int kt = 0; kt < kt_n; ++kt) {
+      if (warp >= 2 && acc_ok) {
+        tc_fence_after();
+        const int rb = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int row = rb * 32 + lane;
+#pragma unroll 1
+        for (int cb = 0; cb < FA_HEAD_DIM / 32; ++cb) {
+          uint32_t r[32];
+          const int col = half * FA_HEAD_DIM + cb * 32;
+          tmem_ld_32x32b_x32(tmem_d + ((uint32_t)(rb * 32) << 16) + kt * CK_BN + col, r);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(stage_f + row * CK_STAGE_LD + col);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+        }
+      }
+      cluster_sync_all();  // every CTA's partial of tile kt is staged
+      const int jt = (kt0 + kt) * CK_BM;
+      const int rows = min(CK_BM, p.k - jt);
+      for (int c = threadIdx.x; c < 2 * per_x; c += CK_THREADS) {
+        const int x = c >= per_x ? 1 : 0;
+        const int rem = c - x * per_x;
+        const int r = r0 + rem / nchunk;
+        const int q = rem - (rem / nchunk) * nchunk;
+        if (r >= rows) continue;
+        const int j = jt + r;
+        const int f = (j + 1) >> 1;
+        const float nrm = (f == 0 || 2 * f == p.P) ? p.norm_single : p.norm_pair;
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = q * 4 + e;
+          float acc = 0.0f;
+          if (i < dc) {
+            const uint32_t off = (uint32_t)(r * CK_STAGE_LD + x * FA_HEAD_DIM + perm_s[i]) * 4u;
+            float part[16];
+#pragma unroll
+            for (int s2 = 0; s2 < 16; ++s2)
+              if (s2 < p.nsplit) part[s2] = ld_shared_cluster_f32(peer[s2] + off);
+            acc = part[0];
+#pragma unroll
+            for (int s2 = 1; s2 < 16; ++s2)
+              if (s2 < p.nsplit) acc += part[s2];
+          }
+          v[e] = (i < dc) ? nrm * acc : 0.0f;
+        }
+        *reinterpret_cast<float4*>((x ? C1 : C0) + (long long)j * dc_ld + q * 4) =
+            make_float4(v[0], v[1], v[2], v[3]);
+      }
+      cluster_sync_all();  // the peers' reads of this CTA's staging rows are done
     }
   }
 
@@ -417,6 +507,42 @@ static PFN_encodeTiled get_encode_fn() {
       fn = reinterpret_cast<PFN_encodeTiled>(ptr);
   }
   return fn;
+}
+
+// Token split of the compress units (one unit = one (batch, KV head) and coefficient-tile
+// pair, one CTA). When the units leave most SMs idle (small batches), each unit's token
+// stages are split over a cluster of nsplit CTAs whose partial coefficients are summed in
+// rank order through distributed shared memory. nsplit is the largest of 16, 8, 4, 2 for
+// which units x nsplit CTAs fit on the SMs at once, all units' clusters can be resident
+// together, and every CTA keeps at least 4 stages (256 tokens); else 1. The choice depends
+// only on the plan and the device, so repeated calls give identical bits.
+static cudaError_t compress_split(const void* fn, int smem, long long units, int stages,
+                                  int* nsplit) {
+  *nsplit = 1;
+  int sms = 0;
+  cudaError_t e = device_sm_count(&sms);
+  if (e != cudaSuccess) return e;
+  if (units * 2 > sms) return cudaSuccess;
+  for (int c = 16; c >= 2; c >>= 1) {
+    if (units * c > sms || stages < 4 * c) continue;
+    if (c > 8) {
+      e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        continue;
+      }
+    }
+    int ncl = 0;
+    if (cached_max_clusters(fn, CK_THREADS, (size_t)smem, c, &ncl) != cudaSuccess) {
+      (void)cudaGetLastError();  // this cluster size is not available here
+      continue;
+    }
+    if (ncl >= units) {
+      *nsplit = c;
+      return cudaSuccess;
+    }
+  }
+  return cudaSuccess;
 }
 
 // Returns a CUDA error, or cudaErrorInvalidValue with *why set for a host-side reason.
@@ -505,19 +631,39 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
   // One tile per CTA when k <= 128, else pairs of tiles (512 TMEM columns).
   const int KT = cp.n_ktiles >= 2 ? 2 : 1;
   cp.n_pairs = (cp.n_ktiles + KT - 1) / KT;
-  const long long grid = (long long)cp.n_pairs * n_heads;
+  const long long units = (long long)cp.n_pairs * n_heads;
   const int smem = KT == 2 ? CkCfg<2>::BASE_SMEM : CkCfg<1>::BASE_SMEM;
-  cudaError_t e;
-  if (KT == 2) {
-    e = raise_smem_limit(reinterpret_cast<const void*>(compress_kernel<2>), smem);
-    if (e != cudaSuccess) return e;
-    compress_kernel<2><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
-  } else {
-    e = raise_smem_limit(reinterpret_cast<const void*>(compress_kernel<1>), smem);
-    if (e != cudaSuccess) return e;
-    compress_kernel<1><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
+  const void* fn = KT == 2 ? reinterpret_cast<const void*>(compress_kernel<2>)
+                           : reinterpret_cast<const void*>(compress_kernel<1>);
+  cudaError_t e = raise_smem_limit(fn, smem);
+  if (e != cudaSuccess) return e;
+  int nsplit = 1;
+  if ((e = compress_split(fn, smem, units, (plan->M + CK_BK - 1) / CK_BK, &nsplit)) != cudaSuccess)
+    return e;
+  cp.nsplit = nsplit;
+  const long long grid = units * nsplit;
+  if (nsplit == 1) {
+    if (KT == 2)
+      compress_kernel<2><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
+    else
+      compress_kernel<1><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
+    return cudaGetLastError();
   }
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(CK_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)nsplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (KT == 2) return cudaLaunchKernelEx(&cfg, compress_kernel<2>, tm_phi, tm_k, tm_v, cp);
+  return cudaLaunchKernelEx(&cfg, compress_kernel<1>, tm_phi, tm_k, tm_v, cp);
 }
 
 }  // namespace fa

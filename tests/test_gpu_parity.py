@@ -397,3 +397,28 @@ def test_compress_many_heads_is_deterministic():
     fa.fa_device_status()
     assert torch.equal(c1.C_K, c2.C_K) and torch.equal(c1.C_V, c2.C_V)
     assert torch.equal(c1.E_K, c2.E_K) and torch.equal(c1.E_V, c2.E_V)
+
+
+# ----------------------------------------------------------------------------- token-split compress
+
+@pytest.mark.parametrize("shape", [
+    dict(B=1, Hq=8, Hkv=2, L=20000, k=511),    # 4 units: clusters of up to 16 CTAs
+    dict(B=1, Hq=4, Hkv=1, L=5000, k=255),     # 1 unit, 78 stages: clusters of up to 16
+    dict(B=3, Hq=12, Hkv=3, L=3000, k=63),     # 9 units, 47 stages: clusters of 8
+    dict(B=2, Hq=8, Hkv=4, L=1100, k=127),     # 8 units, 17 stages: clusters of 4
+], ids=["k511_4units", "k255_1unit", "k63_9units", "k127_8units"])
+def test_compress_token_split(shape):
+    """Small batches split each unit's token stages over a cluster and sum the partial
+    coefficients in rank order: parity with the oracle on every head, and repeated calls
+    write identical bits."""
+    w = wl.shrink(wl.LLAMA3_8B_GQA_128K, S=32, R=64, **shape)
+    p = run_small(w)
+    mask = wl.dim_mask(w)
+    K, V = wl.kv_cache(w, "K", device="cuda"), wl.kv_cache(w, "V", device="cuda")
+    phiT = fa.basis_table(p)
+    c1, c2 = fa.Cache(p), fa.Cache(p)
+    fa.fa_compress(p, K, V, phiT, c1)
+    fa.fa_compress(p, K, V, phiT, c2)
+    fa.fa_device_status()
+    assert torch.equal(c1.C_K, c2.C_K) and torch.equal(c1.C_V, c2.C_V)
+    assert torch.equal(c1.E_K, c2.E_K) and torch.equal(c1.E_V, c2.E_V)
