@@ -388,6 +388,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     // so the 8 token rows an ldmatrix reads from 8 slots fall in 8 different banks
     constexpr int RING = EM::RING;
     constexpr int STEP = 512 * NI;
+    // steps per pass of the CUDA-core exact-dim loops (independent chains in flight)
+    constexpr int SB = (EM::NS % 4 == 0 && RING >= 4 && NI <= 4) ? 4 : 1;
     uint8_t* ring = smem + Ly.ring + (warp - 1) * TC_RING_BYTES;
     const int nkv = nvalid / G;
     // this lane's chunks of global step gs, then one commit group (empty past the end)
@@ -410,17 +412,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
       cp_async_commit();
     };
-    // chunks of global step gs (tile-relative token s * TT + tau_l) once this lane's copies
-    // landed; every later step's group may still be in flight
-    auto take = [&](int gs, int s, int nt, uint4 (&x)[NI]) {
-      cp_async_wait<RING - 1>();
-      const int tok = s * EM::TT + tau_l;
+    // chunks of the SB consecutive global steps gs .. gs + SB - 1 (tile steps s .. s + SB - 1)
+    // once this lane's copies landed; every later step's group may still be in flight
+    auto take_batch = [&](int gs, int s, int nt, uint4 (&x)[SB][NI]) {
+      cp_async_wait<RING - SB>();
 #pragma unroll
-      for (int r = 0; r < NI; ++r)
-        x[r] = (ev[r] && tok < nt)
-                   ? *reinterpret_cast<const uint4*>(ring + (gs % RING) * STEP +
-                                                     (((32 * r + lane) ^ (tok & 7)) * 16))
-                   : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < SB; ++u) {
+        const int tok = (s + u) * EM::TT + tau_l;
+#pragma unroll
+        for (int r = 0; r < NI; ++r)
+          x[u][r] = (ev[r] && tok < nt)
+                        ? *reinterpret_cast<const uint4*>(ring + ((gs + u) % RING) * STEP +
+                                                          (((32 * r + lane) ^ (tok & 7)) * 16))
+                        : make_uint4(0, 0, 0, 0);
+      }
     };
     if constexpr (CPS > 0) {
       // rows that are never copied (tokens past the split) are read by the MMA path: they
@@ -479,41 +484,51 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         } else if (nkv > 0) {
           // exact-dim scores: per step, dot products of the lane's chunks with q_e, summed
-          // over the KV head's CPS chunk lanes, into xs[query head][token]
-#pragma unroll 2
-          for (int s1 = 0; s1 < EM::NS; ++s1) {
-            uint4 x[NI];
+          // over the KV head's CPS chunk lanes, into xs[query head][token]. SB steps per
+          // pass: one wait, then SB independent load / multiply / shuffle chains.
+#pragma unroll 1
+          for (int s1 = 0; s1 < EM::NS; s1 += SB) {
             const int gs = i * 2 * EM::NS + s1;
-            take(gs, s1, nt, x);
-            float part[NI][G];
+            uint4 x[SB][NI];
+            take_batch(gs, s1, nt, x);
+            float part[SB][NI][G];
 #pragma unroll
-            for (int r = 0; r < NI; ++r) {
-              float2 x2[4];
-              bf16x8_to_f32x2(x[r], x2);
+            for (int u = 0; u < SB; ++u)
 #pragma unroll
-              for (int hq = 0; hq < G; ++hq) {
-                float2 a = make_float2(0.0f, 0.0f);
+              for (int r = 0; r < NI; ++r) {
+                float2 x2[4];
+                bf16x8_to_f32x2(x[u][r], x2);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) a = __ffma2_rn(qv[r][hq][e], x2[e], a);
-                part[r][hq] = a.x + a.y;
+                for (int hq = 0; hq < G; ++hq) {
+                  float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e) a = __ffma2_rn(qv[r][hq][e], x2[e], a);
+                  part[u][r][hq] = a.x + a.y;
+                }
               }
-            }
 #pragma unroll
             for (int o = 1; o < CPS; o <<= 1)
 #pragma unroll
-              for (int r = 0; r < NI; ++r)
+              for (int u = 0; u < SB; ++u)
 #pragma unroll
-                for (int hq = 0; hq < G; ++hq)
-                  part[r][hq] += __shfl_xor_sync(0xffffffffu, part[r][hq], o);
+                for (int r = 0; r < NI; ++r)
+#pragma unroll
+                  for (int hq = 0; hq < G; ++hq)
+                    part[u][r][hq] += __shfl_xor_sync(0xffffffffu, part[u][r][hq], o);
             if (c_first) {
-              const int tok = s1 * EM::TT + tau_l;
 #pragma unroll
-              for (int r = 0; r < NI; ++r)
+              for (int u = 0; u < SB; ++u) {
+                const int tok = (s1 + u) * EM::TT + tau_l;
 #pragma unroll
-                for (int hq = 0; hq < G; ++hq)
-                  xs[(kap[r] * G + hq) * TC_XS_LD + tok] = part[r][hq];
+                for (int r = 0; r < NI; ++r)
+#pragma unroll
+                  for (int hq = 0; hq < G; ++hq)
+                    xs[(kap[r] * G + hq) * TC_XS_LD + tok] = part[u][r][hq];
+              }
             }
-            issue(gs + RING);  // into the slot just read (its values are consumed above)
+            // into the slots just read (their values are consumed above)
+#pragma unroll
+            for (int u = 0; u < SB; ++u) issue(gs + u + RING);
           }
         } else {
           for (int t = lane; t < 32 * TC_XS_LD; t += 32) xs[t] = 0.0f;
@@ -605,25 +620,30 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         __syncwarp();
         // exact-dim values: accv[r][hq] += p(head kap G + hq, token) E_V chunk
         if (nkv > 0) {
-#pragma unroll 2
-          for (int s1 = 0; s1 < EM::NS; ++s1) {
-            uint4 x[NI];
+#pragma unroll 1
+          for (int s1 = 0; s1 < EM::NS; s1 += SB) {
             const int gs = i * 2 * EM::NS + EM::NS + s1;
-            take(gs, s1, nt, x);
-            const int tok = s1 * EM::TT + tau_l;
+            uint4 x[SB][NI];
+            take_batch(gs, s1, nt, x);
 #pragma unroll
-            for (int r = 0; r < NI; ++r) {
-              float2 x2[4];
-              bf16x8_to_f32x2(x[r], x2);
+            for (int u = 0; u < SB; ++u) {
+              const int tok = (s1 + u) * EM::TT + tau_l;
 #pragma unroll
-              for (int hq = 0; hq < G; ++hq) {
-                const float pv = xs[(kap[r] * G + hq) * TC_XS_LD + tok];
-                const float2 pv2 = make_float2(pv, pv);
+              for (int r = 0; r < NI; ++r) {
+                float2 x2[4];
+                bf16x8_to_f32x2(x[u][r], x2);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) accv[r][hq][e] = __ffma2_rn(pv2, x2[e], accv[r][hq][e]);
+                for (int hq = 0; hq < G; ++hq) {
+                  const float pv = xs[(kap[r] * G + hq) * TC_XS_LD + tok];
+                  const float2 pv2 = make_float2(pv, pv);
+#pragma unroll
+                  for (int e = 0; e < 4; ++e)
+                    accv[r][hq][e] = __ffma2_rn(pv2, x2[e], accv[r][hq][e]);
+                }
               }
             }
-            issue(gs + RING);
+#pragma unroll
+            for (int u = 0; u < SB; ++u) issue(gs + u + RING);
           }
         }
         __syncwarp();  // xs is rewritten by the next tile's scores
