@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch")
     ap.add_argument("--no-clock-probe", action="store_true",
                     help="skip the extra clock-sampling loop after a short timed region")
+    ap.add_argument("--fft-probe", action="store_true",
+                    help="time the cuFFT building blocks of an O(M log M) decode beside fa_decode "
+                         "(k = 511 and k = 1023 workloads); a measurement, not a product path")
     ap.add_argument("--sweep", action="store_true",
                     help="time every single-layer workload and the 32-layer LLaMA-3-8B decode "
                          "sweep (one JSON line each) instead of the default bench line")
@@ -935,10 +938,79 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def run_fft_probe(args):
+    """Measurement for the FFT variant of the decode (the skill page's Steps 2 and 4 use
+    rfft / irfft). An O(M log M) decode of one layer would, per query head: synthesise the
+    compressed-dim scores of all M middle tokens as one inverse real FFT of the zero-padded
+    spectrum w (length P), add the exact-dim scores and take the softmax (one pass over the
+    B Hq x M score matrix), and form u = Phi^T p as one forward real FFT of p. This times those
+    three steps with cuFFT (torch.fft, fp32; the exact-dim stream is not included) at the
+    plan's period P and at the next power of two, beside fa_decode on the same workload
+    (CUDA-graph replays). Library FFTs are a lower bound for a hand-written one."""
+    import torch
+
+    import fourier_basis_attention_b200 as fa
+    import workloads as wl
+    dev = torch.device("cuda", 0)
+    for w in (wl.LLAMA3_8B_GQA_32K, wl.LLAMA3_8B_GQA_128K):
+        mask = wl.dim_mask(w)
+        K = wl.kv_cache(w, "K", device=dev)
+        V = wl.kv_cache(w, "V", device=dev)
+        q = wl.queries(w, device=dev)
+        plan = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+        cache = fa.Cache(plan, device=dev)
+        fa.fa_compress(plan, K, V, fa.basis_table(plan), cache)
+        del K, V
+        ws = torch.empty(fa.fa_decode_workspace_size(plan), dtype=torch.uint8, device=dev)
+        out = torch.empty(w.B, w.Hq, 128, dtype=torch.bfloat16, device=dev)
+        t_dec = _time_graph(lambda s: fa.fa_decode(plan, q, cache, out, ws, 0, s), 30)
+        fa.fa_device_status()
+        del cache, ws
+        torch.cuda.empty_cache()
+        nh = w.B * w.Hq
+        res = {"workload": w.name, "query_heads": nh, "M": plan.M, "k": w.k,
+               "fa_decode_us": round(t_dec * 1e3, 1),
+               "fa_decode_path": SPLIT_NAMES.get(fa.fa_decode_describe(plan, 0).split_kernel)}
+        for P in (plan.P, 1 << (plan.P - 1).bit_length()):
+            spec = torch.zeros(nh, P // 2 + 1, dtype=torch.complex64, device=dev)
+            spec[:, :(w.k + 1) // 2 + 1] = torch.randn(nh, (w.k + 1) // 2 + 1, dtype=torch.complex64,
+                                                      device=dev)
+            sc = torch.empty(nh, P, dtype=torch.float32, device=dev)
+            pr = torch.empty_like(sc)
+            uu = torch.empty(nh, P // 2 + 1, dtype=torch.complex64, device=dev)
+
+            def synth(s):
+                with torch.cuda.stream(s):
+                    torch.fft.irfft(spec, n=P, dim=1, out=sc)
+
+            def softmax(s):
+                with torch.cuda.stream(s):
+                    pr.copy_(torch.softmax(sc, dim=1))
+
+            def analyse(s):
+                with torch.cuda.stream(s):
+                    torch.fft.rfft(pr, dim=1, out=uu)
+
+            ts = [_time_graph(f, 30) for f in (synth, softmax, analyse)]
+            res[f"P{P}"] = {"irfft_scores_us": round(ts[0] * 1e3, 1), "softmax_us": round(ts[1] * 1e3, 1),
+                            "rfft_values_us": round(ts[2] * 1e3, 1),
+                            "sum_us": round(sum(ts) * 1e3, 1)}
+            del spec, sc, pr, uu
+            torch.cuda.empty_cache()
+        print(json.dumps(res), flush=True)
+        del q, out
+
+
+SPLIT_NAMES = {0: "none", 1: "CUDA cores", 2: "tcgen05 token-major", 3: "warp MMA",
+               4: "tcgen05 slot-split cluster"}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.fft_probe:
+        run_fft_probe(args)
     elif args.sweep:
         run_sweep(args)
     else:

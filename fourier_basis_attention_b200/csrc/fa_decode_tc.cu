@@ -389,7 +389,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     constexpr int RING = EM::RING;
     constexpr int STEP = 512 * NI;
     // steps per pass of the CUDA-core exact-dim loops (independent chains in flight)
-    constexpr int SB = (EM::NS % 4 == 0 && RING >= 4 && NI <= 4) ? 4 : 1;
+    constexpr int SB = (EM::NS % 2 == 0 && RING >= 2 && NI <= 4) ? 2 : 1;
     uint8_t* ring = smem + Ly.ring + (warp - 1) * TC_RING_BYTES;
     const int nkv = nvalid / G;
     // this lane's chunks of global step gs, then one commit group (empty past the end)

@@ -422,3 +422,30 @@ def test_compress_token_split(shape):
     fa.fa_device_status()
     assert torch.equal(c1.C_K, c2.C_K) and torch.equal(c1.C_V, c2.C_V)
     assert torch.equal(c1.E_K, c2.E_K) and torch.equal(c1.E_V, c2.E_V)
+
+
+# ----------------------------------------------------------------------------- whole-row head warps
+
+# With Hq = 32 each head warp of the tensor-core decode serves whole token rows of one batch
+# row (G = 1 and 2 with 16- or 32-element KV slices), including a last head set with one
+# populated warp.
+@pytest.mark.parametrize("G,B,rows,ns", [
+    (1, 4, [97, 100, 123, 127] * 8, 0),    # 32-element rows, 4 chunks per lane
+    (1, 5, [114, 120, 126, 124] * 8, 7),   # 16-element rows; 160 heads: last set one warp
+    (2, 4, [97, 128, 108, 120] * 4, 3),    # G = 2, 32-element rows, 2 chunks per lane
+    (2, 5, [126, 120, 128, 116] * 4, 0),   # G = 2, 16-element rows, ragged, 160 heads
+], ids=["G1_w32", "G1_w16_partial_set", "G2_w32", "G2_w16"])
+def test_whole_row_warps_tensor_core(G, B, rows, ns):
+    Hq = 32
+    Hkv = Hq // G
+    w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=B, Hq=Hq, Hkv=Hkv, L=1400, k=255)
+    rng = np.random.default_rng(11)
+    mask = np.zeros((Hkv, D), dtype=np.uint8)
+    for g in range(Hkv):
+        mask[g, rng.permutation(D)[:rows[g]]] = 1
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
+    assert p.e_token_major == 1
+    info = fa.fa_decode_describe(p, ns)
+    assert info.split_kernel == fa.FA_SPLIT_TC_TOKEN_MAJOR
+    run_small(w, mask=mask, num_splits=ns,
+              heads=[(0, 0), (0, Hkv - 1), (B - 1, 0), (B - 1, Hkv // 2), (B - 1, Hkv - 1)])
