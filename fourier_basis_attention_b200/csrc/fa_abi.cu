@@ -41,15 +41,18 @@ int check_ptr(const void* p, const char* name, bool required) {
 // P, kk, G, dc and de (E holds P rows per KV head). E is token-major exactly when the tensor-core decode is used: it can
 // run when k <= 255, G is 1, 2 or 4 and every KV head keeps at most 32 dims, and it is
 // chosen when the k-length work per token and KV head (k G) is at least 255 and there are
-// at least 128 query heads (one full tensor-core head set); below that (k = 63 with
-// G = 4, or small batches) the CUDA-core decode measured faster.
+// at least 128 query heads (one full tensor-core head set), or, for smaller k G (k = 63 with
+// G = 4), when there are at least 1024 query heads (8 head sets). Below that the CUDA-core
+// decode measured faster (LLaMA-3 layer, L = 8K, k = 63: 103 against 115 us at B = 8; the
+// tensor-core decode wins from B = 32: 265 against 344 us, and 452 against 650 us at B = 64).
 void derive_layout(fa_plan* plan) {
   const fa_shape& s = plan->shape;
   int max_de = 0;
   for (int g = 0; g < s.Hkv; ++g) max_de = plan->de[g] > max_de ? plan->de[g] : max_de;
   const int G = plan->G;
   const bool tm = plan->M > 0 && s.k <= 255 && (G == 1 || G == 2 || G == 4) && max_de <= 32 &&
-                  s.k * G >= 255 && (long long)s.B * s.Hq >= 128;
+                  ((s.k * G >= 255 && (long long)s.B * s.Hq >= 128) ||
+                   (long long)s.B * s.Hq >= 1024);
   const int w = max_de == 0 ? 0 : (max_de <= 8 ? 8 : (max_de <= 16 ? 16 : 32));
   plan->e_token_major = tm ? 1 : 0;
   long long ce = 0, ee = 0;

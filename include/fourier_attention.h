@@ -96,8 +96,8 @@ typedef struct fa_shape {
  *       smallest that holds every de[g]; w = 0 when every dim is compressed).
  *     fa_plan_init chooses token-major exactly when fa_decode will run the middle span on
  *     the tensor cores: middle span present, k <= 255, G in {1, 2, 4}, every de[g] <= 32,
- *     k * G >= 255 and B * Hq >= 128 (a warp then reads one token's retained dims of 32
- *     query heads as one coalesced row).
+ *     either k * G >= 255 and B * Hq >= 128, or B * Hq >= 1024 (a warp then reads one
+ *     token's retained dims of 32 query heads as one coalesced row).
  *   C (Fourier coefficients of the middle rows, compressed dims, fp32): block of (b, g)
  *     starts at b * c_batch + c_off[g] and is [kk][dc_ld[g]] row-major,
  *     kk = (M > 0 ? k : 0); columns [dc[g], dc_ld[g]) are zero. Row j is basis function j.

@@ -238,11 +238,12 @@ def test_token_major_choice(w, token_major):
     ([33, 1, 1, 1], 4, 255, 8, None), ([8, 8, 8, 8], 8, 63, 8, None),
     ([8, 8, 8, 8], 4, 257, 8, None), ([8, 8, 8, 8], 4, 63, 8, None),
     ([8, 8, 8, 8], 4, 127, 7, None), ([8, 8, 8, 8], 1, 255, 32, 8),
-    ([8, 8, 8, 8], 2, 127, 16, None)])
+    ([8, 8, 8, 8], 2, 127, 16, None), ([8, 8, 8, 8], 4, 63, 64, 8),
+    ([8, 8, 8, 8], 2, 127, 128, 8), ([8, 8, 8, 8], 4, 63, 63, None)])
 def test_token_major_width(retained, G, k, B, expect):
     """Width = the smallest of 8, 16, 32 holding every KV head's retained dims; blocked
-    (None) past 32 dims, for G = 8, for k > 255, for k G < 255 or fewer than 128 query
-    heads."""
+    (None) past 32 dims, for G = 8, for k > 255, for fewer than 128 query heads, and for
+    k G < 255 unless there are at least 1024 query heads."""
     Hkv = 4
     mask = np.ones((Hkv, 128), dtype=np.uint8)
     for g, r in enumerate(retained):

@@ -449,3 +449,12 @@ def test_whole_row_warps_tensor_core(G, B, rows, ns):
     assert info.split_kernel == fa.FA_SPLIT_TC_TOKEN_MAJOR
     run_small(w, mask=mask, num_splits=ns,
               heads=[(0, 0), (0, Hkv - 1), (B - 1, 0), (B - 1, Hkv // 2), (B - 1, Hkv - 1)])
+
+
+def test_small_k_many_heads_tensor_core():
+    """k G < 255 (k = 63, G = 4) runs on the tensor cores once there are 1024 query heads."""
+    w = wl.shrink(wl.llama3_8b_layer(1, 8192, 0), B=128, Hq=8, Hkv=2, L=1000, R=64, k=63)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    assert p.e_token_major == 1
+    assert fa.fa_decode_describe(p, 0).split_kernel == fa.FA_SPLIT_TC_TOKEN_MAJOR
+    run_small(w, heads=[(0, 0), (0, 1), (63, 1), (127, 0), (127, 1)])
