@@ -51,6 +51,14 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float (&x)[8]) {
   }
 }
 
+// bf16 x 8 -> 4 fp32 pairs (element 2i in .x, 2i + 1 in .y) for paired FMAs.
+__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
+  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+}
+
 // Sink / recent rows of one KV head, rows [fs * FT, fs * FT + FT) of its S + R exact rows
 // (all 128 dims): scores, softmax statistics and values of the G query heads, written as
 // split record n_splits + fs. All DNT threads of the CTA take part; `sm` holds
@@ -66,7 +74,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   float* sc = qs + HL * FA_HEAD_DIM;    // [FT][HL]
   float* mxs = sc + FT * HL;            // [8][HL]
   float* mh = mxs + 8 * HL;             // [HL]
-  float* red = mh + HL;                 // [DNT][8]
+  float* red = mh + HL;                 // [8 warps][16 chunks][4 heads][8]
 
   const __nv_bfloat16* FKh = p.FK + (long long)kvh * p.nF * FA_HEAD_DIM;
   const __nv_bfloat16* FVh = p.FV + (long long)kvh * p.nF * FA_HEAD_DIM;
@@ -81,25 +89,53 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
                       : 0.0f;
   }
   __syncthreads();
-  float s[HL];
+  // scores: warp-cooperative, two rows per load instruction (lanes 0-15 and 16-31, one
+  // 16-byte chunk each) and several row pairs in flight; each lane keeps its chunk of q for
+  // up to 4 query heads in registers, and a 16-lane shuffle sum gives each row's score,
+  // written to sc[row][head]
+  {
+    const int ch = lane & 15, half = lane >> 4;
+    const int npair = (nr + 1) >> 1;
+    for (int hb = 0; hb < G; hb += 4) {
+      float2 qr[4][4];  // q pairs (dims 2e, 2e + 1 of the chunk)
 #pragma unroll
-  for (int h = 0; h < HL; ++h) s[h] = 0.0f;
-  if (tid < nr) {
-    const __nv_bfloat16* row = FKh + (long long)(r0 + tid) * FA_HEAD_DIM;
-    for (int c = 0; c < FA_HEAD_DIM; c += 8) {
-      float x[8];
-      bf16x8_to_f32(*reinterpret_cast<const uint4*>(row + c), x);
+      for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int h = 0; h < HL; ++h) {
-        if (h < G) {
-          const float4 qa = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c);
-          const float4 qb = *reinterpret_cast<const float4*>(qs + h * FA_HEAD_DIM + c + 4);
-          s[h] += qa.x * x[0] + qa.y * x[1] + qa.z * x[2] + qa.w * x[3] + qb.x * x[4] +
-                  qb.y * x[5] + qb.z * x[6] + qb.w * x[7];
+        for (int e = 0; e < 4; ++e)
+          qr[j][e] = (hb + j < G)
+                         ? *reinterpret_cast<const float2*>(qs + (hb + j) * FA_HEAD_DIM + ch * 8 + 2 * e)
+                         : make_float2(0.0f, 0.0f);
+#pragma unroll 4
+      for (int i = warp; i < npair; i += 8) {
+        const int row = 2 * i + half;
+        float2 x[4];
+        bf16x8_to_f32x2(row < nr ? *reinterpret_cast<const uint4*>(FKh + (long long)(r0 + row) * FA_HEAD_DIM + ch * 8)
+                                 : make_uint4(0, 0, 0, 0),
+                        x);
+        float part[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float2 a = make_float2(0.0f, 0.0f);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) a = __ffma2_rn(qr[j][e], x[e], a);
+          part[j] = a.x + a.y;
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+        if (ch == 0 && row < nr) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (hb + j < G) sc[row * HL + hb + j] = part[j];
         }
       }
     }
   }
+  __syncthreads();
+  float s[HL];
+#pragma unroll
+  for (int h = 0; h < HL; ++h) s[h] = (tid < nr && h < G) ? sc[tid * HL + h] : 0.0f;
 #pragma unroll
   for (int h = 0; h < HL; ++h)
     if (tid >= nr || h >= G) s[h] = -INFINITY;
@@ -132,30 +168,62 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
     for (int o = 1; o < 32; o <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
     if (lane == 0) mxs[warp * HL + h] = l[h];
   }
-  // values: item (head h, 8-dim chunk c), token group grp
-  const int items = G * 16;
-  const int it = tid % items, grp = tid / items, ngrp = DNT / items;
-  const int h = it >> 4, c = it & 15;
-  float acc[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
-#pragma unroll 8  // independent row loads in flight
-  for (int rr = grp; rr < nr; rr += ngrp) {
-    const float pv = sc[rr * HL + h];
-    float x[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += pv * x[e];
-  }
-  {
-    float4* dst = reinterpret_cast<float4*>(red + tid * 8);
-    dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-    dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-  }
-  __syncthreads();
+  // values: thread = (16-byte chunk c of a row, row group grp): lanes 0-15 and 16-31 of a warp
+  // read two whole rows per load, and each V row is read once for all G query heads (in
+  // blocks of up to 4 heads). The two row groups of a warp are added by a shuffle, the 8
+  // warps' partials in a fixed order through shared memory.
   const long long bhq = (long long)p.B * p.Hq;
   const int rix = p.n_splits + fs;
-  if (tid < G) {
+  const int c = tid & 15, grp = tid >> 4;
+  constexpr int NGRP = DNT / 16;
+  for (int hb = 0; hb < G; hb += 4) {
+    float2 acc[4][4];  // dims 2e, 2e + 1 of the chunk, per head of the block
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[j][e] = make_float2(0.0f, 0.0f);
+#pragma unroll 4  // independent row loads in flight
+    for (int rr = grp; rr < nr; rr += NGRP) {
+      float2 x[4];
+      bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (hb + j < G) {
+          const float pv = sc[rr * HL + hb + j];
+          const float2 pv2 = make_float2(pv, pv);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[j][e] = __ffma2_rn(pv2, x[e], acc[j][e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[j][e].x += __shfl_xor_sync(0xffffffffu, acc[j][e].x, 16);
+        acc[j][e].y += __shfl_xor_sync(0xffffffffu, acc[j][e].y, 16);
+      }
+    if (lane < 16) {
+      float4* dst = reinterpret_cast<float4*>(red + (warp * 16 + lane) * 32);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        dst[2 * j] = make_float4(acc[j][0].x, acc[j][0].y, acc[j][1].x, acc[j][1].y);
+        dst[2 * j + 1] = make_float4(acc[j][2].x, acc[j][2].y, acc[j][3].x, acc[j][3].y);
+      }
+    }
+    __syncthreads();
+    const int nh = min(4, G - hb);
+    for (int o = tid; o < 16 * nh * 8; o += DNT) {
+      const int c2 = o / (nh * 8), j = (o / 8) % nh, e = o % 8;
+      float v = 0.0f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) v += red[(w * 16 + c2) * 32 + j * 8 + e];
+      p.rec[((long long)rix * bhq + (long long)b * p.Hq + g * G + hb + j) * p.rec_stride + 4 +
+            c2 * 8 + e] = v;
+    }
+    __syncthreads();  // red is rewritten by the next head block
+  }
+  if (tid < G) {  // the warps' sums of p (mxs) are visible after the barriers above
     float ls = 0.0f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) ls += mxs[w * HL + tid];
@@ -163,24 +231,10 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
     rec[0] = mh[tid];
     rec[1] = ls;
   }
-  if (grp == 0) {
-    float v[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = 0.0f;
-    for (int q2 = 0; q2 < ngrp; ++q2) {
-      const float* src = red + (q2 * items + it) * 8;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v[e] += src[e];
-    }
-    float* rec = p.rec + ((long long)rix * bhq + (long long)b * p.Hq + g * G + h) * p.rec_stride +
-                 4 + c * 8;
-    reinterpret_cast<float4*>(rec)[0] = make_float4(v[0], v[1], v[2], v[3]);
-    reinterpret_cast<float4*>(rec)[1] = make_float4(v[4], v[5], v[6], v[7]);
-  }
 }
 
 __host__ __device__ constexpr size_t sink_recent_smem_bytes() {
-  return (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + DNT * 8) * 4;
+  return (size_t)(HL * FA_HEAD_DIM + FT * HL + 8 * HL + HL + 8 * 16 * 32) * 4;
 }
 
 // Warp-MMA split kernel over per-KV-head E blocks, F2 = 512 or 1024 slots.
@@ -189,13 +243,6 @@ size_t decode_hmma_smem_bytes(int F2);
 
 // Tensor-core split kernel over token-major E with de_slot = 0, 8, 16 or 32 retained
 // elements per KV head and token.
-// bf16 x 8 -> 4 fp32 pairs (element 2i in .x, 2i + 1 in .y) for paired FMAs.
-__device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
-  const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    x[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
-}
 
 cudaError_t launch_decode_tc(const DecodeParams& p, int de_slot, cudaStream_t stream);
 
