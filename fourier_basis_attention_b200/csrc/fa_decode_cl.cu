@@ -490,27 +490,42 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
             float* xrw = xsb + sh_row * CL_XS_LD + sb * TB;
             const int ntb = TB;  // tokens past the split's end are masked by the owner
             for (int t0 = sg; t0 < ntb; t0 += 4 * SGN) {
-              float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+              // four tokens x two 8-dim chunks per step: the eight loads are issued before
+              // any of their products (token index clamped into the block, chunk past the
+              // row masked to zero after the load; both reads stay inside the slot: a row
+              // is followed by the next row or by the block's padding)
+              const uint8_t* rowp[4];
 #pragma unroll
-              for (int d8 = 0; d8 < 8; ++d8) {
+              for (int u = 0; u < 4; ++u) rowp[u] = blk + min(t0 + u * SGN, ntb - 1) * sh_pitch;
+              float2 acc4[4];
+#pragma unroll
+              for (int u = 0; u < 4; ++u) acc4[u] = make_float2(0.0f, 0.0f);
+#pragma unroll
+              for (int d8 = 0; d8 < 8; d8 += 2) {
                 if (d8 < sh_c8) {
+                  const bool second = d8 + 1 < sh_c8;
+                  uint4 xq[4][2];
 #pragma unroll
                   for (int u = 0; u < 4; ++u) {
-                    const int t = t0 + u * SGN;
-                    if (t < ntb) {
-                      float2 x2[4];
-                      bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(blk + t * sh_pitch + d8 * 16), x2);
-                      float2 a = make_float2(0.0f, 0.0f);
+                    xq[u][0] = *reinterpret_cast<const uint4*>(rowp[u] + d8 * 16);
+                    xq[u][1] = *reinterpret_cast<const uint4*>(rowp[u] + d8 * 16 + 16);
+                  }
 #pragma unroll
-                      for (int e = 0; e < 4; ++e) a = __ffma2_rn(qv[d8][e], x2[e], a);
-                      acc4[u] += a.x + a.y;
-                    }
+                  for (int u = 0; u < 4; ++u) {
+                    if (!second) xq[u][1] = make_uint4(0, 0, 0, 0);
+                    float2 x2[4], y2[4];
+                    bf16x8_to_f32x2(xq[u][0], x2);
+                    bf16x8_to_f32x2(xq[u][1], y2);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc4[u] = __ffma2_rn(qv[d8][e], x2[e], acc4[u]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc4[u] = __ffma2_rn(qv[d8 + 1][e], y2[e], acc4[u]);
                   }
                 }
               }
 #pragma unroll
               for (int u = 0; u < 4; ++u)
-                if (t0 + u * SGN < ntb) xrw[t0 + u * SGN] = acc4[u] * p.qscale;
+                if (t0 + u * SGN < ntb) xrw[t0 + u * SGN] = (acc4[u].x + acc4[u].y) * p.qscale;
             }
           }
           ring_release(s);
