@@ -559,9 +559,12 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
             const float* prw = xsb + (me.li * 32 + me.row0 + it_jq[u]) * CL_XS_LD + sb * TB;
             const uint8_t* col = slotp + me.off + it_c[u] * 16;
             const int pitch = me.de_ld * 2;
-            float2 a2[4];
+            float2 a2[4], b2[4];  // even / odd tokens: two shorter accumulation chains
 #pragma unroll
-            for (int e = 0; e < 4; ++e) a2[e] = make_float2(acc[u][2 * e], acc[u][2 * e + 1]);
+            for (int e = 0; e < 4; ++e) {
+              a2[e] = make_float2(acc[u][2 * e], acc[u][2 * e + 1]);
+              b2[e] = make_float2(0.0f, 0.0f);
+            }
             int t = 0;
             for (; t + 4 <= ntb; t += 4) {  // four tokens' loads issued together
               uint4 xv[4];
@@ -577,9 +580,16 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
                 bf16x8_to_f32x2(xv[v], x2);
                 const float2 pp = make_float2(pt[v], pt[v]);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) a2[e] = __ffma2_rn(pp, x2[e], a2[e]);
+                for (int e = 0; e < 4; ++e) {
+                  if (v & 1)
+                    b2[e] = __ffma2_rn(pp, x2[e], b2[e]);
+                  else
+                    a2[e] = __ffma2_rn(pp, x2[e], a2[e]);
+                }
               }
             }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) a2[e] = make_float2(a2[e].x + b2[e].x, a2[e].y + b2[e].y);
             for (; t < ntb; ++t) {
               float2 x2[4];
               bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(col + t * pitch), x2);
@@ -664,20 +674,29 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
 #pragma unroll
           for (int t = 0; t < CL_T; ++t) sc[t] += hvalid ? xrow[t] : 0.0f;
         }
-        float tmax = -INFINITY;
 #pragma unroll
-        for (int t = 0; t < CL_T; ++t) {
+        for (int t = 0; t < CL_T; ++t)
           if (t >= nt) sc[t] = -INFINITY;
-          tmax = fmaxf(tmax, sc[t]);
-        }
+        // max and sum over the tile as pairwise trees (short dependency chains)
+        float red[CL_T / 2];
+#pragma unroll
+        for (int t = 0; t < CL_T / 2; ++t) red[t] = fmaxf(sc[2 * t], sc[2 * t + 1]);
+#pragma unroll
+        for (int w2 = CL_T / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int t = 0; t < w2; ++t) red[t] = fmaxf(red[t], red[t + w2]);
+        const float tmax = red[0];
         const float m_new = (tmax > m + CL_LAZY) ? tmax : m;
         alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
-        float psum = 0.0f;
 #pragma unroll
-        for (int t = 0; t < CL_T; ++t) {
-          sc[t] = exp2f(sc[t] - m_new);
-          psum += sc[t];
-        }
+        for (int t = 0; t < CL_T; ++t) sc[t] = exp2f(sc[t] - m_new);
+#pragma unroll
+        for (int t = 0; t < CL_T / 2; ++t) red[t] = sc[2 * t] + sc[2 * t + 1];
+#pragma unroll
+        for (int w2 = CL_T / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+          for (int t = 0; t < w2; ++t) red[t] += red[t + w2];
+        const float psum = red[0];
         l = l * alpha + psum;
         m = m_new;
         // P buffers of tile i - 2 are free in every CTA once their MMA 2 completed
@@ -699,16 +718,14 @@ __global__ void __launch_bounds__(CL_THREADS, 1)
           // rescale factors go to the same places in every peer, by two bulk copies each
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) {
-            for (int peer = 0; peer < C; ++peer) {
-              if (peer == (int)rank) continue;
-              const int pq = quad < peer * NOWN ? quad : quad - NOWN;  // peer's slot for it
-              const uint32_t rb = mapa_shared(smem_u32(&pr_full[b * 4 + pq]), (uint32_t)peer);
-              const uint8_t* prows = PS + b * p_bytes + quad * 32 * 64;
-              const float* alq = al + b * CL_NH + quad * 32;
-              bulk_copy_s2s(mapa_shared(smem_u32(prows), (uint32_t)peer), prows, 32 * 64, rb);
-              bulk_copy_s2s(mapa_shared(smem_u32(alq), (uint32_t)peer), alq, 32 * 4, rb);
-            }
+          if (lane < C && lane != (int)rank) {  // lane p sends to peer p
+            const int peer = lane;
+            const int pq = quad < peer * NOWN ? quad : quad - NOWN;  // peer's slot for it
+            const uint32_t rb = mapa_shared(smem_u32(&pr_full[b * 4 + pq]), (uint32_t)peer);
+            const uint8_t* prows = PS + b * p_bytes + quad * 32 * 64;
+            const float* alq = al + b * CL_NH + quad * 32;
+            bulk_copy_s2s(mapa_shared(smem_u32(prows), (uint32_t)peer), prows, 32 * 64, rb);
+            bulk_copy_s2s(mapa_shared(smem_u32(alq), (uint32_t)peer), alq, 32 * 4, rb);
           }
         }
         // p (fp32) of this head for the exact-dim values

@@ -547,20 +547,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
       for (int t = 0; t < TC_T; ++t)
         sc[t] = hvalid ? __uint_as_float(sr[t]) * w_unscale + sc[t] : 0.0f;
-      float tmax = -INFINITY;
 #pragma unroll
-      for (int t = 0; t < TC_T; ++t) {
+      for (int t = 0; t < TC_T; ++t)
         if (t >= nt) sc[t] = -INFINITY;
-        tmax = fmaxf(tmax, sc[t]);
-      }
+      // max and sum over the tile as pairwise trees (short dependency chains)
+      float red[TC_T / 2];
+#pragma unroll
+      for (int t = 0; t < TC_T / 2; ++t) red[t] = fmaxf(sc[2 * t], sc[2 * t + 1]);
+#pragma unroll
+      for (int w2 = TC_T / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int t = 0; t < w2; ++t) red[t] = fmaxf(red[t], red[t + w2]);
+      const float tmax = red[0];
       const float m_new = (tmax > m + TC_LAZY) ? tmax : m;  // m = -inf: the first tile's max
       const float alpha = (m == -INFINITY) ? 0.0f : exp2f(m - m_new);
-      float psum = 0.0f;
 #pragma unroll
-      for (int t = 0; t < TC_T; ++t) {
-        sc[t] = exp2f(sc[t] - m_new);  // -inf -> 0
-        psum += sc[t];
-      }
+      for (int t = 0; t < TC_T; ++t) sc[t] = exp2f(sc[t] - m_new);  // -inf -> 0
+#pragma unroll
+      for (int t = 0; t < TC_T / 2; ++t) red[t] = sc[2 * t] + sc[2 * t + 1];
+#pragma unroll
+      for (int w2 = TC_T / 4; w2 >= 1; w2 >>= 1)
+#pragma unroll
+        for (int t = 0; t < w2; ++t) red[t] += red[t + w2];
+      const float psum = red[0];
       l = l * alpha + psum;
       m = m_new;
       // a head whose reference max rose rescales its U^T row (after the previous tile's
