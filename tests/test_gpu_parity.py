@@ -458,3 +458,20 @@ def test_small_k_many_heads_tensor_core():
     assert p.e_token_major == 1
     assert fa.fa_decode_describe(p, 0).split_kernel == fa.FA_SPLIT_TC_TOKEN_MAJOR
     run_small(w, heads=[(0, 0), (0, 1), (63, 1), (127, 0), (127, 1)])
+
+
+def test_compress_token_split_extreme_masks():
+    """Token split with a head whose dims are all compressed (no E rows) and one with none
+    compressed (no coefficients: the split CTAs only pack E)."""
+    w = wl.shrink(wl.LLAMA3_8B_GQA_128K, B=1, Hq=8, Hkv=2, L=5000, S=32, R=64, k=255)
+    mask = np.zeros((2, D), dtype=np.uint8)
+    mask[0, :] = 1
+    p = run_small(w, mask=mask)
+    assert p.dc[0] == 128 and p.dc[1] == 0
+    K, V = wl.kv_cache(w, "K", device="cuda"), wl.kv_cache(w, "V", device="cuda")
+    phiT = fa.basis_table(p)
+    c1, c2 = fa.Cache(p), fa.Cache(p)
+    fa.fa_compress(p, K, V, phiT, c1)
+    fa.fa_compress(p, K, V, phiT, c2)
+    fa.fa_device_status()
+    assert torch.equal(c1.C_K, c2.C_K) and torch.equal(c1.E_V, c2.E_V)
