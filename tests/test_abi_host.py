@@ -396,8 +396,8 @@ def test_plan_layout_properties(B, Hkv, G, L, S, R, k, extra, seed):
     assert p.S + p.M + p.R == L and p.P >= p.M
     assert p.f_elems == B * Hkv * (p.S + p.R) * 128
     de = [p.de[g] for g in range(Hkv)]
-    tm = (p.M > 0 and k <= 255 and G in (1, 2, 4) and max(de) <= 32 and k * G >= 255
-          and B * Hq >= 128)
+    tm = (p.M > 0 and k <= 255 and G in (1, 2, 4) and max(de) <= 32
+          and ((k * G >= 255 and B * Hq >= 128) or B * Hq >= 1024))
     assert p.e_token_major == int(tm)
     for g in range(Hkv):
         cd, ed = fa.perm_lists(p, g)
