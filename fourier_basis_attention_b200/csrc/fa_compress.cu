@@ -649,8 +649,7 @@ cudaError_t launch_compress(const fa_plan* plan, const void* K, const void* V,
       compress_kernel<1><<<(unsigned)grid, CK_THREADS, smem, stream>>>(tm_phi, tm_k, tm_v, cp);
     return cudaGetLastError();
   }
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
+  cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid, 1, 1);
   cfg.blockDim = dim3(CK_THREADS, 1, 1);
   cfg.dynamicSmemBytes = (size_t)smem;
