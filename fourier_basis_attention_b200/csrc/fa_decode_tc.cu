@@ -17,8 +17,10 @@
 // 128-byte swizzle: MMA 1 reads it as its K-major B operand, MMA 2 as its MN-major B
 // operand (the layout compress uses for the cache rows).
 //
-// Warp roles: warp 0 = TMEM owner and MMA issuer (one thread); warps 1-4 = head warps,
-// each owning the 32 query heads of its TMEM lane quadrant; warps 5-7 = basis generators
+// Warp roles: warp 0 = TMEM owner and MMA issuer (one thread); warps 1-8 = head warps, two
+// per TMEM lane quadrant (warps w and w + 4 share quadrant w & 3, each taking 16 of its 32
+// query heads; the pair exchanges its rescale factors through shared memory and one of them
+// rescales the quadrant's U rows); warps 9-11 = basis generators
 // (thread = frequency; rotation recurrence along the tile's tokens, started each tile from
 // the exactly reduced phase). Tiles are double-buffered (Phi, P, S); every wait is bounded.
 //
@@ -41,8 +43,8 @@ namespace fa {
 
 constexpr int TC_NH = 128;      // query heads per CTA = MMA M = TMEM lanes
 constexpr int TC_T = 32;        // tokens per tile
-constexpr int TC_THREADS = 256; // 8 warps
-constexpr int TC_GEN = 96;      // generator threads (warps 5-7)
+constexpr int TC_THREADS = 384; // 12 warps
+constexpr int TC_GEN = 96;      // generator threads (warps 9-11)
 
 // The reference max is raised lazily: only when a tile's max exceeds it by more than
 // TC_LAZY (log2 units) are U, the value accumulator and the sum rescaled, so the head
@@ -81,7 +83,7 @@ __host__ __device__ inline TcLayout tc_layout(int F2) {
   L.xs = L.p + 2 * TC_NH * TC_T * 2;
   L.ring = L.xs + 4 * 32 * TC_XS_LD * 4;
   L.misc = L.ring + 4 * tc_ring_bytes(F2);
-  L.total = L.misc + 256 + 1024;  // + alignment slack
+  L.total = L.misc + 256 + 2 * 4 * 32 * 4 + 1024;  // + rescale factors + alignment slack
   return L;
 }
 
@@ -102,7 +104,7 @@ __device__ __forceinline__ uint32_t pack_half2(float a, float b) {
 // l / CH of the step (all warp-local).
 template <int CPS, int G, int RB>
 struct EMap {
-  static constexpr int NK = 32 / G;                                  // KV heads per warp
+  static constexpr int NK = 16 / G;                                  // KV heads per warp
   static constexpr int CH = CPS > 0 ? NK * CPS : 32;                 // chunks per token
   static constexpr int TT = CH >= 32 ? 1 : 32 / CH;                  // tokens per step
   static constexpr int NI = CH >= 32 ? CH / 32 : 1;                  // loads per lane per step
@@ -153,7 +155,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&phi_full[b], TC_GEN / 32);
       mbar_init(&phi_free[b], 1);
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 4);
+      mbar_init(&p_full[b], 8);
     }
     mbar_init(u_done, 1);
     *abort_flag = 0;
@@ -175,18 +177,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   // column); S is scaled back by 2^e on readout
   const int h = (warp & 3) * 32 + lane;  // TMEM lane of a head thread
   const long long gh = (long long)hg * TC_NH + h;
+  // two head warps per TMEM lane quadrant: warps 1-4 (half 0) and 5-8 (half 1) both serve
+  // quadrant warp & 3; warps 1-4 also write W
+  const bool any_head = warp >= 1 && warp <= 8;
   const bool is_head = warp >= 1 && warp <= 4;
-  const bool hvalid = is_head && gh < bhq;
+  const bool qvalid = any_head && gh < bhq;  // the quadrant row of this lane is a query head
   float w_unscale = 1.0f;
-  if (is_head) {
+  if (any_head) {
     const float* wsrc = p.qw + gh * p.qw_stride + FA_HEAD_DIM;
-    const int nslot = hvalid ? 2 * p.F_pad : 0;
+    const int nslot = qvalid ? 2 * p.F_pad : 0;
     float wmax = 0.0f;
     for (int slot = 0; slot < nslot; ++slot) wmax = fmaxf(wmax, fabsf(wsrc[slot]));
     int ex = 0;
     if (wmax > 0.0f) frexpf(wmax, &ex);  // wmax < 2^ex
     const float w_scale = ldexpf(1.0f, -ex);
     w_unscale = ldexpf(1.0f, ex);
+    if (is_head) {
     const uint32_t lanebase_w = (uint32_t)((warp & 3) * 32) << 16;
     for (int c64 = 0; c64 < F2 / 64; ++c64) {  // 64 slots: one swizzle atom, 32 TMEM columns
       uint32_t lo32[32];
@@ -209,6 +215,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     tmem_st_wait();
     fence_proxy_async_smem();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -276,13 +283,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       while (!mbar_try_wait(u_done, 0) && globaltimer_ns() - w0 < 2000000000ull) {
       }
     }
-  } else if (warp >= 5) {
+  } else if (warp >= 9) {
     // -------------------------------------------------------------------- basis generators
     // thread gt: frequencies gt and gt + 96; per tile the unit phasor of f (t0 + tau) / M
     // for tau = 0 .. 31 by rotation, started from the exactly reduced phase f t0 mod M.
     // Slots 2f (cos) and 2f + 1 (sin) are one fp16 pair: atom f / 32, byte 4 (f % 32) of
     // the token's 128-byte row, 16-byte chunk swizzled by the token.
-    const int gt = threadIdx.x - 160;
+    const int gt = threadIdx.x - 288;
     const int nf = F2 / 2;
     float ra[2], rb[2];  // cos, sin of 2 pi f / P
 #pragma unroll
@@ -322,11 +329,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------------- head warps
-    using EM = EMap<CPS, G, RB>;
+    // this warp: query heads [16 hf, 16 hf + 16) of TMEM lane quadrant warp & 3, half of the
+    // quadrant's ring space; its softmax lanes are lanes 16 hf .. 16 hf + 15 (`mine`)
+    using EM = EMap<CPS, G, RB / 2>;
     constexpr int NI = EM::NI;
+    const int hf = (warp - 1) >> 2;
+    const int pair = (warp - 1) & 3;
+    const bool mine = (lane >> 4) == hf;
+    const bool hvalid = mine && qvalid;
     const uint32_t lanebase = (uint32_t)((warp & 3) * 32) << 16;
-    const long long gbase = (long long)hg * TC_NH + (warp & 3) * 32;  // head of lane 0
-    const int nvalid = (int)max(0LL, min(32LL, bhq - gbase));
+    const long long gbase = (long long)hg * TC_NH + (warp & 3) * 32 + 16 * hf;  // warp's first head
+    const int nvalid = (int)max(0LL, min(16LL, bhq - gbase));
+    // rescale factors of the pair's 32 heads, by tile parity (half 1 -> half 0)
+    float* al_s = reinterpret_cast<float*>(smem + Ly.misc + 256);
     const int tau_l = EM::TT > 1 ? lane / EM::CH : 0;  // token of this lane within a step
     // per load r: the lane's KV head (warp-local), its element offset, q_e, accumulator
     int kap[NI], c8r[NI], de_r[NI];
@@ -387,7 +402,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     float m = -INFINITY, l = 0.0f;
     bool ok = true;
-    float* xs = reinterpret_cast<float*>(smem + Ly.xs) + (warp - 1) * 32 * TC_XS_LD;
+    // the quadrant's [32 heads][token] buffer; this warp's rows start at row 16 hf
+    float* xsq = reinterpret_cast<float*>(smem + Ly.xs) + pair * 32 * TC_XS_LD;
+    float* xs = xsq + 16 * hf * TC_XS_LD;
     const int c_first = ((lane % EM::CH) % EM::CPS1) == 0;  // first chunk lane of its KV head
 
     // exact-dim ring: global step gs = (tile, phase K / V, step) uses slot gs % RING; chunk c
@@ -397,7 +414,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     constexpr int STEP = 512 * NI;
     // steps per pass of the CUDA-core exact-dim loops (independent chains in flight)
     constexpr int SB = (EM::NS % 2 == 0 && RING >= 2 && NI <= 4) ? 2 : 1;
-    uint8_t* ring = smem + Ly.ring + (warp - 1) * RB;
+    uint8_t* ring = smem + Ly.ring + (warp - 1) * (RB / 2);
     const int nkv = nvalid / G;
     // this lane's chunks of global step gs, then one commit group (empty past the end)
     auto issue = [&](int gs) {
@@ -437,7 +454,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     if constexpr (CPS > 0) {
       // rows that are never copied (tokens past the split) are read by the MMA path: they
       // must hold finite values
-      for (int o = lane * 16; o < RB; o += 32 * 16)
+      for (int o = lane * 16; o < RB / 2; o += 32 * 16)
         *reinterpret_cast<uint4*>(ring + o) = make_uint4(0, 0, 0, 0);
       __syncwarp();
       if (nkv > 0)
@@ -538,13 +555,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             for (int u = 0; u < SB; ++u) issue(gs + u + RING);
           }
         } else {
-          for (int t = lane; t < 32 * TC_XS_LD; t += 32) xs[t] = 0.0f;
+          for (int t = lane; t < 16 * TC_XS_LD; t += 32) xs[t] = 0.0f;
         }
         __syncwarp();
       }
       float sc[TC_T];
 #pragma unroll
-      for (int t = 0; t < TC_T; ++t) sc[t] = CPS > 0 ? xs[lane * TC_XS_LD + t] : 0.0f;
+      for (int t = 0; t < TC_T; ++t) sc[t] = (CPS > 0 && mine) ? xsq[lane * TC_XS_LD + t] : 0.0f;
       ok = mbar_wait(&s_full[b], (uint32_t)(i >> 1) & 1u, abort_flag, WD_DECODE | 5u) && ok;
       __syncwarp();  // tcgen05.ld is warp-collective
       tc_fence_after();
@@ -580,30 +597,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       l = l * alpha + psum;
       m = m_new;
       // a head whose reference max rose rescales its U^T row (after the previous tile's
-      // MMA 2) and its value accumulators
-      const bool need = i > 0 && alpha < 1.0f;
-      if (__any_sync(0xffffffffu, need)) {
+      // MMA 2; half 0 of the pair does the quadrant's 32 rows, with half 1's factors passed
+      // through shared memory) and its value accumulators
+      const float a_own = (mine && i > 0 && alpha < 1.0f) ? alpha : 1.0f;
+      if (hf == 1 && mine) al_s[(b * 4 + pair) * 32 + lane] = a_own;
+      asm volatile("bar.sync %0, 64;" ::"r"(2 + pair) : "memory");  // the pair's factors
+      const float a_row = mine ? a_own : al_s[(b * 4 + pair) * 32 + lane];
+      if (hf == 0 && __any_sync(0xffffffffu, a_row < 1.0f)) {
         const bool w_ok = mbar_wait(&phi_free[(i - 1) & 1], (uint32_t)((i - 1) >> 1) & 1u,
                                     abort_flag, WD_DECODE | 6u);
         ok = ok && w_ok;
         __syncwarp();
         tc_fence_after();
-        const float a = need ? alpha : 1.0f;
 #pragma unroll 1
         for (int c = 0; c < F2 / 32; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(tmem_u + lanebase + c * 32, r);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * a);
+          for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * a_row);
           tmem_st_32x32b_x32(tmem_u + lanebase + c * 32, r);
         }
         tmem_st_wait();
+      }
+      if (__any_sync(0xffffffffu, a_own < 1.0f)) {
 #pragma unroll
         for (int r = 0; r < NI; ++r)
 #pragma unroll
           for (int hq = 0; hq < G; ++hq) {
-            const float ah = __shfl_sync(0xffffffffu, a, kap[r] * G + hq);
+            const float ah = __shfl_sync(0xffffffffu, a_own, 16 * hf + kap[r] * G + hq);
 #pragma unroll
             for (int e = 0; e < 4; ++e) accv[r][hq][e] = __fmul2_rn(accv[r][hq][e], make_float2(ah, ah));
           }
@@ -618,6 +640,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint8_t* prow = PS + b * p_bytes + h * 64;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
+        if (!mine) break;  // the other half of the pair writes these rows
         uint32_t pv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -632,7 +655,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if constexpr (CPS > 0) {
         // p of this head for the exact-dim values
 #pragma unroll
-        for (int t = 0; t < TC_T; ++t) xs[lane * TC_XS_LD + t] = sc[t];
+        for (int t = 0; t < TC_T; ++t)
+          if (mine) xsq[lane * TC_XS_LD + t] = sc[t];
         __syncwarp();
         // exact-dim values: accv[r][hq] += p(head kap G + hq, token) E_V chunk
         if (nkv > 0) {
