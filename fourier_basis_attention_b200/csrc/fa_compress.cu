@@ -273,6 +273,13 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
                 v[x][j] = *reinterpret_cast<const unsigned short*>(
                     b_s + x * 2 * CK_B_BOX + tau * 128 + boff + ((cbit ^ (tau & 7)) << 4));
             }
+          if (c == ngrp - 1) {
+            // every shared-memory value of the stage is loaded (the release orders this
+            // warp's loads before the arrival): the stage may be refilled while the rows
+            // are stored
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+          }
           if (i < de_ld) {
 #pragma unroll
             for (int x = 0; x < 2; ++x)
@@ -286,9 +293,10 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
               }
           }
         }
-        // the stage's shared-memory values have been consumed: it may be refilled
-        __syncwarp();
-        if (lane == 0) mbar_arrive_relaxed(&empty[s]);
+        if (ngrp == 0) {  // nothing retained: only the release
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+        }
       }
     }
     // all pack warps are done reading the stages before any staging write reuses them
