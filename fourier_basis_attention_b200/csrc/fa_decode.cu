@@ -811,10 +811,15 @@ cudaError_t decode_configure(const fa_plan* plan, int requested, DecodeConfig* c
   while (cols < c->tc_F2 + 64 + c->tc_F2 / 2) cols <<= 1;
   c->tc_tmem_cols = cols;
   // The cluster tensor-core split kernel takes the plans with 256 <= k <= 1023 on
-  // per-KV-head E blocks when G is 2, 4 or 8 and its per-CTA buffers fit (it replaces the
-  // warp-MMA kernel there).
+  // per-KV-head E blocks when G is 2, 4 or 8, its per-CTA buffers fit, and its 128-head
+  // sets are at least three quarters full (it replaces the warp-MMA kernel there). A set's
+  // cost hardly depends on how many of its heads are valid: with 32 query heads the
+  // warp-MMA kernel (16 heads per CTA) decodes in 0.6-0.75 of its time, from 96 on the
+  // cluster kernel wins (up to 1.6x at 128).
   c->cl = 0;
-  if (!c->tc && M > 0 && (plan->G == 2 || plan->G == 4 || plan->G == 8)) {
+  const long long nq = (long long)sh.B * sh.Hq;
+  const bool sets_full = 4 * nq >= 3 * 128 * ((nq + 127) / 128);
+  if (!c->tc && M > 0 && sets_full && (plan->G == 2 || plan->G == 4 || plan->G == 8)) {
     const int slots = 2 * c->F_pad;
     const int C = slots <= 256 ? 1 : (slots <= 512 ? 2 : (slots <= 1024 ? 4 : 0));
     if (C >= 2 && de_ld_max <= 64) cl_configure(plan, C, slots, c);

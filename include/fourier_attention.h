@@ -222,7 +222,9 @@ enum fa_split_kernel {
   FA_SPLIT_CUDA_CORES = 1,  /* fp32 CUDA-core split kernel */
   FA_SPLIT_TC_TOKEN_MAJOR = 2, /* tcgen05 split kernel over token-major E (k <= 255) */
   FA_SPLIT_WARP_MMA = 3,    /* warp-level MMA split kernel (256 <= k <= 1023) */
-  FA_SPLIT_TC_CLUSTER = 4   /* tcgen05 split kernel, coefficient slots split over a cluster */
+  FA_SPLIT_TC_CLUSTER = 4   /* tcgen05 split kernel, coefficient slots split over a cluster
+                               (256 <= k <= 1023, G in {2, 4, 8}, B * Hq filling its sets of
+                               128 query heads at least three quarters; else warp MMA) */
 };
 typedef struct fa_decode_info {
   int32_t split_kernel, num_splits, cluster, launches;

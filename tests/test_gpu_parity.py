@@ -277,15 +277,17 @@ def _ragged_hkv(dcs, Hkv):
 
 
 # Plans with 256 <= k <= 1023, G in {2, 4, 8} and per-KV-head E blocks run the middle span
-# on the cluster tensor-core kernel: the coefficient slots are split over 2 (k <= 511) or 4
-# CTAs of a thread-block cluster, partial scores summed by each quadrant's owner CTA.
+# on the cluster tensor-core kernel when their 128-query-head sets are at least three
+# quarters full: the coefficient slots are split over 2 (k <= 511) or 4 CTAs of a
+# thread-block cluster, partial scores summed by each quadrant's owner CTA. Every case
+# leaves invalid heads in its last set.
 @pytest.mark.parametrize("G,Hkv,k,B,dcs,cluster", [
-    (4, 2, 511, 3, [96, 64], 2),             # ragged exact dims (32 / 64 per KV head)
-    (2, 4, 511, 5, [96, 64, 90, 120], 2),    # G = 2: 32 exact KV heads per CTA
-    (8, 2, 1023, 2, [96, 100], 4),           # G = 8
-    (4, 8, 1023, 5, None, 4),                # 160 query heads: a second, partial head set
-    (4, 2, 257, 2, [96, 96], 2),             # 2 F_pad = 264 slots: 192 per CTA
-    (2, 4, 1023, 3, [100, 64, 96, 128], 4),  # G = 2, a KV head without exact dims
+    (4, 2, 511, 12, [96, 64], 2),            # ragged exact dims (32 / 64 per KV head)
+    (2, 4, 511, 13, [96, 64, 90, 120], 2),   # G = 2: 32 exact KV heads per CTA; 104 heads
+    (8, 2, 1023, 6, [96, 100], 4),           # G = 8
+    (4, 8, 1023, 6, None, 4),                # 192 query heads: a second, half-full head set
+    (4, 2, 257, 12, [96, 96], 2),            # 2 F_pad = 264 slots: 192 per CTA
+    (2, 4, 1023, 12, [100, 64, 96, 128], 4), # G = 2, a KV head without exact dims
 ], ids=["C2_G4_ragged", "C2_G2", "C4_G8", "C4_two_head_sets", "C2_192_slots", "C4_G2_ragged"])
 def test_cluster_decode(G, Hkv, k, B, dcs, cluster):
     w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=B, Hq=Hkv * G, Hkv=Hkv, L=k + 96 + 333, k=k)
@@ -293,7 +295,18 @@ def test_cluster_decode(G, Hkv, k, B, dcs, cluster):
     p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, mask)
     info = fa.fa_decode_describe(p, 1)
     assert info.split_kernel == fa.FA_SPLIT_TC_CLUSTER and info.cluster == cluster
-    run_small(w, mask=mask)
+    run_small(w, mask=mask, heads=sorted({(0, 0), (0, Hkv - 1), (B // 2, Hkv // 2),
+                                          (B - 1, 0), (B - 1, Hkv - 1)}))
+
+
+@pytest.mark.parametrize("B,kind", [(1, 3), (2, 3), (3, 4)])
+def test_cluster_decode_needs_full_head_sets(B, kind):
+    """32 or 64 query heads (a quarter or half of a 128-head set) go to the warp-MMA kernel,
+    96 to the cluster kernel; both agree with the oracle."""
+    w = wl.shrink(wl.LLAMA3_8B_GQA_32K, B=B, L=1800)
+    p = fa.fa_plan_init(w.B, w.Hq, w.Hkv, w.L, w.S, w.R, w.k, wl.dim_mask(w))
+    assert fa.fa_decode_describe(p, 0).split_kernel == kind
+    run_small(w, heads=[(0, 0), (B - 1, w.Hkv - 1)])
 
 
 @pytest.mark.parametrize("ns", [1, 5, 1000])
