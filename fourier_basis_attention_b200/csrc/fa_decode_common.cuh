@@ -64,7 +64,10 @@ __device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
 // split record n_splits + fs. All DNT threads of the CTA take part; `sm` holds
 // sink_recent_smem_bytes() bytes. Run as extra CTAs of the CUDA-core split kernel, or of the
 // prologue launch on the tensor-core and warp-MMA paths.
-__device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float* sm, int fid) {
+// NJ: query heads per block of the score and value passes (1, 2 or 4: G for G < 4), so that
+// MHA and G = 2 plans do no arithmetic or shuffles for empty heads.
+template <int NJ>
+__device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, float* sm, int fid) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int kvh = fid / p.n_fsplits, fs = fid - (fid / p.n_fsplits) * p.n_fsplits;
   const int b = kvh / p.Hkv, g = kvh - (kvh / p.Hkv) * p.Hkv;
@@ -96,10 +99,10 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   {
     const int ch = lane & 15, half = lane >> 4;
     const int npair = (nr + 1) >> 1;
-    for (int hb = 0; hb < G; hb += 4) {
-      float2 qr[4][4];  // q pairs (dims 2e, 2e + 1 of the chunk)
+    for (int hb = 0; hb < G; hb += NJ) {
+      float2 qr[NJ][4];  // q pairs (dims 2e, 2e + 1 of the chunk)
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
+      for (int j = 0; j < NJ; ++j)
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           qr[j][e] = (hb + j < G)
@@ -112,9 +115,9 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
         bf16x8_to_f32x2(row < nr ? *reinterpret_cast<const uint4*>(FKh + (long long)(r0 + row) * FA_HEAD_DIM + ch * 8)
                                  : make_uint4(0, 0, 0, 0),
                         x);
-        float part[4];
+        float part[NJ];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < NJ; ++j) {
           float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
           for (int e = 0; e < 4; ++e) a = __ffma2_rn(qr[j][e], x[e], a);
@@ -123,10 +126,10 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
 #pragma unroll
         for (int o = 1; o < 16; o <<= 1)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
+          for (int j = 0; j < NJ; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
         if (ch == 0 && row < nr) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
+          for (int j = 0; j < NJ; ++j)
             if (hb + j < G) sc[row * HL + hb + j] = part[j];
         }
       }
@@ -141,6 +144,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
     if (tid >= nr || h >= G) s[h] = -INFINITY;
 #pragma unroll
   for (int h = 0; h < HL; ++h) {
+    if (h >= G) break;  // uniform over the CTA
     float m = s[h];
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -164,6 +168,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   __syncthreads();
 #pragma unroll
   for (int h = 0; h < HL; ++h) {
+    if (h >= G) break;  // uniform over the CTA
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) l[h] += __shfl_xor_sync(0xffffffffu, l[h], o);
     if (lane == 0) mxs[warp * HL + h] = l[h];
@@ -176,10 +181,10 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
   const int rix = p.n_splits + fs;
   const int c = tid & 15, grp = tid >> 4;
   constexpr int NGRP = DNT / 16;
-  for (int hb = 0; hb < G; hb += 4) {
-    float2 acc[4][4];  // dims 2e, 2e + 1 of the chunk, per head of the block
+  for (int hb = 0; hb < G; hb += NJ) {
+    float2 acc[NJ][4];  // dims 2e, 2e + 1 of the chunk, per head of the block
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NJ; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[j][e] = make_float2(0.0f, 0.0f);
 #pragma unroll 4  // independent row loads in flight
@@ -187,7 +192,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
       float2 x[4];
       bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < NJ; ++j) {
         if (hb + j < G) {
           const float pv = sc[rr * HL + hb + j];
           const float2 pv2 = make_float2(pv, pv);
@@ -197,7 +202,7 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
       }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j)
+    for (int j = 0; j < NJ; ++j)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         acc[j][e].x += __shfl_xor_sync(0xffffffffu, acc[j][e].x, 16);
@@ -206,13 +211,13 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
     if (lane < 16) {
       float4* dst = reinterpret_cast<float4*>(red + (warp * 16 + lane) * 32);
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < NJ; ++j) {
         dst[2 * j] = make_float4(acc[j][0].x, acc[j][0].y, acc[j][1].x, acc[j][1].y);
         dst[2 * j + 1] = make_float4(acc[j][2].x, acc[j][2].y, acc[j][3].x, acc[j][3].y);
       }
     }
     __syncthreads();
-    const int nh = min(4, G - hb);
+    const int nh = min(NJ, G - hb);
     for (int o = tid; o < 16 * nh * 8; o += DNT) {
       const int c2 = o / (nh * 8), j = (o / 8) % nh, e = o % 8;
       float v = 0.0f;
@@ -231,6 +236,15 @@ __device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float*
     rec[0] = mh[tid];
     rec[1] = ls;
   }
+}
+
+__device__ __forceinline__ void decode_sink_recent(const DecodeParams& p, float* sm, int fid) {
+  if (p.G == 1)
+    decode_sink_recent_t<1>(p, sm, fid);
+  else if (p.G == 2)
+    decode_sink_recent_t<2>(p, sm, fid);
+  else
+    decode_sink_recent_t<4>(p, sm, fid);
 }
 
 __host__ __device__ constexpr size_t sink_recent_smem_bytes() {
