@@ -93,10 +93,13 @@ __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, floa
   }
   __syncthreads();
   // scores: warp-cooperative, two rows per load instruction (lanes 0-15 and 16-31, one
-  // 16-byte chunk each) and several row pairs in flight; each lane keeps its chunk of q for
-  // up to 4 query heads in registers, and a 16-lane shuffle sum gives each row's score,
-  // written to sc[row][head]
+  // 16-byte chunk each); each lane keeps its chunk of q for up to 4 query heads in
+  // registers. A warp takes U = 16 / NJ row pairs at a time (all loads in flight), so each
+  // lane holds 16 partial dot products (row pair u, head j); one reduce-scatter over the 16
+  // lanes of each half-warp (15 shuffles) leaves lane c with the score of partial c, which
+  // it writes to sc[row][head].
   {
+    constexpr int U = 16 / NJ;
     const int ch = lane & 15, half = lane >> 4;
     const int npair = (nr + 1) >> 1;
     for (int hb = 0; hb < G; hb += NJ) {
@@ -108,30 +111,42 @@ __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, floa
           qr[j][e] = (hb + j < G)
                          ? *reinterpret_cast<const float2*>(qs + (hb + j) * FA_HEAD_DIM + ch * 8 + 2 * e)
                          : make_float2(0.0f, 0.0f);
-#pragma unroll 4
-      for (int i = warp; i < npair; i += 8) {
-        const int row = 2 * i + half;
-        float2 x[4];
-        bf16x8_to_f32x2(row < nr ? *reinterpret_cast<const uint4*>(FKh + (long long)(r0 + row) * FA_HEAD_DIM + ch * 8)
-                                 : make_uint4(0, 0, 0, 0),
-                        x);
-        float part[NJ];
+      for (int i0 = warp; i0 < npair; i0 += 8 * U) {
+        uint4 xr[U];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) {
-          float2 a = make_float2(0.0f, 0.0f);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) a = __ffma2_rn(qr[j][e], x[e], a);
-          part[j] = a.x + a.y;
+        for (int u = 0; u < U; ++u) {
+          const int row = 2 * (i0 + 8 * u) + half;
+          xr[u] = row < nr ? *reinterpret_cast<const uint4*>(FKh + (long long)(r0 + row) * FA_HEAD_DIM + ch * 8)
+                           : make_uint4(0, 0, 0, 0);
         }
+        float v[16];
 #pragma unroll
-        for (int o = 1; o < 16; o <<= 1)
+        for (int u = 0; u < U; ++u) {
+          float2 x[4];
+          bf16x8_to_f32x2(xr[u], x);
 #pragma unroll
-          for (int j = 0; j < NJ; ++j) part[j] += __shfl_xor_sync(0xffffffffu, part[j], o);
-        if (ch == 0 && row < nr) {
+          for (int j = 0; j < NJ; ++j) {
+            float2 a = make_float2(0.0f, 0.0f);
 #pragma unroll
-          for (int j = 0; j < NJ; ++j)
-            if (hb + j < G) sc[row * HL + hb + j] = part[j];
+            for (int e = 0; e < 4; ++e) a = __ffma2_rn(qr[j][e], x[e], a);
+            v[u * NJ + j] = a.x + a.y;
+          }
         }
+        // reduce-scatter: at offset o the lanes with bit o set keep the upper half of the
+        // remaining partials, the others the lower half, each adding its partner's copy
+#pragma unroll
+        for (int o = 8; o >= 1; o >>= 1) {
+          const bool up = (ch & o) != 0;
+#pragma unroll
+          for (int t = 0; t < o; ++t) {
+            const float send = up ? v[t] : v[t + o];
+            const float keep = up ? v[t + o] : v[t];
+            v[t] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+          }
+        }
+        const int u = ch / NJ, j = ch - (ch / NJ) * NJ;
+        const int row = 2 * (i0 + 8 * u) + half;
+        if (row < nr && hb + j < G) sc[row * HL + hb + j] = v[0];
       }
     }
   }
