@@ -66,6 +66,8 @@ __device__ __forceinline__ void bf16x8_to_f32x2(const uint4 v, float2 (&x)[4]) {
 // prologue launch on the tensor-core and warp-MMA paths.
 // NJ: query heads per block of the score and value passes (1, 2 or 4: G for G < 4), so that
 // MHA and G = 2 plans do no arithmetic or shuffles for empty heads.
+static_assert(HL == 8 && DNT == FT, "sink / recent pass: 8 heads per score row, one thread per row");
+
 template <int NJ>
 __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, float* sm, int fid) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -151,9 +153,15 @@ __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, floa
     }
   }
   __syncthreads();
+  // row tid's scores (HL = 8 floats, two vector loads); absent rows and heads: -inf
   float s[HL];
-#pragma unroll
-  for (int h = 0; h < HL; ++h) s[h] = (tid < nr && h < G) ? sc[tid * HL + h] : 0.0f;
+  {
+    const float4 lo = tid < nr ? *reinterpret_cast<const float4*>(sc + tid * HL) : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float4 hi = (tid < nr && G > 4) ? *reinterpret_cast<const float4*>(sc + tid * HL + 4)
+                                          : make_float4(0.f, 0.f, 0.f, 0.f);
+    s[0] = lo.x; s[1] = lo.y; s[2] = lo.z; s[3] = lo.w;
+    s[4] = hi.x; s[5] = hi.y; s[6] = hi.z; s[7] = hi.w;
+  }
 #pragma unroll
   for (int h = 0; h < HL; ++h)
     if (tid >= nr || h >= G) s[h] = -INFINITY;
@@ -175,10 +183,10 @@ __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, floa
   __syncthreads();
   float l[HL];
 #pragma unroll
-  for (int h = 0; h < HL; ++h) {
-    const float pv = (h < G && tid < nr) ? exp2f(s[h] - mh[h]) : 0.0f;
-    sc[tid * HL + h] = pv;
-    l[h] = pv;
+  for (int h = 0; h < HL; ++h) l[h] = (h < G && tid < nr) ? exp2f(s[h] - mh[h]) : 0.0f;
+  if (tid < FT) {  // p of row tid (0 past the rows and heads), two vector stores
+    *reinterpret_cast<float4*>(sc + tid * HL) = make_float4(l[0], l[1], l[2], l[3]);
+    *reinterpret_cast<float4*>(sc + tid * HL + 4) = make_float4(l[4], l[5], l[6], l[7]);
   }
   __syncthreads();
 #pragma unroll
@@ -206,10 +214,26 @@ __device__ __forceinline__ void decode_sink_recent_t(const DecodeParams& p, floa
     for (int rr = grp; rr < nr; rr += NGRP) {
       float2 x[4];
       bf16x8_to_f32x2(*reinterpret_cast<const uint4*>(FVh + (long long)(r0 + rr) * FA_HEAD_DIM + c * 8), x);
+      // p of the block's heads for this row, one vector load (sc rows are HL = 8 floats,
+      // hb a multiple of NJ: aligned; heads past G hold 0)
+      float pj[NJ];
+      if constexpr (NJ == 4) {
+        const float4 t = *reinterpret_cast<const float4*>(sc + rr * HL + hb);
+        pj[0] = t.x;
+        pj[1] = t.y;
+        pj[2] = t.z;
+        pj[3] = t.w;
+      } else if constexpr (NJ == 2) {
+        const float2 t = *reinterpret_cast<const float2*>(sc + rr * HL + hb);
+        pj[0] = t.x;
+        pj[1] = t.y;
+      } else {
+        pj[0] = sc[rr * HL + hb];
+      }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
         if (hb + j < G) {
-          const float pv = sc[rr * HL + hb + j];
+          const float pv = pj[j];
           const float2 pv2 = make_float2(pv, pv);
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[j][e] = __ffma2_rn(pv2, x[e], acc[j][e]);
