@@ -39,7 +39,6 @@ constexpr int CK_B_BYTES = 4 * CK_B_BOX;     // 32 KB
 constexpr int CK_THREADS = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 pack + epilogue
 constexpr int CK_PACK_WARPS = 8;
 constexpr int CK_STAGE_LD = CK_BN + 4;       // fp32 staging row stride (bank-conflict free)
-constexpr int CK_PREFETCH = 8;               // stages of K / V rows prefetched into L2 ahead
 
 template <int KT>
 struct CkCfg {
@@ -146,22 +145,11 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
     // ---------------------------------------------------------------- TMA producer
     if (lane == 0) {
       const uint32_t tx = (uint32_t)(kt_n * CK_A_TILE + CK_B_BYTES);
-      // K / V rows of this head are contiguous (256 bytes per token): pull them into L2
-      // CK_PREFETCH stages ahead of their TMA loads so that those see L2, not DRAM, latency.
-      const char* k_rows = static_cast<const char*>(p.K) + (long long)head * p.L * (FA_HEAD_DIM * 2);
-      const char* v_rows = static_cast<const char*>(p.V) + (long long)head * p.L * (FA_HEAD_DIM * 2);
-      auto prefetch_stage = [&](int st) {
-        const int t = p.S + (st0 + st) * CK_BK;
-        const int n = min(CK_BK, p.L - t);
-        if (n > 0) {
-          prefetch_l2_bulk(k_rows + (long long)t * (FA_HEAD_DIM * 2), (uint32_t)n * (FA_HEAD_DIM * 2));
-          prefetch_l2_bulk(v_rows + (long long)t * (FA_HEAD_DIM * 2), (uint32_t)n * (FA_HEAD_DIM * 2));
-        }
-      };
-      for (int st = 0; st < CK_PREFETCH && st < nk; ++st) prefetch_stage(st);
+      // No L2 prefetch of the cache rows ahead of their TMA loads: with 128 or more CTAs in
+      // flight, prefetched lines left L2 before their loads came (B = 4: 2.95 GB read for
+      // 2.15 GB of rows and table, and slower), while the TMA loads alone read each row once.
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
-        if (it + CK_PREFETCH < nk) prefetch_stage(it + CK_PREFETCH);
         const int s = it % STAGES;
         const uint32_t use = (uint32_t)(it / STAGES);
         if (it >= STAGES &&
