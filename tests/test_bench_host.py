@@ -80,6 +80,18 @@ def test_launches_per_step_each_path():
     assert bench.launches_per_step(w0, _plan(w0)) == 4
 
 
+def test_cluster_decode_needs_three_quarter_full_head_sets():
+    """The cluster kernel serves sets of 128 query heads at about the same cost however many
+    are valid, so plans whose sets are less than three quarters full take the warp-MMA kernel:
+    32 and 64 query heads (k = 511 and 1023, G = 4) go to warp MMA, 96 and 128 to the cluster
+    kernel, 160 (1.25 sets) to warp MMA, 192 (1.5 sets) to the cluster kernel."""
+    for base, cluster in ((wl.LLAMA3_8B_GQA_32K, 2), (wl.LLAMA3_8B_GQA_128K, 4)):
+        for B, kind in ((1, 3), (2, 3), (3, 4), (4, 4), (5, 3), (6, 4)):
+            info = fa.fa_decode_describe(_plan(wl.shrink(base, B=B)), 1)
+            assert info.split_kernel == kind, (base.name, B, info.split_kernel)
+            assert info.cluster == (cluster if kind == 4 else 1)
+
+
 def test_append_bytes_by_hand():
     w = wl.shrink(wl.LLAMA2_7B_MHA_32K, B=2, Hkv=4, Hq=4, L=5000)
     mask = np.zeros((4, 128), dtype=np.uint8)
