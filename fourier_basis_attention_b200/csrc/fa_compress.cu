@@ -36,18 +36,24 @@ constexpr int CK_BN = 2 * FA_HEAD_DIM;       // K dims | V dims (MMA N)
 constexpr int CK_A_TILE = CK_BM * CK_BK * 2; // 16 KB per coefficient tile
 constexpr int CK_B_BOX = 64 * CK_BK * 2;     // 8 KB per 64-dim box
 constexpr int CK_B_BYTES = 4 * CK_B_BOX;     // 32 KB
-constexpr int CK_THREADS = 320;               // warp 0 TMA, warp 1 MMA, warps 2-9 pack + epilogue
+constexpr int CK_THREADS = 352;  // warp 0 TMA (cache rows), warp 1 MMA, warps 2-9 pack +
+                                  // epilogue, warp 10 TMA (table tiles)
+constexpr int CK_A_WARP = 10;
 constexpr int CK_PACK_WARPS = 8;
 constexpr int CK_STAGE_LD = CK_BN + 4;       // fp32 staging row stride (bank-conflict free)
 
+// Two rings of stages: the table tiles (A, read from L2) and the cache rows (B, the DRAM
+// stream, one stage deeper so that more of it is in flight), each with its own producer.
 template <int KT>
 struct CkCfg {
   static constexpr int A_BYTES = KT * CK_A_TILE;
-  static constexpr int STAGE_BYTES = A_BYTES + CK_B_BYTES;
-  static constexpr int STAGES = KT == 2 ? 3 : 4;
+  static constexpr int A_STAGES = KT == 2 ? 3 : 4;
+  static constexpr int B_STAGES = KT == 2 ? 4 : 5;
+  static constexpr int RING_BYTES = A_STAGES * A_BYTES + B_STAGES * CK_B_BYTES;
   static constexpr int TMEM_COLS = KT * CK_BN;
-  static constexpr int BASE_SMEM = STAGES * STAGE_BYTES + 1024 /*align*/ + 1024 /*misc*/;
-  static_assert(CK_BM * CK_STAGE_LD * 4 <= STAGES * STAGE_BYTES, "staging fits");
+  static constexpr int BASE_SMEM = RING_BYTES + 1024 /*align*/ + 1024 /*misc*/;
+  static_assert(CK_BM * CK_STAGE_LD * 4 <= RING_BYTES, "staging fits");
+  static_assert(BASE_SMEM <= 227 * 1024, "fits in one SM's shared memory");
 };
 
 
@@ -82,15 +88,19 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CompressParams p) {
   using Cfg = CkCfg<KT>;
-  constexpr int STAGES = Cfg::STAGES;
+  constexpr int SA = Cfg::A_STAGES, SB = Cfg::B_STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* stages = smem;
-  uint8_t* misc = smem + STAGES * Cfg::STAGE_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(misc);
-  uint64_t* empty = full + STAGES;
-  uint64_t* accum = empty + STAGES;
+  uint8_t* stages = smem;                      // both rings (the epilogue's staging reuses them)
+  uint8_t* aring = smem;                       // [SA][A_BYTES] table tiles
+  uint8_t* bring = smem + SA * Cfg::A_BYTES;   // [SB][CK_B_BYTES] cache rows
+  uint8_t* misc = smem + Cfg::RING_BYTES;
+  uint64_t* fullA = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* emptyA = fullA + SA;
+  uint64_t* fullB = emptyA + SA;
+  uint64_t* emptyB = fullB + SB;
+  uint64_t* accum = emptyB + SB;
   uint64_t* drain = accum + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -119,9 +129,13 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   if (dc == 0 && pair != 0) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + (do_pack ? CK_PACK_WARPS : 0));
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(&fullA[s], 1);
+      mbar_init(&emptyA[s], 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(&fullB[s], 1);
+      mbar_init(&emptyB[s], 1 + (do_pack ? CK_PACK_WARPS : 0));
     }
     mbar_init(accum, 1);
     mbar_init(drain, 1);
@@ -141,42 +155,48 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_d = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- TMA producer
+  if (warp == 0 || warp == CK_A_WARP) {
+    // ---------------------------------------------------------------- TMA producers
+    // warp 0: the cache rows (ring B); warp CK_A_WARP: the table tiles (ring A). No L2
+    // prefetch of the rows ahead of their loads: with 128 or more CTAs in flight, prefetched
+    // lines left L2 before their loads came (B = 4: 2.95 GB read for 2.15 GB of rows and
+    // table, and slower), while the TMA loads alone read each row once.
     if (lane == 0) {
-      const uint32_t tx = (uint32_t)(kt_n * CK_A_TILE + CK_B_BYTES);
-      // No L2 prefetch of the cache rows ahead of their TMA loads: with 128 or more CTAs in
-      // flight, prefetched lines left L2 before their loads came (B = 4: 2.95 GB read for
-      // 2.15 GB of rows and table, and slower), while the TMA loads alone read each row once.
+      const bool is_b = warp == 0;
+      const int NS = is_b ? SB : SA;
+      uint64_t* fl = is_b ? fullB : fullA;
+      uint64_t* em = is_b ? emptyB : emptyA;
+      const uint32_t tx = is_b ? (uint32_t)CK_B_BYTES : (uint32_t)(kt_n * CK_A_TILE);
       int issued = 0;
       for (int it = 0; it < nk; ++it) {
-        const int s = it % STAGES;
-        const uint32_t use = (uint32_t)(it / STAGES);
-        if (it >= STAGES &&
-            !mbar_wait(&empty[s], (use & 1u) ^ 1u, abort_flag, WD_COMPRESS | 1u))
+        const int s = it % NS;
+        const uint32_t use = (uint32_t)(it / NS);
+        if (it >= NS && !mbar_wait(&em[s], (use & 1u) ^ 1u, abort_flag, WD_COMPRESS | 1u))
           break;
-        uint8_t* a_s = stages + s * Cfg::STAGE_BYTES;
-        uint8_t* b_s = a_s + Cfg::A_BYTES;
-        const int t = p.S + (st0 + it) * CK_BK;
-        mbar_arrive_expect_tx(&full[s], tx);
-        for (int kt = 0; kt < kt_n; ++kt)
-          tma_load_2d(a_s + kt * CK_A_TILE, &tm_phi, &full[s], (st0 + it) * CK_BK,
-                      (kt0 + kt) * CK_BM);
-        tma_load_3d(b_s, &tm_k, &full[s], 0, t, head);
-        tma_load_3d(b_s + CK_B_BOX, &tm_k, &full[s], 64, t, head);
-        tma_load_3d(b_s + 2 * CK_B_BOX, &tm_v, &full[s], 0, t, head);
-        tma_load_3d(b_s + 3 * CK_B_BOX, &tm_v, &full[s], 64, t, head);
+        mbar_arrive_expect_tx(&fl[s], tx);
+        if (is_b) {
+          uint8_t* b_s = bring + s * CK_B_BYTES;
+          const int t = p.S + (st0 + it) * CK_BK;
+          tma_load_3d(b_s, &tm_k, &fl[s], 0, t, head);
+          tma_load_3d(b_s + CK_B_BOX, &tm_k, &fl[s], 64, t, head);
+          tma_load_3d(b_s + 2 * CK_B_BOX, &tm_v, &fl[s], 0, t, head);
+          tma_load_3d(b_s + 3 * CK_B_BOX, &tm_v, &fl[s], 64, t, head);
+        } else {
+          uint8_t* a_s = aring + s * Cfg::A_BYTES;
+          for (int kt = 0; kt < kt_n; ++kt)
+            tma_load_2d(a_s + kt * CK_A_TILE, &tm_phi, &fl[s], (st0 + it) * CK_BK,
+                        (kt0 + kt) * CK_BM);
+        }
         ++issued;
       }
       if (*abort_flag) {
         // let the copies already issued land before shared memory goes away
-        for (int it = (issued > STAGES ? issued - STAGES : 0); it < issued; ++it)
-          drain_wait(&full[it % STAGES], (uint32_t)(it / STAGES) & 1u);
+        for (int it = (issued > NS ? issued - NS : 0); it < issued; ++it)
+          drain_wait(&fl[it % NS], (uint32_t)(it / NS) & 1u);
       } else {
-        // tail: every stage's last release (MMA commit + pack arrivals) has landed
-        for (int it = (nk > STAGES ? nk - STAGES : 0); it < nk; ++it)
-          mbar_wait(&empty[it % STAGES], (uint32_t)(it / STAGES) & 1u, abort_flag,
-                    WD_COMPRESS | 5u);
+        // tail: every stage's last release (MMA commit, and pack arrivals on ring B) landed
+        for (int it = (nk > NS ? nk - NS : 0); it < nk; ++it)
+          mbar_wait(&em[it % NS], (uint32_t)(it / NS) & 1u, abort_flag, WD_COMPRESS | 5u);
       }
     }
   } else if (warp == 1) {
@@ -185,14 +205,15 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       constexpr uint32_t idesc = idesc_bf16_f32(CK_BM, CK_BN, /*b_mn_major=*/true);
       bool ok = true;
       for (int it = 0; it < nk; ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&full[s], (uint32_t)(it / STAGES) & 1u, abort_flag, WD_COMPRESS | 2u)) {
+        const int sa = it % SA, sb = it % SB;
+        if (!mbar_wait(&fullA[sa], (uint32_t)(it / SA) & 1u, abort_flag, WD_COMPRESS | 2u) ||
+            !mbar_wait(&fullB[sb], (uint32_t)(it / SB) & 1u, abort_flag, WD_COMPRESS | 7u)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(stages + s * Cfg::STAGE_BYTES);
-        const uint32_t b_addr = a_addr + Cfg::A_BYTES;
+        const uint32_t a_addr = smem_u32(aring + sa * Cfg::A_BYTES);
+        const uint32_t b_addr = smem_u32(bring + sb * CK_B_BYTES);
 #pragma unroll
         for (int kk = 0; kk < CK_BK / 16; ++kk) {
           // B: 16 tokens = two 8-row groups of 128-byte rows; the four 64-dim boxes are
@@ -207,7 +228,8 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
             }
           }
         }
-        mma_commit(&empty[s]);
+        mma_commit(&emptyA[sa]);
+        mma_commit(&emptyB[sb]);
       }
       if (ok) {
         mma_commit(accum);
@@ -237,10 +259,10 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
       __nv_bfloat16* const E1 = p.E[1] + (long long)b * p.e_batch + p.e_off[g];
       constexpr int TPW = CK_BK / CK_PACK_WARPS;  // tokens per warp per stage
       for (int it = 0; it < nk; ++it) {
-        const int s = it % STAGES;
-        if (!mbar_wait(&full[s], (uint32_t)(it / STAGES) & 1u, abort_flag, WD_COMPRESS | 3u))
+        const int s = it % SB;
+        if (!mbar_wait(&fullB[s], (uint32_t)(it / SB) & 1u, abort_flag, WD_COMPRESS | 3u))
           break;
-        const uint8_t* b_s = stages + s * Cfg::STAGE_BYTES + Cfg::A_BYTES;
+        const uint8_t* b_s = bring + s * CK_B_BYTES;
         const int ntok = min(CK_BK, p.M - (st0 + it) * CK_BK);
         for (int c = 0; c < ngrp; ++c) {
           const int i = lane + 32 * c;
@@ -266,7 +288,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
             // warp's loads before the arrival): the stage may be refilled while the rows
             // are stored
             __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (lane == 0) mbar_arrive(&emptyB[s]);
           }
           if (i < de_ld) {
 #pragma unroll
@@ -283,7 +305,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
         }
         if (ngrp == 0) {  // nothing retained: only the release
           __syncwarp();
-          if (lane == 0) mbar_arrive(&empty[s]);
+          if (lane == 0) mbar_arrive(&emptyB[s]);
         }
       }
     }
@@ -366,7 +388,7 @@ __global__ void __launch_bounds__(CK_THREADS, 1)
     for (int r = 0; r < 16; ++r)
       peer[r] = r < p.nsplit ? mapa_shared(smem_u32(stage_f), (uint32_t)r) : 0u;
     for (int kt = 0; kt < kt_n; ++kt) {
-      if (warp >= 2 && acc_ok) {
+      if (warp >= 2 && warp < 2 + CK_PACK_WARPS && acc_ok) {  // the pack / epilogue warps
         tc_fence_after();
         const int rb = warp & 3;
         const int half = (warp - 2) >> 2;
